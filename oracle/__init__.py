@@ -1,0 +1,11 @@
+"""CPU oracle for the LAGS sparsify / aggregate / apply path.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference leg of ``bench.py`` may import this package.  The
+product path (``layer_wise_top_b200``) never imports it and has no CPU
+fallback.
+"""
+from .lags_oracle import (  # noqa: F401
+    aggregate, aggregate_layer, apply_update, error_feedback, k_of, layer_plan,
+    magnitude_order, run_workload, select_layer, sparsify, sparsify_layer,
+)
