@@ -1,0 +1,357 @@
+#!/usr/bin/env python
+"""Throughput of the LAGS sparsify + aggregate step on B200.
+
+One step = error feedback + layer-wise exact top-k for all P simulated workers
+(lags_sparsify), the deterministic sparse aggregation (lags_aggregate) and the
+weight update (lags_apply), over one batch of synthetic gradients already in
+HBM.  value = P*N elements per step / step time, in Gelem/s; under torchrun
+each rank runs its own replica (no collective on the data path) and value sums
+the elements of all ranks over the slowest rank's time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config vgg16]
+    python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "LAGS sparsify+aggregate Gelem/s per step; achieved HBM GB/s vs peak"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+POOL_BUDGET_BYTES = 48 * 1024 ** 3
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="vgg16",
+                    choices=["resnet20", "vgg16", "resnet50", "lstm_ptb", "gpt_1_3b"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_config(w, **extra):
+    dens = sorted(set(w.densities))
+    cfg = {"workload": w.name, "P": w.P, "N": w.N, "layers": w.L, "elements_per_step": w.P * w.N,
+           "densities": dens if len(dens) > 1 else dens[0], "lr": w.lr,
+           "grad_dist": "normal(0,1/fan_in)" if w.dist == 0 else "student_t3/sqrt(fan_in)"}
+    cfg.update(extra)
+    return cfg
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------- reference arm
+def oracle_sample_layers(w, budget_elems):
+    """Consecutive layers of one worker, from the first, up to ~budget elements."""
+    layers, total = [], 0
+    for l, d in enumerate(w.sizes):
+        if layers and total + d > budget_elems:
+            break
+        layers.append(l)
+        total += d
+    return layers, total
+
+
+def time_oracle(w, worker, step, layers):
+    """Oracle sparsify + aggregate of one worker's sampled layers (zero
+    residual, worker `worker`, step `step`); returns seconds and elements."""
+    import numpy as np
+    import oracle.lags_oracle as lo
+    import synth
+    grads = {l: synth.layer_grads_host(w, worker, step, l) for l in layers}
+    t0 = time.perf_counter()
+    elems = 0
+    for l in layers:
+        d = w.sizes[l]
+        k = lo.k_of(d, w.densities[l])
+        off = w.offsets[l]
+        idx, val, _ = lo.sparsify_layer(off, k, [grads[l]], [np.zeros(d, np.float32)], w.lr)
+        lo.aggregate_layer(off, d, idx, val)
+        elems += d
+    return time.perf_counter() - t0, elems
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from synth.configs import WORKLOADS
+    w = WORKLOADS[args.config]
+    layers, total = oracle_sample_layers(w, 4_000_000)
+    sample = (f"one worker per step (worker = step mod P), layers {layers[0]}..{layers[-1]} "
+              f"({total} elements), zero residual; numpy oracle, single thread")
+    for s in range(args.warmup):
+        time_oracle(w, s % w.P, s, layers)
+    secs, elems = 0.0, 0
+    for s in range(args.steps):
+        t, e = time_oracle(w, (args.warmup + s) % w.P, args.warmup + s, layers)
+        secs += t
+        elems += e
+    value = elems / secs / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Gelem/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w, sample_elements_per_step=total),
+        "cpu_baseline": {"kind": "oracle", "value": value, "unit": "Gelem/s", "cores": 1,
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------- our arm
+def cpu_baseline(w):
+    layers, total = oracle_sample_layers(w, 8_000_000)
+    secs, elems, step = 0.0, 0, 0
+    while secs < 10.0 and step < 8:
+        t, e = time_oracle(w, step % w.P, step, layers)
+        secs += t
+        elems += e
+        step += 1
+    return {"value": elems / secs / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+            "sample": (f"{step} x one worker's layers {layers[0]}..{layers[-1]} ({total} "
+                       f"elements, zero residual), sparsify+aggregate, numpy single thread "
+                       f"on {os.cpu_count()} host cores"),
+            "seconds": secs}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import synth
+    from layer_wise_top_b200 import Plan
+    from synth.configs import WORKLOADS
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    w = WORKLOADS[args.config]
+    P, N = w.P, w.N
+    plan = Plan(w.sizes, w.densities, P, device=dev)
+    step_bytes = P * N * 4
+    pool = max(1, min(args.warmup + args.steps, POOL_BUDGET_BYTES // step_bytes))
+    grads = []
+    for s in range(pool):
+        bufs = [torch.empty(N, dtype=torch.float32, device=dev) for _ in range(P)]
+        for p in range(P):
+            synth.worker_grads_device(w, p, s + 1000 * rank, bufs[p])
+        grads.append(bufs)
+    res = [torch.zeros(N, dtype=torch.float32, device=dev) for _ in range(P)]
+    idx, val = plan.empty_picks()
+    dense = torch.empty(N, dtype=torch.float32, device=dev)
+    weights = torch.zeros(N, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+
+    n_sparse = sum(1 for l, d in enumerate(w.sizes) if plan.layers[l][1] < d)
+    n_large = sum(1 for l, d in enumerate(w.sizes) if plan.layers[l][1] < d and d >= (1 << 20))
+    launches_per_step = (1 if n_sparse else 0) + 1 + (1 if n_sparse - n_large else 0) + \
+        (1 if n_large else 0) + 3
+
+    def step(i):
+        plan.sparsify(grads[i % pool], res, w.lr, idx, val)
+        plan.aggregate(idx, val, dense)
+        plan.apply(weights, dense)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    flags, fallbacks = plan.poll()
+
+    K = args.steps
+    ev_k1 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(K)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t0.record()
+    for i in range(K):
+        plan.set_events(*ev_k1[i])
+        step(args.warmup + i)
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    plan.set_events(None, None)
+    ms = t0.elapsed_time(t1)
+    k1_ms = [a.elapsed_time(b) for a, b in ev_k1]
+    flags2, fallbacks2 = plan.poll()
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    # end to end through the same calls: inputs from pinned host memory each
+    # step, the updated weights read back each step
+    e2e = None
+    if not args.no_e2e:
+        host = [torch.empty(N, dtype=torch.float32, pin_memory=True) for _ in range(P)]
+        for p in range(P):
+            host[p].copy_(grads[0][p])
+        w_host = torch.empty(N, dtype=torch.float32, pin_memory=True)
+        dev_g = grads[0]
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        ke = max(3, min(K, 10))
+        barrier()
+        torch.cuda.synchronize()
+        e0.record()
+        for i in range(ke):
+            for p in range(P):
+                dev_g[p].copy_(host[p], non_blocking=True)
+            plan.sparsify(dev_g, res, w.lr, idx, val)
+            plan.aggregate(idx, val, dense)
+            plan.apply(weights, dense)
+            w_host.copy_(weights, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * P * N * ke / (float(e_ms.item()) / 1e3) / 1e9,
+               "unit": "Gelem/s", "steps": ke, "h2d_bytes_per_step": P * N * 4,
+               "d2h_bytes_per_step": N * 4}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peak, peak_kind = measured_peak()
+    k1_avg = sum(k1_ms) / len(k1_ms)
+    k1_bytes = 12 * P * N
+    achieved = k1_bytes / (k1_avg / 1e3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": world * P * N * K / (ms_max / 1e3) / 1e9,
+        "unit": "Gelem/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_max / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic: Philox4x32-10 gradients with the workload's tensor shapes",
+        "config": workload_config(
+            w, parallelism=f"replicas x{world}", grad_pool_steps=pool,
+            l2=f"inputs larger than L2: {12 * P * N / 1e9:.2f} GB streamed per step vs "
+               f"{L2_BYTES / 1e6:.0f} MB L2",
+            step="lags_sparsify + lags_aggregate + lags_apply"),
+        "roofline": {"kernel": "k_ef_capture", "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes_per_launch": k1_bytes, "avg_launch_ms": k1_avg,
+                     "share_of_step": k1_avg / (ms_max / K)},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk,
+        "status": {"flags": flags | flags2, "exact_fallback_segments": fallbacks + fallbacks2},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,190 @@
+/*
+ * lags.h - C ABI of the B200 LAGS sparsification library (liblags.so).
+ *
+ * The operation is the data-parallel hot path of LAGS-SGD, as described by
+ * "Layer-wise Adaptive Gradient Sparsification for Distributed Deep Learning
+ * with Convergence Guarantees" (nubint.ai review; abstract and section
+ * "proposed method"): every worker, for every layer independently, adds its
+ * error-compensation residual to the scaled gradient, keeps the k entries of
+ * largest magnitude of that layer, sends them as (index, value) pairs and
+ * keeps the remainder as its next residual; the workers' sparse sets are then
+ * summed into the averaged dense update of sparsified synchronous SGD, which
+ * is applied to the weights.
+ *
+ * Exact arithmetic (the pages give no formula; these are the readings the
+ * library implements and tests bit for bit against its CPU oracle):
+ *   acc_i      = fl32(residual_i + fl32(lr * grad_i))         (two roundings)
+ *   k_l        = min(d_l, max(1, ceil(fl64(rho_l * d_l))))   (rho_l a double)
+ *   selection  = the k_l largest |acc| of the layer; equal magnitudes are
+ *                ordered by the lower index; +0 and -0 tie; +-inf are largest
+ *   picks      = (global index, acc) of the selected entries, ascending index
+ *   residual_i = +0.0f where picked, acc_i elsewhere
+ *   dense_j    = fl32( (((+0 + v_0j) + v_1j) + ... + v_(P-1)j) / P ), workers
+ *                in order 0..P-1, absent picks contributing nothing
+ *   weights_j  = fl32(weights_j - dense_j)
+ * NaN inputs are not supported (a NaN magnitude orders above +inf).
+ *
+ * Conventions shared by every call:
+ *   - "device" pointers are CUDA device memory of the current device; "host"
+ *     pointers are ordinary host memory read during the call only.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every compute call only enqueues work on that stream: it never
+ *     allocates, never synchronises and returns before the work runs.  Work on
+ *     one plan must be issued in stream order (one stream, or events).
+ *   - Argument errors are reported by the return value before anything is
+ *     enqueued.  Errors a kernel detects are recorded in the plan's device
+ *     status word and read with lags_status_poll().
+ *   - The library owns only the plan's host-side tables.  All device memory
+ *     (inputs, outputs and the plan workspace) belongs to the caller.
+ */
+#ifndef LAGS_H
+#define LAGS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LAGS_API __attribute__((visibility("default")))
+#else
+#define LAGS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct lags_plan lags_plan; /* opaque; created and destroyed by the caller */
+
+typedef enum {
+  LAGS_OK = 0,
+  LAGS_ERR_INVALID_ARG = 1,        /* null pointer, size or count out of range */
+  LAGS_ERR_ALIGNMENT = 2,          /* a device pointer is not aligned as required */
+  LAGS_ERR_CUDA = 3,               /* a CUDA runtime call or launch failed */
+  LAGS_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not sm_100 (B200) */
+  LAGS_ERR_WORKSPACE = 5,          /* workspace missing or smaller than required */
+  LAGS_ERR_BAD_PICKS = 6           /* (status word) pick lists not ascending/in layer */
+} lags_status;
+
+/* Largest number of simulated workers one plan accepts. */
+#define LAGS_MAX_WORKERS 256
+
+/* Bits of the device status word returned by lags_status_poll(). */
+#define LAGS_FLAG_BAD_PICKS 0x1u /* lags_aggregate saw an unsorted or out-of-layer index */
+#define LAGS_FLAG_INTERNAL 0x2u  /* a selection kernel failed a self-check (a library bug);
+                                    the write it guarded was skipped */
+
+/*
+ * lags_plan_create - describe one flattened gradient buffer.
+ *   layer_sizes  host, [num_layers] int64: d_l > 0, layers stored back to back
+ *                in this order; N = sum d_l must be < 2^32.
+ *   densities    host, [num_layers] double: rho_l in (0, 1]; k_l follows the
+ *                rule above (rho_l = 1 or k_l = d_l sends the layer densely).
+ *   num_workers  P, 1 <= P <= LAGS_MAX_WORKERS.
+ *   out_plan     host, receives the plan.
+ * Host only: computes k_l, the layer and tile tables and the workspace size.
+ * Returns LAGS_ERR_INVALID_ARG on any bad argument (nothing is created).
+ */
+LAGS_API lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities,
+                             int32_t num_layers, int32_t num_workers, lags_plan** out_plan);
+
+/* Frees the host tables.  The workspace stays the caller's. */
+LAGS_API lags_status lags_plan_destroy(lags_plan* plan);
+
+/*
+ * lags_plan_info - sizes of the plan (any output pointer may be NULL).
+ *   N                elements per worker buffer
+ *   K                picks per worker (sum of k_l); out_idx/out_val are [P][K]
+ *   workspace_bytes  device bytes lags_plan_set_workspace() needs
+ */
+LAGS_API lags_status lags_plan_info(const lags_plan* plan, int64_t* N, int64_t* K,
+                           size_t* workspace_bytes);
+
+/*
+ * lags_plan_layer - placement of layer l: its first element in a worker buffer
+ * (offset), its pick count k_l and the first slot of its picks in a worker's
+ * pick list (pick_offset).  Picks of layer l occupy
+ * out[p*K + pick_offset .. p*K + pick_offset + k_l).
+ */
+LAGS_API lags_status lags_plan_layer(const lags_plan* plan, int32_t l, int64_t* offset, int64_t* k,
+                            int64_t* pick_offset);
+
+/*
+ * lags_plan_set_workspace - bind caller-owned device memory to the plan and
+ * upload the plan's tables into it (enqueued on `stream`; the host tables are
+ * owned by the plan, so nothing has to outlive the call on the caller side).
+ *   workspace  device, 256-byte aligned, >= workspace_bytes of lags_plan_info.
+ * Also checks that the current device is an sm_100 part.  Call it again after
+ * freeing or moving the workspace.  Not for use inside stream capture.
+ */
+LAGS_API lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t bytes,
+                                    void* stream);
+
+/*
+ * lags_sparsify - error feedback and layer-wise top-k for all P workers.
+ *   grads      host array of P device pointers, each a float[N] gradient
+ *              buffer (16-byte aligned); read only.
+ *   residuals  host array of P device pointers, each a float[N] residual
+ *              buffer (16-byte aligned); read, then overwritten with the new
+ *              residual.  Buffers of different workers must not overlap.
+ *   lr         learning rate (fp32).
+ *   out_idx    device uint32[P*K] (4-byte aligned): worker p's picks at
+ *              [p*K, (p+1)*K), layer by layer, ascending global index.
+ *   out_val    device float[P*K]: acc at those indices.
+ * The pointer arrays are copied into the launch arguments, so they need not
+ * outlive the call.  Enqueues a few kernels on `stream`.
+ */
+LAGS_API lags_status lags_sparsify(lags_plan* plan, const float* const* grads, float* const* residuals,
+                          float lr, uint32_t* out_idx, float* out_val, void* stream);
+
+/*
+ * lags_aggregate - dense averaged update from P workers' pick lists.
+ *   idx, val   device [P*K] in the layout lags_sparsify writes (each layer's
+ *              indices ascending and inside the layer; otherwise the status
+ *              word gets LAGS_FLAG_BAD_PICKS and dense_out is unspecified).
+ *   dense_out  device float[N], 16-byte aligned; fully overwritten.
+ * Uses the plan workspace; order it after lags_sparsify on the same stream
+ * when it consumes that call's output.
+ */
+LAGS_API lags_status lags_aggregate(lags_plan* plan, const uint32_t* idx, const float* val,
+                           float* dense_out, void* stream);
+
+/*
+ * lags_apply - weights <- weights - dense_out over the plan's N elements.
+ *   weights    device float[N], 16-byte aligned, updated in place.
+ *   dense_out  device float[N], 16-byte aligned.
+ */
+LAGS_API lags_status lags_apply(const lags_plan* plan, float* weights, const float* dense_out,
+                       void* stream);
+
+/*
+ * lags_status_poll - synchronise `stream`, read and clear the plan's device
+ * status word.
+ *   flags              host, receives LAGS_FLAG_* bits (may be NULL)
+ *   exact_fallbacks    host, receives how many (worker, layer) segments since
+ *                      the last poll were selected by the exhaustive path
+ *                      because the sampled candidate threshold did not hold
+ *                      (results are exact either way; may be NULL)
+ * Returns LAGS_ERR_BAD_PICKS if that flag was set, else LAGS_OK (or
+ * LAGS_ERR_CUDA).
+ */
+LAGS_API lags_status lags_status_poll(lags_plan* plan, uint32_t* flags, uint32_t* exact_fallbacks,
+                             void* stream);
+
+/*
+ * lags_plan_set_events - timing instrumentation.  When `before` and `after`
+ * (cudaEvent_t passed as void*, created by the caller) are both non-NULL, each
+ * later lags_sparsify on this plan records `before` on its stream just before
+ * it launches the fused error-feedback pass and `after` just after it, so
+ * cudaEventElapsedTime(before, after) is that kernel's device time.  Pass
+ * NULL, NULL to stop.  The events stay the caller's.
+ */
+LAGS_API lags_status lags_plan_set_events(lags_plan* plan, void* before, void* after);
+
+/* Static, human-readable text for a status code. */
+LAGS_API const char* lags_error_string(lags_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LAGS_H */

@@ -1,0 +1,21 @@
+"""B200-native LAGS sparsification: error feedback, layer-wise exact top-k,
+deterministic sparse aggregation and the SGD update, as hand-written sm_100a
+CUDA kernels behind the C ABI in include/lags.h.
+
+Importing the package loads liblags.so and fails if it is missing; there is no
+CPU fallback.
+"""
+from ._binding import (  # noqa: F401
+    EXPORTED, LAGS_ERR_ALIGNMENT, LAGS_ERR_BAD_PICKS, LAGS_ERR_CUDA, LAGS_ERR_INVALID_ARG,
+    LAGS_ERR_UNSUPPORTED_DEVICE, LAGS_ERR_WORKSPACE, LAGS_FLAG_BAD_PICKS, LAGS_MAX_WORKERS,
+    LAGS_OK, LIB_PATH, LagsError, lags_aggregate, lags_apply, lags_error_string,
+    lags_plan_create, lags_plan_destroy, lags_plan_info, lags_plan_layer,
+    lags_plan_set_events, lags_plan_set_workspace, lags_sparsify, lags_status_poll, library,
+)
+
+
+def __getattr__(name):
+    if name == "Plan":
+        from .plan import Plan
+        return Plan
+    raise AttributeError(name)

@@ -1,0 +1,146 @@
+"""ctypes binding of liblags.so: one Python function per C entry point, same
+names, argument marshalling only.  Every step of the computation runs in the
+library's CUDA kernels; there is no Python or CPU fallback, and importing this
+module fails if the library has not been built."""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Sequence, Tuple
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblags.so")
+
+LAGS_OK = 0
+LAGS_ERR_INVALID_ARG = 1
+LAGS_ERR_ALIGNMENT = 2
+LAGS_ERR_CUDA = 3
+LAGS_ERR_UNSUPPORTED_DEVICE = 4
+LAGS_ERR_WORKSPACE = 5
+LAGS_ERR_BAD_PICKS = 6
+LAGS_MAX_WORKERS = 256
+LAGS_FLAG_BAD_PICKS = 0x1
+LAGS_FLAG_INTERNAL = 0x2
+
+EXPORTED = ("lags_plan_create", "lags_plan_destroy", "lags_plan_info", "lags_plan_layer",
+            "lags_plan_set_workspace", "lags_sparsify", "lags_aggregate", "lags_apply",
+            "lags_status_poll", "lags_plan_set_events", "lags_error_string")
+
+
+class LagsError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lags_error_string(status)} (status {status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m layer_wise_top_b200.build` "
+            "(there is no fallback implementation)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64p = ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(ctypes.c_int64)
+    st = ctypes.c_int
+    lib.lags_plan_create.argtypes = [i64p, ctypes.POINTER(ctypes.c_double), i32, i32,
+                                     ctypes.POINTER(vp)]
+    lib.lags_plan_destroy.argtypes = [vp]
+    lib.lags_plan_info.argtypes = [vp, i64p, i64p, ctypes.POINTER(ctypes.c_size_t)]
+    lib.lags_plan_layer.argtypes = [vp, i32, i64p, i64p, i64p]
+    lib.lags_plan_set_workspace.argtypes = [vp, vp, ctypes.c_size_t, vp]
+    lib.lags_sparsify.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.c_float,
+                                  vp, vp, vp]
+    lib.lags_aggregate.argtypes = [vp, vp, vp, vp, vp]
+    lib.lags_apply.argtypes = [vp, vp, vp, vp]
+    lib.lags_status_poll.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32),
+                                     ctypes.POINTER(ctypes.c_uint32), vp]
+    lib.lags_plan_set_events.argtypes = [vp, vp, vp]
+    lib.lags_error_string.argtypes = [st]
+    lib.lags_error_string.restype = ctypes.c_char_p
+    for name in EXPORTED[:-1]:
+        getattr(lib, name).restype = st
+    return lib
+
+
+_LIB = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _LIB
+
+
+def _check(status: int, where: str) -> None:
+    if status != LAGS_OK:
+        raise LagsError(status, where)
+
+
+def lags_error_string(status: int) -> str:
+    return _LIB.lags_error_string(int(status)).decode()
+
+
+def lags_plan_create(layer_sizes: Sequence[int], densities: Sequence[float],
+                     num_workers: int) -> ctypes.c_void_p:
+    L = len(layer_sizes)
+    if len(densities) != L:
+        raise ValueError("layer_sizes and densities differ in length")
+    sizes = (ctypes.c_int64 * max(L, 1))(*[int(x) for x in layer_sizes])
+    dens = (ctypes.c_double * max(L, 1))(*[float(x) for x in densities])
+    out = ctypes.c_void_p()
+    _check(_LIB.lags_plan_create(sizes, dens, L, int(num_workers), ctypes.byref(out)),
+           "lags_plan_create")
+    return out
+
+
+def lags_plan_destroy(plan) -> None:
+    _check(_LIB.lags_plan_destroy(plan), "lags_plan_destroy")
+
+
+def lags_plan_info(plan) -> Tuple[int, int, int]:
+    n, k, ws = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_size_t()
+    _check(_LIB.lags_plan_info(plan, ctypes.byref(n), ctypes.byref(k), ctypes.byref(ws)),
+           "lags_plan_info")
+    return n.value, k.value, ws.value
+
+
+def lags_plan_layer(plan, l: int) -> Tuple[int, int, int]:
+    o, k, ko = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    _check(_LIB.lags_plan_layer(plan, int(l), ctypes.byref(o), ctypes.byref(k),
+                                ctypes.byref(ko)), "lags_plan_layer")
+    return o.value, k.value, ko.value
+
+
+def lags_plan_set_workspace(plan, workspace: int, nbytes: int, stream: int = 0) -> None:
+    _check(_LIB.lags_plan_set_workspace(plan, ctypes.c_void_p(workspace), int(nbytes),
+                                        ctypes.c_void_p(stream)), "lags_plan_set_workspace")
+
+
+def lags_sparsify(plan, grads: Sequence[int], residuals: Sequence[int], lr: float,
+                  out_idx: int, out_val: int, stream: int = 0) -> None:
+    P = len(grads)
+    g = (ctypes.c_void_p * max(P, 1))(*[ctypes.c_void_p(x) for x in grads])
+    r = (ctypes.c_void_p * max(len(residuals), 1))(*[ctypes.c_void_p(x) for x in residuals])
+    _check(_LIB.lags_sparsify(plan, g, r, ctypes.c_float(lr), ctypes.c_void_p(out_idx),
+                              ctypes.c_void_p(out_val), ctypes.c_void_p(stream)),
+           "lags_sparsify")
+
+
+def lags_aggregate(plan, idx: int, val: int, dense_out: int, stream: int = 0) -> None:
+    _check(_LIB.lags_aggregate(plan, ctypes.c_void_p(idx), ctypes.c_void_p(val),
+                               ctypes.c_void_p(dense_out), ctypes.c_void_p(stream)),
+           "lags_aggregate")
+
+
+def lags_apply(plan, weights: int, dense_out: int, stream: int = 0) -> None:
+    _check(_LIB.lags_apply(plan, ctypes.c_void_p(weights), ctypes.c_void_p(dense_out),
+                           ctypes.c_void_p(stream)), "lags_apply")
+
+
+def lags_plan_set_events(plan, before: int, after: int) -> None:
+    _check(_LIB.lags_plan_set_events(plan, ctypes.c_void_p(before), ctypes.c_void_p(after)),
+           "lags_plan_set_events")
+
+
+def lags_status_poll(plan, stream: int = 0) -> Tuple[int, int]:
+    """Returns (flags, exact_fallbacks); raises on LAGS_ERR_BAD_PICKS."""
+    f, fb = ctypes.c_uint32(), ctypes.c_uint32()
+    _check(_LIB.lags_status_poll(plan, ctypes.byref(f), ctypes.byref(fb),
+                                 ctypes.c_void_p(stream)), "lags_status_poll")
+    return f.value, fb.value

@@ -1,0 +1,166 @@
+// Fused error-feedback and candidate-capture pass (the streaming hot loop).
+//
+// One CTA per (tile, worker).  Each thread loads 8 float4 of the gradient and
+// 8 float4 of the residual with 128-bit coalesced loads, forms
+// acc = fl32(residual + fl32(lr * grad)) (error compensation, "Layer-wise
+// Adaptive Gradient Sparsification ..." review, "proposed method") and writes
+// acc back over the residual.  This is the only full pass over the data:
+// 12 bytes per element (read g, read r, write r).
+//
+//  - sparse layers: every entry whose magnitude key reaches the layer's
+//    sampled threshold lo_key is appended, in index order, to the tile's
+//    candidate slots (value, global index), and the tile's candidate count is
+//    recorded (counts above the slot capacity mark an overflow);
+//  - dense layers (k_l = d_l): every entry is a pick; it goes straight to the
+//    pick list and its residual becomes +0.
+#include "block_ops.cuh"
+#include "lags_internal.cuh"
+
+namespace lags {
+
+__device__ __forceinline__ float4 ld_stream(const float* p) {
+  return __ldcs(reinterpret_cast<const float4*>(p));
+}
+__device__ __forceinline__ void st_stream(float* p, float4 v) {
+  __stcs(reinterpret_cast<float4*>(p), v);
+}
+__device__ __forceinline__ float comp(const float4& v, int j) {
+  return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+}
+
+__global__ void __launch_bounds__(kEfThreads) k_ef_capture(DevPlan dp, WorkerPtrs wp, float lr,
+                                                           uint32_t* __restrict__ out_idx,
+                                                           float* __restrict__ out_val) {
+  constexpr int V = kEfVecPerThread;
+  constexpr int NWARP = kEfThreads / 32;
+  __shared__ uint32_t s_wtot[V * NWARP];  // candidates per (v, warp), v-major
+  __shared__ uint32_t s_base[V * NWARP];
+  __shared__ uint32_t s_total;
+
+  const uint32_t t = blockIdx.x, p = blockIdx.y;
+  const TileDesc td = dp.tiles[t];
+  const LayerDesc ld = dp.layers[td.layer];
+  const float* __restrict__ g = wp.g[p];
+  float* __restrict__ r = wp.r[p];
+  const uint32_t start = td.start, end = td.start + td.len;
+  const uint32_t base = start & ~3u;
+  const uint32_t N = dp.N;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  float4 a[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    const uint32_t e0 = base + 4u * (v * kEfThreads + threadIdx.x);
+    float4 gv = make_float4(0.f, 0.f, 0.f, 0.f), rv = gv;
+    if (e0 < end) {
+      if (e0 + 4 <= N) {
+        gv = ld_stream(g + e0);
+        rv = ld_stream(r + e0);
+      } else {
+        gv.x = g[e0];
+        rv.x = r[e0];
+        if (e0 + 1 < N) { gv.y = g[e0 + 1]; rv.y = r[e0 + 1]; }
+        if (e0 + 2 < N) { gv.z = g[e0 + 2]; rv.z = r[e0 + 2]; }
+      }
+    }
+    a[v].x = __fadd_rn(rv.x, __fmul_rn(lr, gv.x));
+    a[v].y = __fadd_rn(rv.y, __fmul_rn(lr, gv.y));
+    a[v].z = __fadd_rn(rv.z, __fmul_rn(lr, gv.z));
+    a[v].w = __fadd_rn(rv.w, __fmul_rn(lr, gv.w));
+  }
+
+  if (ld.k == ld.d) {
+    // dense layer: all entries are picks, residual becomes +0
+    const uint64_t ob = (uint64_t)p * dp.K + ld.koff;
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const uint32_t e0 = base + 4u * (v * kEfThreads + threadIdx.x);
+      if (e0 >= end) continue;
+      if (e0 >= start && e0 + 4 <= end) {
+        st_stream(r + e0, make_float4(0.f, 0.f, 0.f, 0.f));
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t e = e0 + j;
+        if (e < start || e >= end) continue;
+        out_idx[ob + (e - ld.off)] = e;
+        out_val[ob + (e - ld.off)] = comp(a[v], j);
+        if (!(e0 >= start && e0 + 4 <= end)) r[e] = 0.0f;
+      }
+    }
+    return;
+  }
+
+  // sparse layer: write acc back and capture candidates in index order
+  const uint32_t lo = dp.lo_key[(size_t)p * dp.L + td.layer];
+  uint32_t masks = 0;
+  uint32_t excl[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    const uint32_t e0 = base + 4u * (v * kEfThreads + threadIdx.x);
+    uint32_t m4 = 0;
+    if (e0 < end) {
+      const bool full = e0 >= start && e0 + 4 <= end;
+      if (full) st_stream(r + e0, a[v]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t e = e0 + j;
+        if (e < start || e >= end) continue;
+        const float x = comp(a[v], j);
+        if (!full) r[e] = x;
+        if (mag_key(x) >= lo) m4 |= 1u << j;
+      }
+    }
+    masks |= m4 << (4 * v);
+    const uint32_t c = __popc(m4);
+    excl[v] = 0;
+    if (__ballot_sync(kFull, c != 0u)) {
+      const uint32_t incl = warp_incl_scan(c);
+      excl[v] = incl - c;
+      if (lane == 31) s_wtot[v * NWARP + warp] = incl;
+    } else if (lane == 0) {
+      s_wtot[v * NWARP + warp] = 0;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // 64 (v, warp) totals, two per lane, scanned in v-major order
+    const uint32_t x0 = s_wtot[2 * lane], x1 = s_wtot[2 * lane + 1];
+    const uint32_t incl = warp_incl_scan(x0 + x1);
+    const uint32_t ex = incl - x0 - x1;
+    s_base[2 * lane] = ex;
+    s_base[2 * lane + 1] = ex + x0;
+    if (lane == 31) s_total = incl;
+  }
+  __syncthreads();
+
+  const uint32_t cap = ld.slot_cap;
+  const uint64_t slot0 =
+      (uint64_t)p * dp.C + ld.slot_base + (uint64_t)(t - ld.tile_begin) * cap;
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    const uint32_t m4 = (masks >> (4 * v)) & 0xFu;
+    if (!m4) continue;
+    const uint32_t e0 = base + 4u * (v * kEfThreads + threadIdx.x);
+    uint32_t pos = s_base[v * NWARP + warp] + excl[v];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (!((m4 >> j) & 1u)) continue;
+      if (pos < cap) {
+        dp.cand_val[slot0 + pos] = comp(a[v], j);
+        dp.cand_idx[slot0 + pos] = e0 + j;
+      }
+      ++pos;
+    }
+  }
+  if (threadIdx.x == 0) dp.tile_cnt[(size_t)p * dp.T + t] = s_total;
+}
+
+cudaError_t launch_ef_capture(const DevPlan& dp, const WorkerPtrs& wp, float lr,
+                              uint32_t* out_idx, float* out_val, cudaStream_t s) {
+  dim3 grid(dp.T, dp.P);
+  k_ef_capture<<<grid, kEfThreads, 0, s>>>(dp, wp, lr, out_idx, out_val);
+  return cudaGetLastError();
+}
+
+}  // namespace lags

@@ -1,0 +1,75 @@
+// Candidate threshold estimate.
+//
+// Before the fused pass streams a layer, one CTA per sparse (worker, layer)
+// draws a sample of m_l entries of acc = residual + lr*grad (the whole layer
+// when it is at most kSampleMax long, otherwise 256 evenly spaced runs of 64
+// contiguous entries) and finds the magnitude key of the sample's r*-th
+// largest entry, rounded down to a level-1 radix bin edge.  The fused pass
+// then keeps every entry at or above that key as a candidate.  r* is chosen on
+// the host so that, for a sample drawn from the layer, the candidates hold the
+// layer's k largest entries with overwhelming probability; when they do not
+// (or a tile overflows its candidate slots) the selection kernel falls back to
+// an exhaustive radix select, so the estimate only affects speed, never the
+// result.  For layers sampled whole r* = k, which makes the bound certain.
+#include "block_ops.cuh"
+#include "lags_internal.cuh"
+
+namespace lags {
+
+__global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs wp, float lr) {
+  extern __shared__ uint32_t s_keys[];  // kSampleMax
+  __shared__ uint32_t s_hist[kBins];
+  __shared__ uint32_t s_tmp[kEstThreads + kEstThreads / 32 + 4];
+
+  const uint32_t layer = dp.sparse[blockIdx.x];
+  const uint32_t p = blockIdx.y;
+  const LayerDesc ld = dp.layers[layer];
+  const float* __restrict__ g = wp.g[p];
+  const float* __restrict__ r = wp.r[p];
+  const uint32_t m = ld.sample;
+  const uint32_t nchunk = m / kSampleChunk;
+
+  for (uint32_t i = threadIdx.x; i < kBins; i += kEstThreads) s_hist[i] = 0;
+  for (uint32_t i = threadIdx.x; i < m; i += kEstThreads) {
+    uint32_t e;
+    if (m == ld.d) {
+      e = ld.off + i;
+    } else {
+      uint32_t c = i / kSampleChunk, j = i % kSampleChunk;
+      e = ld.off + (uint32_t)((uint64_t)c * (ld.d - kSampleChunk) / (nchunk - 1)) + j;
+    }
+    float acc = __fadd_rn(__ldg(r + e), __fmul_rn(lr, __ldg(g + e)));
+    s_keys[i] = mag_key(acc);
+  }
+  __syncthreads();
+
+  // level 0: bits 30..20
+  for (uint32_t i = threadIdx.x; i < m; i += kEstThreads) atomicAdd(&s_hist[s_keys[i] >> 20], 1u);
+  __syncthreads();
+  BinPick b0 = block_find_bin<kEstThreads, kBins>(s_hist, ld.rank, s_tmp);
+  const uint32_t rem = ld.rank - b0.above;
+  for (uint32_t i = threadIdx.x; i < kBins; i += kEstThreads) s_hist[i] = 0;
+  __syncthreads();
+  // level 1: bits 19..9 among keys of bin b0
+  for (uint32_t i = threadIdx.x; i < m; i += kEstThreads) {
+    uint32_t k = s_keys[i];
+    if ((k >> 20) == b0.bin) atomicAdd(&s_hist[(k >> 9) & 0x7FFu], 1u);
+  }
+  __syncthreads();
+  BinPick b1 = block_find_bin<kEstThreads, kBins>(s_hist, rem, s_tmp);
+  if (threadIdx.x == 0) dp.lo_key[(size_t)p * dp.L + layer] = (b0.bin << 20) | (b1.bin << 9);
+}
+
+cudaError_t configure_estimate() {
+  return cudaFuncSetAttribute(k_estimate, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)(kSampleMax * sizeof(uint32_t)));
+}
+
+cudaError_t launch_estimate(const DevPlan& dp, const WorkerPtrs& wp, float lr, cudaStream_t s) {
+  if (dp.n_sparse == 0) return cudaSuccess;
+  dim3 grid(dp.n_sparse, dp.P);
+  k_estimate<<<grid, kEstThreads, kSampleMax * sizeof(uint32_t), s>>>(dp, wp, lr);
+  return cudaGetLastError();
+}
+
+}  // namespace lags

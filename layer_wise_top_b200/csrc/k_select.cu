@@ -1,0 +1,323 @@
+// Exact per-layer top-k (radix select) and ordered emission.
+//
+// One thread-block cluster of CL CTAs per sparse (worker, layer); each CTA owns
+// a contiguous, index-ordered share of the layer.  The CTAs count the layer's
+// candidates; if the sampled threshold held (at least k_l candidates and no
+// tile overflowed its slots) they work on the candidate lists, otherwise on
+// the full acc of the layer (held in the residual buffer after the fused
+// pass).  Either way the result is the exact top-k of the layer:
+//
+//  1. radix select on the magnitude key (bits 30..20, 19..9, 8..0): every CTA
+//     builds a shared-memory histogram of its share (warp-aggregated with
+//     __match_any_sync), the CTAs add their bins into CTA 0's histogram
+//     through distributed shared memory, and every CTA reads the merged
+//     histogram to pick the bin holding the k-th largest key.  It stops early
+//     once a whole bin is taken.  The result is a key prefix (shift s, value
+//     T): entries with key>>s > T are picks, entries with key>>s == T are ties
+//     of which the `need` lowest indices are picks ("lower index wins").
+//  2. each CTA counts its strict picks and ties, the counts are exchanged, and
+//     each CTA emits its picks in index order at
+//         pos = strict_before + min(need, ties_before)
+//     with block-wide scans, writing (index, acc) to the pick list and +0 over
+//     the picked residuals.
+// No CTA ever waits on another outside the hardware cluster barrier.
+#include <cooperative_groups.h>
+
+#include "block_ops.cuh"
+#include "lags_internal.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace lags {
+
+namespace {
+
+constexpr int NT = kSelectThreads;
+
+template <int CL>
+struct Cluster {
+  __device__ __forceinline__ static void sync() {
+    if constexpr (CL > 1) {
+      cg::this_cluster().sync();
+    } else {
+      __syncthreads();
+    }
+  }
+  __device__ __forceinline__ static uint32_t rank() {
+    if constexpr (CL > 1) {
+      return cg::this_cluster().block_rank();
+    } else {
+      return 0;
+    }
+  }
+  template <typename T>
+  __device__ __forceinline__ static T* remote(T* p, uint32_t r) {
+    if constexpr (CL > 1) {
+      return cg::this_cluster().map_shared_rank(p, r);
+    } else {
+      return p;
+    }
+  }
+};
+
+struct SelectShared {
+  uint32_t hist[kBins];          // this CTA's histogram (then the merged copy)
+  uint32_t merged[3][kBins];     // CTA 0: cluster-wide histograms, one per level
+  uint32_t tpre[kSelectWindow + 1];
+  uint32_t tmp[NT + NT / 32 + 4];
+  uint32_t xch[4];               // read by the other CTAs of the cluster
+};
+
+}  // namespace
+
+template <int CL>
+__global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const uint32_t* list,
+                                               uint32_t* __restrict__ out_idx,
+                                               float* __restrict__ out_val) {
+  using C = Cluster<CL>;
+  __shared__ SelectShared sh;
+  const uint32_t rank = C::rank();
+  const uint32_t layer = list[blockIdx.x / CL];
+  const uint32_t p = blockIdx.y;
+  const LayerDesc ld = dp.layers[layer];
+  const int tid = threadIdx.x, lane = tid & 31;
+  float* __restrict__ r = wp.r[p];
+
+  for (int i = tid; i < (int)kBins; i += NT) {
+    sh.hist[i] = 0;
+    sh.merged[0][i] = 0;
+    sh.merged[1][i] = 0;
+    sh.merged[2][i] = 0;
+  }
+
+  // ---- mode: candidate lists or exhaustive ----
+  const uint32_t nt = ld.tile_end - ld.tile_begin;
+  const uint32_t ta = ld.tile_begin + (uint32_t)((uint64_t)nt * rank / CL);
+  const uint32_t tb = ld.tile_begin + (uint32_t)((uint64_t)nt * (rank + 1) / CL);
+  const uint32_t cap = ld.slot_cap;
+  const uint32_t* cnt = dp.tile_cnt + (size_t)p * dp.T;
+  uint32_t my = 0, ovf = 0;
+  for (uint32_t t = ta + tid; t < tb; t += NT) {
+    const uint32_t c = cnt[t];
+    my += c;
+    ovf |= c > cap;
+  }
+  my = block_sum<NT>(my, sh.tmp);
+  ovf = block_sum<NT>(ovf, sh.tmp);
+  if (tid == 0) {
+    sh.xch[0] = my;
+    sh.xch[1] = ovf;
+  }
+  C::sync();  // also publishes the zeroed histograms cluster-wide
+  uint64_t total = 0;
+  uint32_t any_ovf = 0;
+#pragma unroll
+  for (int q = 0; q < CL; ++q) {
+    const uint32_t* x = C::remote(sh.xch, q);
+    total += x[0];
+    any_ovf |= x[1];
+  }
+  const bool fast = !any_ovf && total >= ld.k;
+  if (!fast && rank == 0 && tid == 0) atomicAdd(dp.status + kStatusFallbacks, 1u);
+
+  const uint32_t ea = ld.off + (uint32_t)((uint64_t)ld.d * rank / CL);
+  const uint32_t eb = ld.off + (uint32_t)((uint64_t)ld.d * (rank + 1) / CL);
+  const uint64_t cbase = (uint64_t)p * dp.C + ld.slot_base;
+
+  // Visit this CTA's share in index order, NT entries per round; every thread
+  // calls fn once per round (valid or not), so fn may contain barriers.
+  auto traverse = [&](auto&& fn) {
+    if (fast) {
+      for (uint32_t w0 = ta; w0 < tb; w0 += kSelectWindow) {
+        const uint32_t nw = min(kSelectWindow, tb - w0);
+        constexpr int PER = kSelectWindow / NT;
+        uint32_t c[PER], s = 0;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const uint32_t q = tid * PER + i;
+          c[i] = q < nw ? cnt[w0 + q] : 0u;
+          s += c[i];
+        }
+        uint32_t wtotal;
+        uint32_t ex = block_excl_scan<NT>(s, sh.tmp, &wtotal);
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const uint32_t q = tid * PER + i;
+          if (q < nw) sh.tpre[q] = ex;
+          ex += c[i];
+        }
+        __syncthreads();
+        for (uint32_t b = 0; b < wtotal; b += NT) {
+          const uint32_t v = b + tid;
+          const bool valid = v < wtotal;
+          uint32_t idx = 0;
+          float val = 0.f;
+          if (valid) {
+            uint32_t lo = 0, hi = nw - 1;
+            while (lo < hi) {
+              const uint32_t mid = (lo + hi + 1) >> 1;
+              if (sh.tpre[mid] <= v) lo = mid; else hi = mid - 1;
+            }
+            const uint64_t slot =
+                cbase + (uint64_t)(w0 + lo - ld.tile_begin) * cap + (v - sh.tpre[lo]);
+            idx = dp.cand_idx[slot];
+            val = dp.cand_val[slot];
+          }
+          fn(valid, idx, val);
+        }
+        __syncthreads();
+      }
+    } else {
+      for (uint32_t b = ea; b < eb; b += NT) {
+        const uint32_t e = b + tid;
+        const bool valid = e < eb;
+        const float val = valid ? r[e] : 0.f;
+        fn(valid, e, val);
+      }
+    }
+  };
+
+  // One radix level: histogram of digit (key >> dshift) & dmask over the keys
+  // whose prefix key >> mshift equals mval (all keys when mshift == 32),
+  // merged across the cluster into sh.hist.
+  auto hist_level = [&](int level, int mshift, uint32_t mval, int dshift, uint32_t dmask) {
+    traverse([&](bool valid, uint32_t, float val) {
+      const uint32_t key = mag_key(val);
+      const bool m = valid && (mshift >= 32 || (key >> mshift) == mval);
+      const uint32_t dig = m ? ((key >> dshift) & dmask) : 0xFFFFFFFFu;
+      const unsigned peers = __match_any_sync(kFull, dig);
+      if (m && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
+    });
+    __syncthreads();
+    if constexpr (CL > 1) {
+      uint32_t* dst = C::remote(sh.merged[level], 0);
+      for (int i = tid; i < (int)kBins; i += NT) {
+        const uint32_t h = sh.hist[i];
+        if (h) atomicAdd(dst + i, h);
+      }
+      C::sync();
+      const uint32_t* src = C::remote(sh.merged[level], 0);
+      for (int i = tid; i < (int)kBins; i += NT) sh.hist[i] = src[i];
+      __syncthreads();
+    }
+  };
+  auto clear_hist = [&]() {
+    for (int i = tid; i < (int)kBins; i += NT) sh.hist[i] = 0;
+    __syncthreads();
+  };
+
+  // ---- radix select ----
+  uint32_t rem = ld.k;
+  int fshift;
+  uint32_t fpfx;
+  {
+    hist_level(0, 32, 0, kDigitShift0, 0x7FFu);
+    BinPick b = block_find_bin<NT, kBins>(sh.hist, rem, sh.tmp);
+    rem -= b.above;
+    fpfx = b.bin;
+    fshift = kDigitShift0;
+    if (b.count != rem) {
+      clear_hist();
+      hist_level(1, kDigitShift0, fpfx, kDigitShift1, 0x7FFu);
+      b = block_find_bin<NT, kBins>(sh.hist, rem, sh.tmp);
+      rem -= b.above;
+      fpfx = (fpfx << 11) | b.bin;
+      fshift = kDigitShift1;
+      if (b.count != rem) {
+        clear_hist();
+        hist_level(2, kDigitShift1, fpfx, kDigitShift2, 0x1FFu);
+        b = block_find_bin<NT, 512>(sh.hist, rem, sh.tmp);
+        rem -= b.above;
+        fpfx = (fpfx << 9) | b.bin;
+        fshift = kDigitShift2;
+      }
+    }
+  }
+  const uint32_t need = rem;
+
+  // ---- count strict picks and ties of this CTA, exchange prefixes ----
+  uint32_t na = 0, nb = 0;
+  traverse([&](bool valid, uint32_t, float val) {
+    const uint32_t s = mag_key(val) >> fshift;
+    na += valid && s > fpfx;
+    nb += valid && s == fpfx;
+  });
+  na = block_sum<NT>(na, sh.tmp);
+  nb = block_sum<NT>(nb, sh.tmp);
+  if (tid == 0) {
+    sh.xch[2] = na;
+    sh.xch[3] = nb;
+  }
+  C::sync();
+  uint32_t a_run = 0, b_run = 0;
+  for (uint32_t q = 0; q < rank; ++q) {
+    const uint32_t* x = C::remote(sh.xch, q);
+    a_run += x[2];
+    b_run += x[3];
+  }
+
+  // ---- ordered emission ----
+  const uint64_t ob = (uint64_t)p * dp.K + ld.koff;
+  traverse([&](bool valid, uint32_t idx, float val) {
+    const uint32_t s = mag_key(val) >> fshift;
+    const bool st = valid && s > fpfx;
+    const bool ti = valid && s == fpfx;
+    uint32_t tot;
+    const uint32_t ex = block_excl_scan<NT>(((uint32_t)st << 16) | (uint32_t)ti, sh.tmp, &tot);
+    const uint32_t at = a_run + (ex >> 16), bt = b_run + (ex & 0xFFFFu);
+    bool emit = false;
+    uint32_t pos = 0;
+    if (st) {
+      emit = true;
+      pos = at + min(need, bt);
+    } else if (ti && bt < need) {
+      emit = true;
+      pos = at + bt;
+    }
+    if (emit) {
+      if (pos < ld.k) {
+        out_idx[ob + pos] = idx;
+        out_val[ob + pos] = val;
+        r[idx] = 0.0f;
+      } else {
+        atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
+      }
+    }
+    a_run += tot >> 16;
+    b_run += tot & 0xFFFFu;
+  });
+  C::sync();  // no CTA leaves while another may still read its shared memory
+}
+
+cudaError_t configure_select() { return cudaSuccess; }
+
+cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out_idx,
+                          float* out_val, cudaStream_t s) {
+  if (dp.n_small) {
+    dim3 grid(dp.n_small, dp.P);
+    k_select<1><<<grid, NT, 0, s>>>(dp, wp, dp.sel_small, out_idx, out_val);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (dp.n_large) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(dp.n_large * kSelectCluster, dp.P);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kSelectCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_select<kSelectCluster>, dp, wp, dp.sel_large,
+                                       out_idx, out_val);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
+  return cudaSuccess;
+}
+
+}  // namespace lags

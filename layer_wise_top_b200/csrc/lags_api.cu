@@ -1,0 +1,326 @@
+// C ABI of liblags.so: plan construction (host), workspace binding, argument
+// validation and the launches.  See include/lags.h for the contract.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "lags.h"
+#include "lags_internal.cuh"
+
+namespace lags {
+cudaError_t configure_estimate();
+cudaError_t configure_select();
+}  // namespace lags
+
+using namespace lags;
+
+struct lags_plan {
+  int32_t L = 0, P = 0;
+  uint64_t N = 0, K = 0, C = 0;
+  std::vector<LayerDesc> layers;
+  std::vector<TileDesc> tiles;
+  std::vector<uint32_t> sel_large, sel_small, sparse;
+  std::vector<int64_t> off, k, koff;
+  // workspace sections (byte offsets)
+  size_t o_layers = 0, o_tiles = 0, o_large = 0, o_small = 0, o_sparse = 0, o_lo = 0, o_cnt = 0,
+         o_cval = 0, o_cidx = 0, o_first = 0, o_status = 0, ws_bytes = 0;
+  void* ws = nullptr;
+  int device = -1;
+  cudaEvent_t ev_before = nullptr, ev_after = nullptr;
+  DevPlan dp{};
+};
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t section(size_t& cursor, size_t bytes) {
+  size_t at = (cursor + kAlign - 1) / kAlign * kAlign;
+  cursor = at + bytes;
+  return at;
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// Candidate slots per tile for a layer picking k of d entries: about six times
+// the expected number of candidates per tile plus a floor, in warp multiples.
+uint32_t slot_capacity(uint64_t d, uint64_t k) {
+  double expect = (double)kTile * 6.0 * (double)k / (double)d;
+  double cap = std::ceil(expect) + 64.0;
+  uint64_t c = ((uint64_t)cap + 31) / 32 * 32;
+  return (uint32_t)(c < kTile ? c : kTile);
+}
+
+// Sample rank r* for a sample of m entries out of d, k picks: 1.5x the
+// expected number of sampled entries above the k-th largest, plus four
+// standard deviations and a floor of 8.  A whole-layer sample uses r* = k.
+uint32_t sample_rank(uint64_t m, uint64_t d, uint64_t k) {
+  if (m == d) return (uint32_t)k;
+  double mu = (double)m * (double)k / (double)d;
+  double r = std::ceil(1.5 * mu + 4.0 * std::sqrt(mu) + 8.0);
+  if (r > (double)m) r = (double)m;
+  if (r < 1.0) r = 1.0;
+  return (uint32_t)r;
+}
+
+lags_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LAGS_OK : LAGS_ERR_CUDA; }
+
+bool fill_workers(const lags_plan* plan, const float* const* grads, float* const* residuals,
+                  WorkerPtrs* wp, lags_status* err) {
+  std::memset(wp, 0, sizeof(*wp));
+  for (int p = 0; p < plan->P; ++p) {
+    if (!grads[p] || !residuals[p]) {
+      *err = LAGS_ERR_INVALID_ARG;
+      return false;
+    }
+    if (!aligned(grads[p], 16) || !aligned(residuals[p], 16)) {
+      *err = LAGS_ERR_ALIGNMENT;
+      return false;
+    }
+    wp->g[p] = grads[p];
+    wp->r[p] = residuals[p];
+  }
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities,
+                             int32_t num_layers, int32_t num_workers, lags_plan** out_plan) {
+  if (!out_plan) return LAGS_ERR_INVALID_ARG;
+  *out_plan = nullptr;
+  if (!layer_sizes || !densities || num_layers < 1 || num_layers > (1 << 24) ||
+      num_workers < 1 || num_workers > LAGS_MAX_WORKERS)
+    return LAGS_ERR_INVALID_ARG;
+  lags_plan* plan = new (std::nothrow) lags_plan();
+  if (!plan) return LAGS_ERR_INVALID_ARG;
+  plan->L = num_layers;
+  plan->P = num_workers;
+  uint64_t off = 0, koff = 0, slots = 0;
+  for (int32_t l = 0; l < num_layers; ++l) {
+    const int64_t d = layer_sizes[l];
+    const double rho = densities[l];
+    if (d <= 0 || !(rho > 0.0) || !(rho <= 1.0)) {
+      delete plan;
+      return LAGS_ERR_INVALID_ARG;
+    }
+    double kd = std::ceil(rho * (double)d);
+    uint64_t k = kd < 1.0 ? 1 : (kd >= (double)d ? (uint64_t)d : (uint64_t)kd);
+    if (off + (uint64_t)d >= (1ull << 32)) {  // indices are uint32
+      delete plan;
+      return LAGS_ERR_INVALID_ARG;
+    }
+    LayerDesc ld{};
+    ld.off = (uint32_t)off;
+    ld.d = (uint32_t)d;
+    ld.k = (uint32_t)k;
+    ld.koff = (uint32_t)koff;
+    ld.tile_begin = (uint32_t)plan->tiles.size();
+    const uint64_t j0 = off / kTile, j1 = (off + d - 1) / kTile;
+    for (uint64_t j = j0; j <= j1; ++j) {
+      uint64_t s = j * kTile > off ? j * kTile : off;
+      uint64_t e = (j + 1) * kTile < off + d ? (j + 1) * kTile : off + d;
+      TileDesc td{(uint32_t)s, (uint32_t)(e - s), (uint32_t)l, 0};
+      plan->tiles.push_back(td);
+    }
+    ld.tile_end = (uint32_t)plan->tiles.size();
+    const bool dense = k == (uint64_t)d;
+    if (!dense) {
+      ld.slot_cap = slot_capacity(d, k);
+      ld.slot_base = (uint32_t)slots;
+      slots += (uint64_t)(ld.tile_end - ld.tile_begin) * ld.slot_cap;
+      ld.sample = (uint32_t)((uint64_t)d < kSampleMax ? d : kSampleMax);
+      ld.rank = sample_rank(ld.sample, d, k);
+      plan->sparse.push_back((uint32_t)l);
+      ((uint64_t)d >= kLargeLayer ? plan->sel_large : plan->sel_small).push_back((uint32_t)l);
+    }
+    if (slots >= (1ull << 32) || koff + k >= (1ull << 32)) {
+      delete plan;
+      return LAGS_ERR_INVALID_ARG;
+    }
+    plan->layers.push_back(ld);
+    plan->off.push_back((int64_t)off);
+    plan->k.push_back((int64_t)k);
+    plan->koff.push_back((int64_t)koff);
+    off += (uint64_t)d;
+    koff += k;
+  }
+  plan->N = off;
+  plan->K = koff;
+  plan->C = slots;
+  const uint64_t P = (uint64_t)num_workers, T = plan->tiles.size();
+  size_t cur = 0;
+  plan->o_layers = section(cur, plan->layers.size() * sizeof(LayerDesc));
+  plan->o_tiles = section(cur, T * sizeof(TileDesc));
+  plan->o_large = section(cur, (plan->sel_large.size() + 1) * 4);
+  plan->o_small = section(cur, (plan->sel_small.size() + 1) * 4);
+  plan->o_sparse = section(cur, (plan->sparse.size() + 1) * 4);
+  plan->o_lo = section(cur, P * (uint64_t)num_layers * 4);
+  plan->o_cnt = section(cur, P * T * 4);
+  plan->o_cval = section(cur, P * (plan->C + 1) * 4);
+  plan->o_cidx = section(cur, P * (plan->C + 1) * 4);
+  plan->o_first = section(cur, P * T * 4);
+  plan->o_status = section(cur, kStatusWords * 4);
+  plan->ws_bytes = (cur + kAlign - 1) / kAlign * kAlign;
+  *out_plan = plan;
+  return LAGS_OK;
+}
+
+lags_status lags_plan_destroy(lags_plan* plan) {
+  if (!plan) return LAGS_ERR_INVALID_ARG;
+  delete plan;
+  return LAGS_OK;
+}
+
+lags_status lags_plan_info(const lags_plan* plan, int64_t* N, int64_t* K,
+                           size_t* workspace_bytes) {
+  if (!plan) return LAGS_ERR_INVALID_ARG;
+  if (N) *N = (int64_t)plan->N;
+  if (K) *K = (int64_t)plan->K;
+  if (workspace_bytes) *workspace_bytes = plan->ws_bytes;
+  return LAGS_OK;
+}
+
+lags_status lags_plan_layer(const lags_plan* plan, int32_t l, int64_t* offset, int64_t* k,
+                            int64_t* pick_offset) {
+  if (!plan || l < 0 || l >= plan->L) return LAGS_ERR_INVALID_ARG;
+  if (offset) *offset = plan->off[l];
+  if (k) *k = plan->k[l];
+  if (pick_offset) *pick_offset = plan->koff[l];
+  return LAGS_OK;
+}
+
+lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t bytes,
+                                    void* stream) {
+  if (!plan || !workspace) return LAGS_ERR_INVALID_ARG;
+  if (!aligned(workspace, kAlign)) return LAGS_ERR_ALIGNMENT;
+  if (bytes < plan->ws_bytes) return LAGS_ERR_WORKSPACE;
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LAGS_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return LAGS_ERR_CUDA;
+  if (major != 10 || minor != 0) return LAGS_ERR_UNSUPPORTED_DEVICE;
+  if (configure_estimate() != cudaSuccess || configure_select() != cudaSuccess)
+    return LAGS_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* base = (char*)workspace;
+  auto up = [&](size_t o, const void* src, size_t n) {
+    return n ? cudaMemcpyAsync(base + o, src, n, cudaMemcpyHostToDevice, s) : cudaSuccess;
+  };
+  cudaError_t e = cudaSuccess;
+  if (e == cudaSuccess) e = up(plan->o_layers, plan->layers.data(), plan->layers.size() * sizeof(LayerDesc));
+  if (e == cudaSuccess) e = up(plan->o_tiles, plan->tiles.data(), plan->tiles.size() * sizeof(TileDesc));
+  if (e == cudaSuccess) e = up(plan->o_large, plan->sel_large.data(), plan->sel_large.size() * 4);
+  if (e == cudaSuccess) e = up(plan->o_small, plan->sel_small.data(), plan->sel_small.size() * 4);
+  if (e == cudaSuccess) e = up(plan->o_sparse, plan->sparse.data(), plan->sparse.size() * 4);
+  if (e == cudaSuccess) e = cudaMemsetAsync(base + plan->o_status, 0, kStatusWords * 4, s);
+  // pageable sources: make sure the copies are done before returning
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return LAGS_ERR_CUDA;
+  DevPlan& dp = plan->dp;
+  dp.layers = (const LayerDesc*)(base + plan->o_layers);
+  dp.tiles = (const TileDesc*)(base + plan->o_tiles);
+  dp.sel_large = (const uint32_t*)(base + plan->o_large);
+  dp.sel_small = (const uint32_t*)(base + plan->o_small);
+  dp.sparse = (const uint32_t*)(base + plan->o_sparse);
+  dp.lo_key = (uint32_t*)(base + plan->o_lo);
+  dp.tile_cnt = (uint32_t*)(base + plan->o_cnt);
+  dp.cand_val = (float*)(base + plan->o_cval);
+  dp.cand_idx = (uint32_t*)(base + plan->o_cidx);
+  dp.pick_first = (uint32_t*)(base + plan->o_first);
+  dp.status = (uint32_t*)(base + plan->o_status);
+  dp.L = (uint32_t)plan->L;
+  dp.T = (uint32_t)plan->tiles.size();
+  dp.P = (uint32_t)plan->P;
+  dp.n_large = (uint32_t)plan->sel_large.size();
+  dp.n_small = (uint32_t)plan->sel_small.size();
+  dp.n_sparse = (uint32_t)plan->sparse.size();
+  dp.N = (uint32_t)plan->N;
+  dp.K = plan->K;
+  dp.C = plan->C;
+  plan->ws = workspace;
+  plan->device = dev;
+  return LAGS_OK;
+}
+
+lags_status lags_sparsify(lags_plan* plan, const float* const* grads, float* const* residuals,
+                          float lr, uint32_t* out_idx, float* out_val, void* stream) {
+  if (!plan || !grads || !residuals || !out_idx || !out_val) return LAGS_ERR_INVALID_ARG;
+  if (!plan->ws) return LAGS_ERR_WORKSPACE;
+  if (!aligned(out_idx, 4) || !aligned(out_val, 4)) return LAGS_ERR_ALIGNMENT;
+  WorkerPtrs wp;
+  lags_status err = LAGS_OK;
+  if (!fill_workers(plan, grads, residuals, &wp, &err)) return err;
+  cudaStream_t s = (cudaStream_t)stream;
+  const bool timed = plan->ev_before && plan->ev_after;
+  cudaError_t e = launch_estimate(plan->dp, wp, lr, s);
+  if (e == cudaSuccess && timed) e = cudaEventRecord(plan->ev_before, s);
+  if (e == cudaSuccess) e = launch_ef_capture(plan->dp, wp, lr, out_idx, out_val, s);
+  if (e == cudaSuccess && timed) e = cudaEventRecord(plan->ev_after, s);
+  if (e == cudaSuccess) e = launch_select(plan->dp, wp, out_idx, out_val, s);
+  return cuda_status(e);
+}
+
+lags_status lags_aggregate(lags_plan* plan, const uint32_t* idx, const float* val,
+                           float* dense_out, void* stream) {
+  if (!plan || !idx || !val || !dense_out) return LAGS_ERR_INVALID_ARG;
+  if (!plan->ws) return LAGS_ERR_WORKSPACE;
+  if (!aligned(idx, 4) || !aligned(val, 4) || !aligned(dense_out, 16)) return LAGS_ERR_ALIGNMENT;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_pick_bounds(plan->dp, idx, s);
+  if (e == cudaSuccess) e = launch_aggregate(plan->dp, idx, val, dense_out, s);
+  return cuda_status(e);
+}
+
+lags_status lags_apply(const lags_plan* plan, float* weights, const float* dense_out,
+                       void* stream) {
+  if (!plan || !weights || !dense_out) return LAGS_ERR_INVALID_ARG;
+  if (!aligned(weights, 16) || !aligned(dense_out, 16)) return LAGS_ERR_ALIGNMENT;
+  return cuda_status(launch_apply((uint32_t)plan->N, weights, dense_out, (cudaStream_t)stream));
+}
+
+lags_status lags_plan_set_events(lags_plan* plan, void* before, void* after) {
+  if (!plan) return LAGS_ERR_INVALID_ARG;
+  const bool on = before && after;
+  plan->ev_before = on ? (cudaEvent_t)before : nullptr;
+  plan->ev_after = on ? (cudaEvent_t)after : nullptr;
+  return LAGS_OK;
+}
+
+lags_status lags_status_poll(lags_plan* plan, uint32_t* flags, uint32_t* exact_fallbacks,
+                             void* stream) {
+  if (!plan) return LAGS_ERR_INVALID_ARG;
+  if (!plan->ws) return LAGS_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t words[2] = {0, 0};
+  uint32_t* dev = plan->dp.status;
+  cudaError_t e = cudaMemcpyAsync(words, dev, sizeof(words), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dev, 0, sizeof(words), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return LAGS_ERR_CUDA;
+  if (flags) *flags = words[kStatusFlags];
+  if (exact_fallbacks) *exact_fallbacks = words[kStatusFallbacks];
+  return (words[kStatusFlags] & LAGS_FLAG_BAD_PICKS) ? LAGS_ERR_BAD_PICKS : LAGS_OK;
+}
+
+const char* lags_error_string(lags_status status) {
+  switch (status) {
+    case LAGS_OK: return "ok";
+    case LAGS_ERR_INVALID_ARG: return "invalid argument";
+    case LAGS_ERR_ALIGNMENT: return "device pointer not aligned as required";
+    case LAGS_ERR_CUDA: return "CUDA runtime error";
+    case LAGS_ERR_UNSUPPORTED_DEVICE: return "current device is not sm_100 (B200)";
+    case LAGS_ERR_WORKSPACE: return "workspace missing or too small";
+    case LAGS_ERR_BAD_PICKS: return "pick list not ascending or outside its layer";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,104 @@
+// Internal declarations shared by the kernels and the C ABI of liblags.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lags.h"
+
+namespace lags {
+
+// Elements per tile: the unit of the fused error-feedback pass, of candidate
+// storage and of aggregation.  Tiles never cross a layer boundary; interior
+// tile boundaries sit on multiples of kTile in the flattened buffer, so every
+// tile but a layer's first and last is 16-byte aligned at both ends.
+constexpr uint32_t kTile = 8192;
+constexpr uint32_t kEfThreads = 256;                        // fused pass block
+constexpr uint32_t kEfVecPerThread = kTile / 4 / kEfThreads;  // float4 per thread = 8
+
+// Largest sample the threshold estimate draws per (worker, layer).
+constexpr uint32_t kSampleMax = 16384;
+constexpr uint32_t kSampleChunk = 64;  // contiguous elements per sample chunk
+constexpr uint32_t kEstThreads = 512;
+
+// Cluster size used to select the large layers; small layers use one CTA.
+constexpr int kSelectCluster = 8;
+constexpr uint32_t kSelectThreads = 512;
+constexpr uint32_t kSelectWindow = 2048;  // tiles whose prefix sits in smem at once
+constexpr uint32_t kLargeLayer = 1u << 20;  // d_l at or above: clustered select
+
+// Radix digits of the magnitude key (bits 30..0 of the fp32 pattern).
+constexpr int kDigitShift0 = 20;  // level 0: bits 30..20, 2048 bins
+constexpr int kDigitShift1 = 9;   // level 1: bits 19..9,  2048 bins
+constexpr int kDigitShift2 = 0;   // level 2: bits 8..0,    512 bins
+constexpr uint32_t kBins = 2048;
+
+struct LayerDesc {
+  uint32_t off;         // first element in a worker buffer
+  uint32_t d;           // elements
+  uint32_t k;           // picks
+  uint32_t koff;        // first slot of this layer's picks in a worker pick list
+  uint32_t tile_begin;  // first tile id
+  uint32_t tile_end;    // one past the last tile id
+  uint32_t slot_cap;    // candidate slots per tile (0: dense layer)
+  uint32_t slot_base;   // first candidate slot of the layer in a worker region
+  uint32_t sample;      // threshold-estimate sample size m_l
+  uint32_t rank;        // sample rank r*_l that sets the candidate threshold
+  uint32_t pad0, pad1;
+};
+static_assert(sizeof(LayerDesc) == 48, "LayerDesc layout");
+
+struct TileDesc {
+  uint32_t start;  // first element (flattened index)
+  uint32_t len;    // elements, 1..kTile
+  uint32_t layer;
+  uint32_t pad;
+};
+static_assert(sizeof(TileDesc) == 16, "TileDesc layout");
+
+// Worker buffers, passed by value in the launch arguments.
+struct WorkerPtrs {
+  const float* g[LAGS_MAX_WORKERS];
+  float* r[LAGS_MAX_WORKERS];
+};
+
+// Device status words (in the workspace).
+enum StatusWord : uint32_t { kStatusFlags = 0, kStatusFallbacks = 1, kStatusWords = 64 };
+
+// Device-side view of a plan with its workspace bound.
+struct DevPlan {
+  const LayerDesc* layers;
+  const TileDesc* tiles;
+  const uint32_t* sel_large;  // sparse layers selected by a cluster
+  const uint32_t* sel_small;  // sparse layers selected by one CTA
+  const uint32_t* sparse;     // all sparse layers (estimate pass)
+  uint32_t* lo_key;           // [P][L] candidate threshold key
+  uint32_t* tile_cnt;         // [P][T] candidates found per tile
+  float* cand_val;            // [P][C]
+  uint32_t* cand_idx;         // [P][C]
+  uint32_t* pick_first;       // [P][T] first pick slot of each tile (aggregate)
+  uint32_t* status;           // kStatusWords
+  uint32_t L, T, P;
+  uint32_t n_large, n_small, n_sparse;
+  uint32_t N;
+  uint64_t K;
+  uint64_t C;  // candidate slots per worker
+};
+
+// Launchers (each returns the launch's cudaError_t).
+cudaError_t launch_estimate(const DevPlan& dp, const WorkerPtrs& wp, float lr, cudaStream_t s);
+cudaError_t launch_ef_capture(const DevPlan& dp, const WorkerPtrs& wp, float lr,
+                              uint32_t* out_idx, float* out_val, cudaStream_t s);
+cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out_idx,
+                          float* out_val, cudaStream_t s);
+cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStream_t s);
+cudaError_t launch_aggregate(const DevPlan& dp, const uint32_t* idx, const float* val,
+                             float* dense, cudaStream_t s);
+cudaError_t launch_apply(uint32_t N, float* w, const float* dense, cudaStream_t s);
+
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ uint32_t mag_key(float x) {
+  return __float_as_uint(x) & 0x7FFFFFFFu;
+}
+
+}  // namespace lags

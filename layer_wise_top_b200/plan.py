@@ -1,0 +1,100 @@
+"""A plan bound to torch-owned device memory: the convenience layer the tests
+and the benchmark use.  It only checks tensors and passes their pointers and
+the current CUDA stream to the C entry points."""
+from __future__ import annotations
+
+from typing import List, Optional, Sequence
+
+import torch
+
+from . import _binding as B
+
+
+def _stream(stream: Optional[torch.cuda.Stream], device) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+def _need(t: torch.Tensor, dtype, numel: int, what: str) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{what} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous() or t.numel() < numel:
+        raise ValueError(f"{what} must be contiguous with at least {numel} elements")
+
+
+class Plan:
+    """Layer table of one flattened gradient buffer shared by P workers."""
+
+    def __init__(self, layer_sizes: Sequence[int], densities: Sequence[float], P: int,
+                 device: Optional[torch.device] = None):
+        self.device = torch.device(device if device is not None else "cuda")
+        self.handle = B.lags_plan_create(layer_sizes, densities, P)
+        self.P = int(P)
+        self.L = len(layer_sizes)
+        self.N, self.K, self.workspace_bytes = B.lags_plan_info(self.handle)
+        self.layers = [B.lags_plan_layer(self.handle, l) for l in range(self.L)]
+        self.sizes = [int(x) for x in layer_sizes]
+        with torch.cuda.device(self.device):
+            self.workspace = torch.empty(max(self.workspace_bytes, 256), dtype=torch.uint8,
+                                         device=self.device)
+            B.lags_plan_set_workspace(self.handle, self.workspace.data_ptr(),
+                                      self.workspace.numel(), _stream(None, self.device))
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and h.value:
+            B.lags_plan_destroy(h)
+            self.handle = None
+
+    # ---------------------------------------------------------------- buffers
+    def empty_picks(self):
+        idx = torch.empty(self.P * self.K, dtype=torch.int32, device=self.device)
+        val = torch.empty(self.P * self.K, dtype=torch.float32, device=self.device)
+        return idx, val
+
+    # ---------------------------------------------------------------- calls
+    def sparsify(self, grads: List[torch.Tensor], residuals: List[torch.Tensor], lr: float,
+                 out_idx: torch.Tensor, out_val: torch.Tensor,
+                 stream: Optional[torch.cuda.Stream] = None) -> None:
+        if len(grads) != self.P or len(residuals) != self.P:
+            raise ValueError(f"need {self.P} gradient and residual buffers")
+        for i, (g, r) in enumerate(zip(grads, residuals)):
+            _need(g, torch.float32, self.N, f"grads[{i}]")
+            _need(r, torch.float32, self.N, f"residuals[{i}]")
+        _need(out_idx, torch.int32, self.P * self.K, "out_idx")
+        _need(out_val, torch.float32, self.P * self.K, "out_val")
+        B.lags_sparsify(self.handle, [g.data_ptr() for g in grads],
+                        [r.data_ptr() for r in residuals], lr, out_idx.data_ptr(),
+                        out_val.data_ptr(), _stream(stream, self.device))
+
+    def aggregate(self, idx: torch.Tensor, val: torch.Tensor, dense_out: torch.Tensor,
+                  stream: Optional[torch.cuda.Stream] = None) -> None:
+        _need(idx, torch.int32, self.P * self.K, "idx")
+        _need(val, torch.float32, self.P * self.K, "val")
+        _need(dense_out, torch.float32, self.N, "dense_out")
+        B.lags_aggregate(self.handle, idx.data_ptr(), val.data_ptr(), dense_out.data_ptr(),
+                         _stream(stream, self.device))
+
+    def apply(self, weights: torch.Tensor, dense_out: torch.Tensor,
+              stream: Optional[torch.cuda.Stream] = None) -> None:
+        _need(weights, torch.float32, self.N, "weights")
+        _need(dense_out, torch.float32, self.N, "dense_out")
+        B.lags_apply(self.handle, weights.data_ptr(), dense_out.data_ptr(),
+                     _stream(stream, self.device))
+
+    def set_events(self, before: Optional[torch.cuda.Event],
+                   after: Optional[torch.cuda.Event]) -> None:
+        """Record `before`/`after` around the fused pass of later sparsify calls."""
+        if before is None or after is None:
+            B.lags_plan_set_events(self.handle, 0, 0)
+            return
+        for ev in (before, after):
+            if not ev.cuda_event:  # torch creates the event on first record
+                ev.record()
+        B.lags_plan_set_events(self.handle, before.cuda_event, after.cuda_event)
+
+    def poll(self, stream: Optional[torch.cuda.Stream] = None):
+        """(flags, exact_fallbacks) since the last poll; synchronises the stream."""
+        return B.lags_status_poll(self.handle, _stream(stream, self.device))

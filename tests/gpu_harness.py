@@ -1,0 +1,127 @@
+"""Drives the CUDA path through the C ABI (via layer_wise_top_b200.Plan) and
+checks it against the oracle and against full-size invariants (torch on the
+GPU as an independent checker).  Test infrastructure."""
+from __future__ import annotations
+
+from typing import Callable, Dict, Iterable, List, Optional, Sequence
+
+import numpy as np
+import torch
+
+import oracle.lags_oracle as lo
+
+F32 = np.float32
+
+
+def u32(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy().view(np.uint32)
+
+
+class GpuRun:
+    """Runs steps of sparsify -> aggregate -> apply on the GPU."""
+
+    def __init__(self, sizes: Sequence[int], densities: Sequence[float], P: int, lr: float,
+                 keep_prev: bool = False):
+        from layer_wise_top_b200 import Plan
+        self.plan = Plan(sizes, densities, P)
+        self.P, self.lr = P, lr
+        N, K = self.plan.N, self.plan.K
+        dev = torch.device("cuda")
+        self.grads = [torch.empty(N, dtype=torch.float32, device=dev) for _ in range(P)]
+        self.res = [torch.zeros(N, dtype=torch.float32, device=dev) for _ in range(P)]
+        self.idx, self.val = self.plan.empty_picks()
+        self.dense = torch.empty(N, dtype=torch.float32, device=dev)
+        self.weights = torch.zeros(N, dtype=torch.float32, device=dev)
+        self.keep_prev = keep_prev
+        self.prev: Optional[List[torch.Tensor]] = None
+
+    def step(self) -> None:
+        if self.keep_prev:
+            self.prev = [r.clone() for r in self.res]
+        self.plan.sparsify(self.grads, self.res, self.lr, self.idx, self.val)
+        self.plan.aggregate(self.idx, self.val, self.dense)
+        self.plan.apply(self.weights, self.dense)
+
+
+def oracle_layer_steps(off: int, d: int, k: int, P: int, lr: float, steps: int,
+                       grad_fn: Callable[[int, int], np.ndarray]):
+    """Oracle history of one layer: grad_fn(p, s) -> that layer's gradient."""
+    res = [np.zeros(d, dtype=F32) for _ in range(P)]
+    w = np.zeros(d, dtype=F32)
+    out = []
+    for s in range(steps):
+        grads = [grad_fn(p, s) for p in range(P)]
+        idx, val, res = lo.sparsify_layer(off, k, grads, res, lr)
+        dense = lo.aggregate_layer(off, d, idx, val)
+        w = lo.apply_update(w, dense)
+        out.append((idx, val, [r.copy() for r in res], dense, w.copy()))
+    return out
+
+
+def compare_layer(run: GpuRun, l: int, exp, where: str) -> None:
+    """Bit-exact comparison of one layer's slices with an oracle step."""
+    off, k, koff = run.plan.layers[l]
+    d = run.plan.sizes[l]
+    e_idx, e_val, e_res, e_dense, e_w = exp
+    K = run.plan.K
+    idx = u32(run.idx).reshape(run.P, K)[:, koff:koff + k]
+    val = u32(run.val).reshape(run.P, K)[:, koff:koff + k]
+    assert np.array_equal(idx, e_idx), f"{where}: indices differ"
+    assert np.array_equal(val, e_val.view(np.uint32)), f"{where}: values differ"
+    for p in range(run.P):
+        r = u32(run.res[p][off:off + d])
+        assert np.array_equal(r, e_res[p].view(np.uint32)), f"{where}: residual p={p}"
+    assert np.array_equal(u32(run.dense[off:off + d]), e_dense.view(np.uint32)), \
+        f"{where}: dense update"
+    assert np.array_equal(u32(run.weights[off:off + d]), e_w.view(np.uint32)), \
+        f"{where}: weights"
+
+
+def check_invariants(run: GpuRun, workers: Iterable[int], check_dense: bool = True) -> None:
+    """Full-size properties that determine the result uniquely: for every layer
+    the picks are ascending and inside the layer, each value is acc at its
+    index, picked residuals are +0 and the others keep acc, every picked
+    magnitude is >= every unpicked one, and among entries tied at the smallest
+    picked magnitude the picked ones have the lowest indices.  The dense update
+    is recomputed in worker order with one rounding per add."""
+    assert run.prev is not None, "run with keep_prev=True"
+    lr = torch.tensor(run.lr, dtype=torch.float32, device="cuda")
+    K = run.plan.K
+    idx_all = run.idx.view(run.P, K)
+    val_all = run.val.view(run.P, K)
+    for p in workers:
+        acc = run.prev[p] + lr * run.grads[p]  # two separate fp32 roundings
+        res = run.res[p]
+        for l, (off, k, koff) in enumerate(run.plan.layers):
+            d = run.plan.sizes[l]
+            li = idx_all[p, koff:koff + k].to(torch.int64) & 0xFFFFFFFF
+            lv = val_all[p, koff:koff + k]
+            assert bool((li >= off).all() and (li < off + d).all()), (p, l, "range")
+            if k > 1:
+                assert bool((li[1:] > li[:-1]).all()), (p, l, "ascending")
+            a = acc[off:off + d]
+            loc = li - off
+            assert torch.equal(lv.view(torch.int32), a[loc].view(torch.int32)), (p, l, "val")
+            rl = res[off:off + d]
+            mask = torch.zeros(d, dtype=torch.bool, device="cuda")
+            mask[loc] = True
+            assert bool((rl[mask].view(torch.int32) == 0).all()), (p, l, "zeroed")
+            assert torch.equal(rl[~mask].view(torch.int32), a[~mask].view(torch.int32)), \
+                (p, l, "residual")
+            if k < d:
+                mag = a.abs()
+                tmin = mag[mask].min()
+                assert bool(tmin >= mag[~mask].max()), (p, l, "magnitude")
+                tie_unpicked = (~mask) & (mag == tmin)
+                if bool(tie_unpicked.any()):
+                    tie_picked = mask & (mag == tmin)
+                    first_unpicked = int(torch.nonzero(tie_unpicked)[0])
+                    last_picked = int(torch.nonzero(tie_picked)[-1])
+                    assert last_picked < first_unpicked, (p, l, "tie order")
+    if check_dense:
+        dense = torch.zeros(run.plan.N, dtype=torch.float32, device="cuda")
+        for p in range(run.P):
+            li = idx_all[p].to(torch.int64) & 0xFFFFFFFF
+            dense[li] = dense[li] + val_all[p]
+        dense = dense / torch.tensor(float(run.P), dtype=torch.float32, device="cuda")
+        assert torch.equal(dense.view(torch.int32), run.dense.view(torch.int32)), "dense"

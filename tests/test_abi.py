@@ -1,0 +1,100 @@
+"""The C ABI on the CPU: the library loads, exports every entry point that
+include/lags.h declares, and plan creation validates and lays out correctly.
+No compute call is made here (no GPU)."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import layer_wise_top_b200 as L
+import oracle.lags_oracle as lo
+from conftest import ROOT
+from synth.configs import WORKLOADS
+
+
+def declared():
+    with open(os.path.join(ROOT, "include", "lags.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"LAGS_API\s+[\w\s\*]+?\b(lags_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    names = declared()
+    assert len(names) == 11, names
+    lib = ctypes.CDLL(L.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(L.EXPORTED) == names
+
+
+def test_error_strings():
+    for code in range(7):
+        assert L.lags_error_string(code) not in ("", "unknown status")
+    assert L.lags_error_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_plan_matches_oracle_layout(name):
+    w = WORKLOADS[name]
+    h = L.lags_plan_create(w.sizes, w.densities, w.P)
+    try:
+        offs, ks, koffs, N, K = lo.layer_plan(w.sizes, w.densities)
+        assert L.lags_plan_info(h)[:2] == (N, K)
+        for l in range(w.L):
+            assert L.lags_plan_layer(h, l) == (offs[l], ks[l], koffs[l])
+    finally:
+        L.lags_plan_destroy(h)
+
+
+@pytest.mark.parametrize("sizes,dens,P", [
+    ([], [], 1),
+    ([10], [0.5], 0),
+    ([10], [0.5], 257),
+    ([0], [0.5], 1),
+    ([-3], [0.5], 1),
+    ([10], [0.0], 1),
+    ([10], [1.5], 1),
+    ([10], [float("nan")], 1),
+    ([1 << 31, 1 << 31], [0.1, 0.1], 1),   # N >= 2^32
+])
+def test_plan_rejects(sizes, dens, P):
+    with pytest.raises(L.LagsError) as e:
+        L.lags_plan_create(sizes, dens, P)
+    assert e.value.status == L.LAGS_ERR_INVALID_ARG
+
+
+def test_calls_reject_null_and_unbound_plan():
+    h = L.lags_plan_create([100], [0.1], 2)
+    try:
+        with pytest.raises(L.LagsError) as e:
+            L.lags_sparsify(h, [0, 0], [0, 0], 0.1, 0, 0)
+        assert e.value.status == L.LAGS_ERR_INVALID_ARG
+        with pytest.raises(L.LagsError) as e:
+            L.lags_sparsify(h, [16, 32], [48, 64], 0.1, 16, 32)
+        assert e.value.status == L.LAGS_ERR_WORKSPACE   # no workspace bound yet
+        with pytest.raises(L.LagsError) as e:
+            L.lags_aggregate(h, 16, 16, 16)
+        assert e.value.status == L.LAGS_ERR_WORKSPACE
+        with pytest.raises(L.LagsError) as e:
+            L.lags_apply(h, 8, 16)
+        assert e.value.status == L.LAGS_ERR_ALIGNMENT
+        with pytest.raises(L.LagsError) as e:
+            L.lags_plan_set_workspace(h, 128, 1 << 20)
+        assert e.value.status == L.LAGS_ERR_ALIGNMENT
+        with pytest.raises(L.LagsError) as e:
+            L.lags_plan_set_workspace(h, 256, 16)
+        assert e.value.status == L.LAGS_ERR_WORKSPACE
+    finally:
+        L.lags_plan_destroy(h)
+
+
+def test_k_rule_uses_double_density():
+    h = L.lags_plan_create([18_000_000, 2_048_000], [0.001, 0.001], 1)
+    try:
+        assert L.lags_plan_layer(h, 0)[1] == 18000
+        assert L.lags_plan_layer(h, 1)[1] == 2048
+    finally:
+        L.lags_plan_destroy(h)

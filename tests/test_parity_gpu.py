@@ -1,0 +1,208 @@
+"""CUDA path vs the CPU oracle, bit for bit, through the C ABI.
+
+Small cases are compared element by element over every output; the full-size
+workloads are compared on sampled layers (the oracle replays those layers for
+all workers and steps, which is exact because layers are independent) and on
+the invariants that determine the result uniquely for every layer."""
+import numpy as np
+import pytest
+
+import oracle.lags_oracle as lo
+import synth
+from synth.configs import WORKLOADS, Tensor
+
+pytestmark = pytest.mark.gpu
+
+F32 = np.float32
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def run_full_compare(sizes, densities, P, lr, steps, grad_fn, expect_fallbacks=None):
+    """Element-by-element parity of every output for `steps` steps."""
+    torch = _torch()
+    from gpu_harness import GpuRun, u32
+    run = GpuRun(sizes, densities, P, lr)
+    hist = lo.run_workload(sizes, densities, P, lr, steps, grad_fn)
+    total_fb = 0
+    for s in range(steps):
+        for p in range(P):
+            run.grads[p].copy_(torch.from_numpy(grad_fn(p, s)))
+        run.step()
+        flags, fb = run.plan.poll()
+        assert flags == 0
+        total_fb += fb
+        e_idx, e_val, e_res, e_dense, e_w = hist[s]
+        K = run.plan.K
+        assert np.array_equal(u32(run.idx).reshape(P, K), e_idx), f"step {s}: idx"
+        assert np.array_equal(u32(run.val).reshape(P, K), e_val.view(np.uint32)), f"step {s}: val"
+        for p in range(P):
+            assert np.array_equal(u32(run.res[p]), e_res[p].view(np.uint32)), f"step {s}: res {p}"
+        assert np.array_equal(u32(run.dense), e_dense.view(np.uint32)), f"step {s}: dense"
+        assert np.array_equal(u32(run.weights), e_w.view(np.uint32)), f"step {s}: weights"
+    if expect_fallbacks is not None:
+        assert expect_fallbacks(total_fb), total_fb
+    return total_fb
+
+
+def synth_grad_fn(w):
+    cache = {}
+
+    def fn(p, s):
+        if (p, s) not in cache:
+            cache[(p, s)] = synth.worker_grads_host(w, p, s)
+        return cache[(p, s)]
+    return fn
+
+
+# ----------------------------------------------------------------- full small
+def test_resnet20_all_steps_bitexact():
+    w = WORKLOADS["resnet20"]
+    run_full_compare(w.sizes, w.densities, w.P, w.lr, w.steps, synth_grad_fn(w),
+                     expect_fallbacks=lambda fb: fb == 0)
+
+
+RAGGED = [1, 3, 5, 7, 8191, 8192, 8193, 20000, 100003, 36864, 2, 65537]
+
+
+@pytest.mark.parametrize("dist", [synth.NORMAL, synth.STUDENT_T3])
+def test_ragged_layers_mixed_density(dist):
+    rng = np.random.default_rng(11)
+    dens = [float(x) for x in rng.choice([0.001, 0.01, 0.1, 0.5, 1.0], len(RAGGED))]
+    w = WORKLOADS["resnet20"].scaled(
+        "ragged", P=3, steps=4,
+        tensors=[Tensor(f"t{i}", (d,)) for i, d in enumerate(RAGGED)],
+        density_rule=lambda d: 0.0)
+    w = type(w)(w.name, w.tensors, w.P, 0.5, w.steps, dist, 21, w.density_rule)
+    run_full_compare(RAGGED, dens, w.P, w.lr, w.steps, synth_grad_fn(w))
+
+
+def test_large_layers_cluster_select():
+    sizes = [1_100_003, 5, 2_000_001, 1 << 20]
+    dens = [0.001, 1.0, 0.001, 0.01]
+    w = WORKLOADS["lstm_ptb"].scaled("big", P=2, steps=3,
+                                     tensors=[Tensor(f"t{i}", (d,)) for i, d in enumerate(sizes)])
+    run_full_compare(sizes, dens, 2, w.lr, 3, synth_grad_fn(w),
+                     expect_fallbacks=lambda fb: fb == 0)
+
+
+# ----------------------------------------------------------------- ties / degenerate
+def _np_grads(gen, sizes, P, steps):
+    N = sum(sizes)
+    data = {(p, s): gen(N) for p in range(P) for s in range(steps)}
+    return lambda p, s: data[(p, s)]
+
+
+def test_integer_ties_force_exact_path():
+    rng = np.random.default_rng(5)
+    sizes = [9000, 40000, 1_048_577, 17]
+    dens = [0.01, 0.001, 0.001, 0.3]
+    fn = _np_grads(lambda n: rng.integers(-2, 3, n).astype(F32), sizes, 2, 3)
+    fb = run_full_compare(sizes, dens, 2, 1.0, 3, fn)
+    assert fb > 0  # massive ties overflow the candidate slots
+
+
+def test_all_zero_gradients():
+    sizes = [100, 8192, 30000, 1_048_576]
+    fn = _np_grads(lambda n: np.zeros(n, dtype=F32), sizes, 2, 2)
+    run_full_compare(sizes, [0.01, 0.001, 0.5, 0.001], 2, 0.1, 2, fn)
+
+
+def test_signed_zero_denormal_inf():
+    rng = np.random.default_rng(6)
+
+    def gen(n):
+        x = rng.standard_normal(n).astype(F32)
+        x[rng.random(n) < 0.3] = F32(-0.0)
+        x[rng.random(n) < 0.1] = F32(0.0)
+        x[rng.random(n) < 0.05] = (rng.integers(1, 100, 1) * F32(1e-45)).astype(F32)[0]
+        x[rng.random(n) < 0.0005] = F32(np.inf)
+        x[rng.random(n) < 0.0005] = F32(-np.inf)
+        return x
+    sizes = [5000, 70000, 3]
+    fn = _np_grads(gen, sizes, 3, 2)
+    run_full_compare(sizes, [0.01, 0.001, 1.0], 3, 1.0, 2, fn)
+
+
+def test_single_worker_and_k_equals_d():
+    rng = np.random.default_rng(7)
+    sizes = [4096, 10, 12345]
+    fn = _np_grads(lambda n: rng.standard_normal(n).astype(F32), sizes, 1, 2)
+    run_full_compare(sizes, [1.0, 1.0, 0.999], 1, 0.1, 2, fn)
+
+
+def test_k_equals_one_everywhere():
+    rng = np.random.default_rng(8)
+    sizes = [1, 2, 3, 64, 9000, 300000]
+    fn = _np_grads(lambda n: rng.standard_normal(n).astype(F32), sizes, 4, 2)
+    run_full_compare(sizes, [1e-9] * len(sizes), 4, 0.1, 2, fn)
+
+
+def test_deterministic_repeat():
+    torch = _torch()
+    from gpu_harness import GpuRun, u32
+    w = WORKLOADS["vgg16"]
+    outs = []
+    for _ in range(2):
+        run = GpuRun(w.sizes, w.densities, w.P, w.lr)
+        for s in range(2):
+            for p in range(w.P):
+                synth.worker_grads_device(w, p, s, run.grads[p])
+            run.step()
+        torch.cuda.synchronize()
+        outs.append((u32(run.idx), u32(run.val), u32(run.dense), u32(run.res[3])))
+    for a, b in zip(*outs):
+        assert np.array_equal(a, b)
+
+
+# ----------------------------------------------------------------- full size
+SAMPLED = {
+    "vgg16": [1, 0, 2, 27, 26],                      # biases, conv0, conv1, fc
+    "resnet50": [1, 2, 0, 3, 12, 15, 160, 41],       # BN (dense), convs at 0.01, fc bias
+    "lstm_ptb": [2, 3, 8],                           # the bias vectors
+    "gpt_1_3b": [1, 2, 5, 6],                        # LayerNorm gamma/beta
+}
+
+
+def _full_size(name, steps, inv_workers):
+    torch = _torch()
+    from gpu_harness import GpuRun, check_invariants, compare_layer, oracle_layer_steps
+    w = WORKLOADS[name]
+    run = GpuRun(w.sizes, w.densities, w.P, w.lr, keep_prev=True)
+    exp = {}
+    for l in SAMPLED[name]:
+        off, k, _ = run.plan.layers[l]
+        exp[l] = oracle_layer_steps(off, w.sizes[l], k, w.P, w.lr, steps,
+                                    lambda p, s, l=l: synth.layer_grads_host(w, p, s, l))
+    fallbacks = 0
+    for s in range(steps):
+        for p in range(w.P):
+            synth.worker_grads_device(w, p, s, run.grads[p])
+        run.step()
+        flags, fb = run.plan.poll()
+        assert flags == 0
+        fallbacks += fb
+        for l in SAMPLED[name]:
+            compare_layer(run, l, exp[l][s], f"{name} step {s} layer {l}")
+        check_invariants(run, inv_workers, check_dense=True)
+    assert fallbacks == 0, f"{fallbacks} segments took the exhaustive path"
+
+
+def test_full_vgg16():
+    _full_size("vgg16", 10, [0, 5, 15])
+
+
+def test_full_resnet50():
+    _full_size("resnet50", 10, [0, 9])
+
+
+def test_full_lstm():
+    _full_size("lstm_ptb", 10, [0, 7, 15])
+
+
+@pytest.mark.slow
+def test_full_gpt_1_3b():
+    _full_size("gpt_1_3b", 2, [0, 5])
