@@ -21,6 +21,15 @@ def _torch():
     return torch
 
 
+def same_bits_or_nan(got_u32, exp_f32):
+    """Bitwise equality, except that a NaN matches any NaN: IEEE 754 leaves the
+    payload and sign of an invalid operation's NaN (inf - inf) unspecified."""
+    exp_u32 = exp_f32.view(np.uint32)
+    got_f = got_u32.view(np.float32)
+    both_nan = np.isnan(got_f) & np.isnan(exp_f32)
+    return bool(np.all((got_u32 == exp_u32) | both_nan))
+
+
 def run_full_compare(sizes, densities, P, lr, steps, grad_fn, expect_fallbacks=None):
     """Element-by-element parity of every output for `steps` steps."""
     torch = _torch()
@@ -41,8 +50,8 @@ def run_full_compare(sizes, densities, P, lr, steps, grad_fn, expect_fallbacks=N
         assert np.array_equal(u32(run.val).reshape(P, K), e_val.view(np.uint32)), f"step {s}: val"
         for p in range(P):
             assert np.array_equal(u32(run.res[p]), e_res[p].view(np.uint32)), f"step {s}: res {p}"
-        assert np.array_equal(u32(run.dense), e_dense.view(np.uint32)), f"step {s}: dense"
-        assert np.array_equal(u32(run.weights), e_w.view(np.uint32)), f"step {s}: weights"
+        assert same_bits_or_nan(u32(run.dense), e_dense), f"step {s}: dense"
+        assert same_bits_or_nan(u32(run.weights), e_w), f"step {s}: weights"
     if expect_fallbacks is not None:
         assert expect_fallbacks(total_fb), total_fb
     return total_fb
