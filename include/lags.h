@@ -171,6 +171,28 @@ LAGS_API lags_status lags_status_poll(lags_plan* plan, uint32_t* flags, uint32_t
                              void* stream);
 
 /*
+ * lags_sparsify_static - lags_sparsify for callers that cannot allocate device
+ * memory (code running inside an allocator or memory-pool callback, runtimes
+ * that own every device allocation, hosts that forbid cudaMalloc after
+ * start-up).  The pages have no counterpart: it is a deployment variant, not
+ * part of the method.  Arguments and results are those of lags_sparsify, and
+ * the plan needs no workspace: the scratch lives in a 16 MiB array with static
+ * storage in the library, present on every GPU that loads it until exit.
+ *   - Returns LAGS_ERR_WORKSPACE, before enqueuing anything, when the plan's
+ *     workspace_bytes exceed 16 MiB.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating routine.
+ *   - All calls share the array, which keeps the last call's contents; each
+ *     call uploads its plan's tables and clears what must start at zero.
+ *     Calls whose work overlaps on the GPU race on it.
+ *   - The first call on a device resolves the array's address there and
+ *     configures the kernels: make it before any stream capture.
+ *   - The status word it writes is not read by lags_status_poll.
+ */
+LAGS_API lags_status lags_sparsify_static(lags_plan* plan, const float* const* grads,
+                                          float* const* residuals, float lr, uint32_t* out_idx,
+                                          float* out_val, void* stream);
+
+/*
  * lags_plan_set_events - timing instrumentation.  When `before` and `after`
  * (cudaEvent_t passed as void*, created by the caller) are both non-NULL, each
  * later lags_sparsify on this plan records `before` on its stream just before

@@ -23,7 +23,8 @@ LAGS_FLAG_INTERNAL = 0x2
 
 EXPORTED = ("lags_plan_create", "lags_plan_destroy", "lags_plan_info", "lags_plan_layer",
             "lags_plan_set_workspace", "lags_sparsify", "lags_aggregate", "lags_apply",
-            "lags_status_poll", "lags_plan_set_events", "lags_error_string")
+            "lags_status_poll", "lags_plan_set_events", "lags_sparsify_static",
+            "lags_error_string")
 
 
 class LagsError(RuntimeError):
@@ -53,6 +54,8 @@ def _load() -> ctypes.CDLL:
     lib.lags_status_poll.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32),
                                      ctypes.POINTER(ctypes.c_uint32), vp]
     lib.lags_plan_set_events.argtypes = [vp, vp, vp]
+    lib.lags_sparsify_static.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                         ctypes.c_float, vp, vp, vp]
     lib.lags_error_string.argtypes = [st]
     lib.lags_error_string.restype = ctypes.c_char_p
     for name in EXPORTED[:-1]:
@@ -120,6 +123,18 @@ def lags_sparsify(plan, grads: Sequence[int], residuals: Sequence[int], lr: floa
     _check(_LIB.lags_sparsify(plan, g, r, ctypes.c_float(lr), ctypes.c_void_p(out_idx),
                               ctypes.c_void_p(out_val), ctypes.c_void_p(stream)),
            "lags_sparsify")
+
+
+def lags_sparsify_static(plan, grads: Sequence[int], residuals: Sequence[int], lr: float,
+                         out_idx: int, out_val: int, stream: int = 0) -> None:
+    """lags_sparsify with the library's static scratch instead of a workspace,
+    for callers that cannot allocate device memory (see include/lags.h)."""
+    P = len(grads)
+    g = (ctypes.c_void_p * max(P, 1))(*[ctypes.c_void_p(x) for x in grads])
+    r = (ctypes.c_void_p * max(len(residuals), 1))(*[ctypes.c_void_p(x) for x in residuals])
+    _check(_LIB.lags_sparsify_static(plan, g, r, ctypes.c_float(lr), ctypes.c_void_p(out_idx),
+                                     ctypes.c_void_p(out_val), ctypes.c_void_p(stream)),
+           "lags_sparsify_static")
 
 
 def lags_aggregate(plan, idx: int, val: int, dense_out: int, stream: int = 0) -> None:

@@ -1,0 +1,54 @@
+// Host-side plan object shared by the C entry points of liblags.so.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+#include "lags.h"
+#include "lags_internal.cuh"
+
+struct lags_plan {
+  int32_t L = 0, P = 0;
+  uint64_t N = 0, K = 0, C = 0;
+  std::vector<lags::LayerDesc> layers;
+  std::vector<lags::TileDesc> tiles;
+  std::vector<uint32_t> sel_large, sel_small, sparse;
+  std::vector<int64_t> off, k, koff;
+  // workspace sections (byte offsets)
+  size_t o_layers = 0, o_tiles = 0, o_large = 0, o_small = 0, o_sparse = 0, o_lo = 0, o_cnt = 0,
+         o_cval = 0, o_cidx = 0, o_first = 0, o_status = 0, ws_bytes = 0;
+  void* ws = nullptr;
+  int device = -1;
+  cudaEvent_t ev_before = nullptr, ev_after = nullptr;
+  lags::DevPlan dp{};  // device view once a workspace is bound
+};
+
+
+// Device view of `plan` with its tables and scratch laid out at `base`
+// (the workspace sections the plan computed).
+inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out) {
+  using namespace lags;
+  DevPlan& dp = *out;
+  dp.layers = (const LayerDesc*)(base + plan->o_layers);
+  dp.tiles = (const TileDesc*)(base + plan->o_tiles);
+  dp.sel_large = (const uint32_t*)(base + plan->o_large);
+  dp.sel_small = (const uint32_t*)(base + plan->o_small);
+  dp.sparse = (const uint32_t*)(base + plan->o_sparse);
+  dp.lo_key = (uint32_t*)(base + plan->o_lo);
+  dp.tile_cnt = (uint32_t*)(base + plan->o_cnt);
+  dp.cand_val = (float*)(base + plan->o_cval);
+  dp.cand_idx = (uint32_t*)(base + plan->o_cidx);
+  dp.pick_first = (uint32_t*)(base + plan->o_first);
+  dp.status = (uint32_t*)(base + plan->o_status);
+  dp.L = (uint32_t)plan->L;
+  dp.T = (uint32_t)plan->tiles.size();
+  dp.P = (uint32_t)plan->P;
+  dp.n_large = (uint32_t)plan->sel_large.size();
+  dp.n_small = (uint32_t)plan->sel_small.size();
+  dp.n_sparse = (uint32_t)plan->sparse.size();
+  dp.N = (uint32_t)plan->N;
+  dp.K = plan->K;
+  dp.C = plan->C;
+}

@@ -1,0 +1,115 @@
+// lags_sparsify_static: lags_sparsify without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they call the
+// library: code running inside a custom allocator or memory-pool callback,
+// runtimes that own every device allocation and forbid side allocations, and
+// hosts that reserve the device up front and forbid cudaMalloc afterwards.
+// For them this entry point keeps its scratch (the plan tables, the sampled
+// thresholds, the per-tile candidate counts and the candidate slots) in one
+// array with static storage that is part of the library image on each device.
+//
+//  - Limit: a plan whose workspace exceeds kStaticScratchBytes (16 MiB) is
+//    rejected with LAGS_ERR_WORKSPACE before anything is enqueued.
+//  - Every GPU that loads liblags.so holds the 16 MiB until the process exits.
+//  - All calls share the one array and it keeps the last call's contents:
+//    each call re-uploads its plan's tables and clears the status words.
+//    Calls whose work overlaps on the GPU (different streams without ordering,
+//    or several host threads) race on the array.
+//  - The first call on a device resolves the array's device address there
+//    (cudaGetSymbolAddress, with that device current) and configures the
+//    kernels; make that first call before any stream capture.
+//  - It calls no cudaMalloc, cudaFree or other allocating routine.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "lags.h"
+#include "lags_internal.cuh"
+#include "lags_plan.cuh"
+
+namespace lags {
+cudaError_t configure_estimate();
+cudaError_t configure_select();
+}  // namespace lags
+
+using namespace lags;
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = 16u << 20;
+constexpr int kMaxDevices = 64;
+
+// Host code must not use g_static_scratch as an address: on the host it names
+// a shadow object, not device memory.  Kernels get g_scratch_dev[device].
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_setup_mutex;
+char* g_scratch_dev[kMaxDevices] = {};
+
+// Once per device, with that device current: the scratch array's device
+// address, the sm_100 check and the kernel attributes.
+lags_status scratch_for_current_device(char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LAGS_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return LAGS_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (!g_scratch_dev[dev]) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return LAGS_ERR_CUDA;
+    if (major != 10 || minor != 0) return LAGS_ERR_UNSUPPORTED_DEVICE;
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr)
+      return LAGS_ERR_CUDA;
+    if (configure_estimate() != cudaSuccess || configure_select() != cudaSuccess)
+      return LAGS_ERR_CUDA;
+    g_scratch_dev[dev] = (char*)ptr;
+  }
+  *out = g_scratch_dev[dev];
+  return LAGS_OK;
+}
+
+bool aligned_to(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+}  // namespace
+
+extern "C" lags_status lags_sparsify_static(lags_plan* plan, const float* const* grads,
+                                            float* const* residuals, float lr,
+                                            uint32_t* out_idx, float* out_val, void* stream) {
+  if (!plan || !grads || !residuals || !out_idx || !out_val) return LAGS_ERR_INVALID_ARG;
+  if (plan->ws_bytes > kStaticScratchBytes) return LAGS_ERR_WORKSPACE;
+  if (!aligned_to(out_idx, 4) || !aligned_to(out_val, 4)) return LAGS_ERR_ALIGNMENT;
+  WorkerPtrs wp;
+  std::memset(&wp, 0, sizeof(wp));
+  for (int p = 0; p < plan->P; ++p) {
+    if (!grads[p] || !residuals[p]) return LAGS_ERR_INVALID_ARG;
+    if (!aligned_to(grads[p], 16) || !aligned_to(residuals[p], 16)) return LAGS_ERR_ALIGNMENT;
+    wp.g[p] = grads[p];
+    wp.r[p] = residuals[p];
+  }
+  char* base = nullptr;
+  lags_status st = scratch_for_current_device(&base);
+  if (st != LAGS_OK) return st;
+
+  cudaStream_t s = (cudaStream_t)stream;
+  auto up = [&](size_t o, const void* src, size_t n) {
+    return n ? cudaMemcpyAsync(base + o, src, n, cudaMemcpyHostToDevice, s) : cudaSuccess;
+  };
+  cudaError_t e = up(plan->o_layers, plan->layers.data(), plan->layers.size() * sizeof(LayerDesc));
+  if (e == cudaSuccess) e = up(plan->o_tiles, plan->tiles.data(), plan->tiles.size() * sizeof(TileDesc));
+  if (e == cudaSuccess) e = up(plan->o_large, plan->sel_large.data(), plan->sel_large.size() * 4);
+  if (e == cudaSuccess) e = up(plan->o_small, plan->sel_small.data(), plan->sel_small.size() * 4);
+  if (e == cudaSuccess) e = up(plan->o_sparse, plan->sparse.data(), plan->sparse.size() * 4);
+  if (e == cudaSuccess) e = cudaMemsetAsync(base + plan->o_status, 0, kStatusWords * 4, s);
+  if (e != cudaSuccess) return LAGS_ERR_CUDA;
+
+  DevPlan dp;
+  bind_dev_plan(plan, base, &dp);
+  e = launch_estimate(dp, wp, lr, s);
+  if (e == cudaSuccess) e = launch_ef_capture(dp, wp, lr, out_idx, out_val, s);
+  if (e == cudaSuccess) e = launch_select(dp, wp, out_idx, out_val, s);
+  return e == cudaSuccess ? LAGS_OK : LAGS_ERR_CUDA;
+}
