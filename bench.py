@@ -230,7 +230,7 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     n_sparse = sum(1 for l, d in enumerate(w.sizes) if plan.layers[l][1] < d)
-    n_large = sum(1 for l, d in enumerate(w.sizes) if plan.layers[l][1] < d and d >= (1 << 20))
+    n_large = sum(1 for l, d in enumerate(w.sizes) if d > plan.layers[l][1] >= 4096)
     launches_per_step = (1 if n_sparse else 0) + 1 + (1 if n_sparse - n_large else 0) + \
         (1 if n_large else 0) + 3
 

@@ -19,6 +19,7 @@ namespace lags {
 __global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs wp, float lr) {
   extern __shared__ uint32_t s_keys[];  // kSampleMax
   __shared__ uint32_t s_hist[kBins];
+  __shared__ uint32_t s_chunk[kSampleMax / kSampleChunk];  // first element of each run
   __shared__ uint32_t s_tmp[kEstThreads + kEstThreads / 32 + 4];
 
   const uint32_t layer = dp.sparse[blockIdx.x];
@@ -30,16 +31,31 @@ __global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs
   const uint32_t nchunk = m / kSampleChunk;
 
   for (uint32_t i = threadIdx.x; i < kBins; i += kEstThreads) s_hist[i] = 0;
-  for (uint32_t i = threadIdx.x; i < m; i += kEstThreads) {
-    uint32_t e;
-    if (m == ld.d) {
-      e = ld.off + i;
-    } else {
-      uint32_t c = i / kSampleChunk, j = i % kSampleChunk;
-      e = ld.off + (uint32_t)((uint64_t)c * (ld.d - kSampleChunk) / (nchunk - 1)) + j;
+  // sample positions: the whole layer, or nchunk runs of kSampleChunk spread
+  // evenly over it
+  if (m != ld.d)
+    for (uint32_t c = threadIdx.x; c < nchunk; c += kEstThreads)
+      s_chunk[c] = ld.off + (uint32_t)((uint64_t)c * (ld.d - kSampleChunk) / (nchunk - 1));
+  __syncthreads();
+  constexpr uint32_t U = 8;  // loads per array in flight per thread
+  for (uint32_t i0 = 0; i0 < m; i0 += kEstThreads * U) {
+    float gv[U], rv[U];
+#pragma unroll
+    for (uint32_t u = 0; u < U; ++u) {
+      const uint32_t i = i0 + u * kEstThreads + threadIdx.x;
+      gv[u] = 0.f;
+      rv[u] = 0.f;
+      if (i < m) {
+        const uint32_t e = m == ld.d ? ld.off + i : s_chunk[i / kSampleChunk] + i % kSampleChunk;
+        gv[u] = __ldg(g + e);
+        rv[u] = __ldg(r + e);
+      }
     }
-    float acc = __fadd_rn(__ldg(r + e), __fmul_rn(lr, __ldg(g + e)));
-    s_keys[i] = mag_key(acc);
+#pragma unroll
+    for (uint32_t u = 0; u < U; ++u) {
+      const uint32_t i = i0 + u * kEstThreads + threadIdx.x;
+      if (i < m) s_keys[i] = mag_key(__fadd_rn(rv[u], __fmul_rn(lr, gv[u])));
+    }
   }
   __syncthreads();
 
@@ -52,7 +68,7 @@ __global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs
   __syncthreads();
   // level 1: bits 19..9 among keys of bin b0
   for (uint32_t i = threadIdx.x; i < m; i += kEstThreads) {
-    uint32_t k = s_keys[i];
+    const uint32_t k = s_keys[i];
     if ((k >> 20) == b0.bin) atomicAdd(&s_hist[(k >> 9) & 0x7FFu], 1u);
   }
   __syncthreads();

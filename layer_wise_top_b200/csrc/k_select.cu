@@ -76,6 +76,9 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
                                                float* __restrict__ out_val) {
   using C = Cluster<CL>;
   __shared__ SelectShared sh;
+  extern __shared__ __align__(16) uint32_t sel_stage[];  // kSelectStage idx, then values
+  uint32_t* stage_idx = sel_stage;
+  float* stage_val = reinterpret_cast<float*>(sel_stage + kSelectStage);
   const uint32_t rank = C::rank();
   const uint32_t layer = list[blockIdx.x / CL];
   const uint32_t p = blockIdx.y;
@@ -125,34 +128,87 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   const uint64_t cbase = (uint64_t)p * dp.C + ld.slot_base;
 
   // Visit this CTA's share in index order, NT entries per round; every thread
-  // calls fn once per round (valid or not), so fn may contain barriers.
-  auto traverse = [&](auto&& fn) {
-    if (fast) {
-      for (uint32_t w0 = ta; w0 < tb; w0 += kSelectWindow) {
-        const uint32_t nw = min(kSelectWindow, tb - w0);
-        constexpr int PER = kSelectWindow / NT;
-        uint32_t c[PER], s = 0;
+  // calls fn(valid, idx, val) once per round, so fn may contain barriers.
+  // `stream_candidates` walks the candidate slots tile by tile (gathering
+  // through a window of tile prefix sums); once the share has been copied to
+  // shared memory (`staged`) the walks read it from there.
+  auto stream_candidates = [&](auto&& fn) {
+    uint32_t seen = 0;  // candidates of earlier windows
+    for (uint32_t w0 = ta; w0 < tb; w0 += kSelectWindow) {
+      const uint32_t nw = min(kSelectWindow, tb - w0);
+      constexpr int PER = kSelectWindow / NT;
+      uint32_t c[PER], sum = 0;
 #pragma unroll
-        for (int i = 0; i < PER; ++i) {
-          const uint32_t q = tid * PER + i;
-          c[i] = q < nw ? cnt[w0 + q] : 0u;
-          s += c[i];
-        }
-        uint32_t wtotal;
-        uint32_t ex = block_excl_scan<NT>(s, sh.tmp, &wtotal);
+      for (int i = 0; i < PER; ++i) {
+        const uint32_t q = tid * PER + i;
+        c[i] = q < nw ? cnt[w0 + q] : 0u;
+        sum += c[i];
+      }
+      uint32_t wtotal;
+      uint32_t ex = block_excl_scan<NT>(sum, sh.tmp, &wtotal);
 #pragma unroll
-        for (int i = 0; i < PER; ++i) {
-          const uint32_t q = tid * PER + i;
-          if (q < nw) sh.tpre[q] = ex;
-          ex += c[i];
+      for (int i = 0; i < PER; ++i) {
+        const uint32_t q = tid * PER + i;
+        if (q < nw) sh.tpre[q] = ex;
+        ex += c[i];
+      }
+      __syncthreads();
+      for (uint32_t b = 0; b < wtotal; b += NT) {
+        const uint32_t v = b + tid;
+        const bool valid = v < wtotal;
+        uint32_t idx = 0;
+        float val = 0.f;
+        if (valid) {
+          uint32_t lo = 0, hi = nw - 1;
+          while (lo < hi) {
+            const uint32_t mid = (lo + hi + 1) >> 1;
+            if (sh.tpre[mid] <= v) lo = mid; else hi = mid - 1;
+          }
+          const uint64_t slot =
+              cbase + (uint64_t)(w0 + lo - ld.tile_begin) * cap + (v - sh.tpre[lo]);
+          idx = dp.cand_idx[slot];
+          val = dp.cand_val[slot];
         }
-        __syncthreads();
-        for (uint32_t b = 0; b < wtotal; b += NT) {
-          const uint32_t v = b + tid;
-          const bool valid = v < wtotal;
-          uint32_t idx = 0;
-          float val = 0.f;
-          if (valid) {
+        fn(valid, seen + v, idx, val);
+      }
+      seen += wtotal;
+      __syncthreads();
+    }
+  };
+  const bool staged = fast && my <= kSelectStage;
+  if (staged) {
+    // copy the share's candidates to shared memory in index order, 8 rounds of
+    // loads in flight per thread
+    uint32_t seen = 0;
+    for (uint32_t w0 = ta; w0 < tb; w0 += kSelectWindow) {
+      const uint32_t nw = min(kSelectWindow, tb - w0);
+      constexpr int PER = kSelectWindow / NT;
+      uint32_t c[PER], sum = 0;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const uint32_t q = tid * PER + i;
+        c[i] = q < nw ? cnt[w0 + q] : 0u;
+        sum += c[i];
+      }
+      uint32_t wtotal;
+      uint32_t ex = block_excl_scan<NT>(sum, sh.tmp, &wtotal);
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const uint32_t q = tid * PER + i;
+        if (q < nw) sh.tpre[q] = ex;
+        ex += c[i];
+      }
+      __syncthreads();
+      constexpr uint32_t U = 8;
+      for (uint32_t b = 0; b < wtotal; b += NT * U) {
+        uint32_t iv[U];
+        float fv[U];
+#pragma unroll
+        for (uint32_t u = 0; u < U; ++u) {
+          const uint32_t v = b + u * NT + tid;
+          iv[u] = 0;
+          fv[u] = 0.f;
+          if (v < wtotal) {
             uint32_t lo = 0, hi = nw - 1;
             while (lo < hi) {
               const uint32_t mid = (lo + hi + 1) >> 1;
@@ -160,13 +216,32 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
             }
             const uint64_t slot =
                 cbase + (uint64_t)(w0 + lo - ld.tile_begin) * cap + (v - sh.tpre[lo]);
-            idx = dp.cand_idx[slot];
-            val = dp.cand_val[slot];
+            iv[u] = dp.cand_idx[slot];
+            fv[u] = dp.cand_val[slot];
           }
-          fn(valid, idx, val);
         }
-        __syncthreads();
+#pragma unroll
+        for (uint32_t u = 0; u < U; ++u) {
+          const uint32_t v = b + u * NT + tid;
+          if (v < wtotal) {
+            stage_idx[seen + v] = iv[u];
+            stage_val[seen + v] = fv[u];
+          }
+        }
       }
+      seen += wtotal;
+      __syncthreads();
+    }
+  }
+  auto traverse = [&](auto&& fn) {
+    if (staged) {
+      for (uint32_t b = 0; b < my; b += NT) {
+        const uint32_t v = b + tid;
+        const bool valid = v < my;
+        fn(valid, valid ? stage_idx[v] : 0u, valid ? stage_val[v] : 0.f);
+      }
+    } else if (fast) {
+      stream_candidates([&](bool valid, uint32_t, uint32_t idx, float val) { fn(valid, idx, val); });
     } else {
       for (uint32_t b = ea; b < eb; b += NT) {
         const uint32_t e = b + tid;
@@ -185,8 +260,12 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
       const uint32_t key = mag_key(val);
       const bool m = valid && (mshift >= 32 || (key >> mshift) == mval);
       const uint32_t dig = m ? ((key >> dshift) & dmask) : 0xFFFFFFFFu;
-      const unsigned peers = __match_any_sync(kFull, dig);
-      if (m && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
+      if (fast) {  // candidates sit in the sparse tail: few collisions
+        if (m) atomicAdd(&sh.hist[dig], 1u);
+      } else {     // a whole layer: keys crowd into few bins, add once per warp and bin
+        const unsigned peers = __match_any_sync(kFull, dig);
+        if (m && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
+      }
     });
     __syncthreads();
     if constexpr (CL > 1) {
@@ -289,13 +368,21 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   C::sync();  // no CTA leaves while another may still read its shared memory
 }
 
-cudaError_t configure_select() { return cudaSuccess; }
+constexpr size_t kSelectDynSmem = 2 * kSelectStage * sizeof(uint32_t);
+
+cudaError_t configure_select() {
+  cudaError_t e = cudaFuncSetAttribute(k_select<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSelectDynSmem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_select<kSelectCluster>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelectDynSmem);
+}
 
 cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out_idx,
                           float* out_val, cudaStream_t s) {
   if (dp.n_small) {
     dim3 grid(dp.n_small, dp.P);
-    k_select<1><<<grid, NT, 0, s>>>(dp, wp, dp.sel_small, out_idx, out_val);
+    k_select<1><<<grid, NT, kSelectDynSmem, s>>>(dp, wp, dp.sel_small, out_idx, out_val);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -303,7 +390,7 @@ cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(dp.n_large * kSelectCluster, dp.P);
     cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = kSelectDynSmem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;

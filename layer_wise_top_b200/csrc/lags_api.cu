@@ -2,6 +2,7 @@
 // validation and the launches.  See include/lags.h for the contract.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -15,6 +16,7 @@
 namespace lags {
 cudaError_t configure_estimate();
 cudaError_t configure_select();
+cudaError_t configure_aggregate();
 }  // namespace lags
 
 using namespace lags;
@@ -123,7 +125,7 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
       ld.sample = (uint32_t)((uint64_t)d < kSampleMax ? d : kSampleMax);
       ld.rank = sample_rank(ld.sample, d, k);
       plan->sparse.push_back((uint32_t)l);
-      ((uint64_t)d >= kLargeLayer ? plan->sel_large : plan->sel_small).push_back((uint32_t)l);
+      (k >= kLargeK ? plan->sel_large : plan->sel_small).push_back((uint32_t)l);
     }
     if (slots >= (1ull << 32) || koff + k >= (1ull << 32)) {
       delete plan;
@@ -136,6 +138,13 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
     off += (uint64_t)d;
     koff += k;
   }
+  // select the layers with the most picks first, so the longest CTAs start early
+  auto by_k_desc = [plan](uint32_t a, uint32_t b) {
+    return plan->layers[a].k != plan->layers[b].k ? plan->layers[a].k > plan->layers[b].k : a < b;
+  };
+  std::sort(plan->sel_large.begin(), plan->sel_large.end(), by_k_desc);
+  std::sort(plan->sel_small.begin(), plan->sel_small.end(), by_k_desc);
+  std::sort(plan->sparse.begin(), plan->sparse.end(), by_k_desc);
   plan->N = off;
   plan->K = koff;
   plan->C = slots;
@@ -192,7 +201,8 @@ lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t byt
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
     return LAGS_ERR_CUDA;
   if (major != 10 || minor != 0) return LAGS_ERR_UNSUPPORTED_DEVICE;
-  if (configure_estimate() != cudaSuccess || configure_select() != cudaSuccess)
+  if (configure_estimate() != cudaSuccess || configure_select() != cudaSuccess ||
+      configure_aggregate() != cudaSuccess)
     return LAGS_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
   char* base = (char*)workspace;

@@ -25,7 +25,8 @@ constexpr uint32_t kEstThreads = 512;
 constexpr int kSelectCluster = 8;
 constexpr uint32_t kSelectThreads = 512;
 constexpr uint32_t kSelectWindow = 2048;  // tiles whose prefix sits in smem at once
-constexpr uint32_t kLargeLayer = 1u << 20;  // d_l at or above: clustered select
+constexpr uint32_t kSelectStage = 8192;   // candidates per CTA copied to smem
+constexpr uint32_t kLargeK = 4096;  // k_l at or above: clustered select
 
 // Radix digits of the magnitude key (bits 30..0 of the fp32 pattern).
 constexpr int kDigitShift0 = 20;  // level 0: bits 30..20, 2048 bins

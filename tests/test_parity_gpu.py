@@ -90,8 +90,9 @@ def test_ragged_layers_mixed_density(dist):
 
 
 def test_large_layers_cluster_select():
+    # k >= 4096 selects with an 8-CTA cluster, smaller k with one CTA
     sizes = [1_100_003, 5, 2_000_001, 1 << 20]
-    dens = [0.001, 1.0, 0.001, 0.01]
+    dens = [0.001, 1.0, 0.003, 0.01]
     w = WORKLOADS["lstm_ptb"].scaled("big", P=2, steps=3,
                                      tensors=[Tensor(f"t{i}", (d,)) for i, d in enumerate(sizes)])
     run_full_compare(sizes, dens, 2, w.lr, 3, synth_grad_fn(w),
@@ -107,17 +108,17 @@ def _np_grads(gen, sizes, P, steps):
 
 def test_integer_ties_force_exact_path():
     rng = np.random.default_rng(5)
-    sizes = [9000, 40000, 1_048_577, 17]
-    dens = [0.01, 0.001, 0.001, 0.3]
+    sizes = [9000, 40000, 1_048_577, 17, 600_000]
+    dens = [0.01, 0.001, 0.001, 0.3, 0.01]
     fn = _np_grads(lambda n: rng.integers(-2, 3, n).astype(F32), sizes, 2, 3)
     fb = run_full_compare(sizes, dens, 2, 1.0, 3, fn)
     assert fb > 0  # massive ties overflow the candidate slots
 
 
 def test_all_zero_gradients():
-    sizes = [100, 8192, 30000, 1_048_576]
+    sizes = [100, 8192, 30000, 1_048_576, 600_000]
     fn = _np_grads(lambda n: np.zeros(n, dtype=F32), sizes, 2, 2)
-    run_full_compare(sizes, [0.01, 0.001, 0.5, 0.001], 2, 0.1, 2, fn)
+    run_full_compare(sizes, [0.01, 0.001, 0.5, 0.001, 0.01], 2, 0.1, 2, fn)
 
 
 def test_signed_zero_denormal_inf():
