@@ -70,6 +70,8 @@ typedef enum {
 
 /* Bits of the device status word returned by lags_status_poll(). */
 #define LAGS_FLAG_BAD_PICKS 0x1u /* lags_aggregate saw an unsorted or out-of-layer index */
+#define LAGS_FLAG_TIMEOUT 0x4u   /* a kernel's bounded wait on its own bulk copies gave up;
+                                    the outputs of that call are incomplete */
 #define LAGS_FLAG_INTERNAL 0x2u  /* a selection kernel failed a self-check (a library bug);
                                     the write it guarded was skipped */
 

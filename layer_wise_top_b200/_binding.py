@@ -20,6 +20,7 @@ LAGS_ERR_BAD_PICKS = 6
 LAGS_MAX_WORKERS = 256
 LAGS_FLAG_BAD_PICKS = 0x1
 LAGS_FLAG_INTERNAL = 0x2
+LAGS_FLAG_TIMEOUT = 0x4
 
 EXPORTED = ("lags_plan_create", "lags_plan_destroy", "lags_plan_info", "lags_plan_layer",
             "lags_plan_set_workspace", "lags_sparsify", "lags_aggregate", "lags_apply",

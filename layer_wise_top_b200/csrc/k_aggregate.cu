@@ -69,7 +69,6 @@ __global__ void __launch_bounds__(256) k_pick_bounds(DevPlan dp, const uint32_t*
 constexpr uint32_t kAggPickCap = 4096;
 
 struct AggShared {
-  float out[kTile];               // the tile of the update
   uint16_t loc[kAggPickCap];      // pick position inside the tile, per worker ascending
   float val[kAggPickCap];
   uint32_t base[LAGS_MAX_WORKERS + 1];  // first staged pick of each worker
@@ -111,7 +110,18 @@ __global__ void __launch_bounds__(kAggThreads)
     return;
   }
 
-  for (uint32_t i = tid; i < td.len; i += kAggThreads) sh.out[i] = 0.0f;
+  // positions nobody picked are +0: write the whole tile as zeros first
+  // (16-byte stores where aligned); picked positions are overwritten below
+  // after a barrier, which orders the two writes
+  {
+    const uint32_t head = min(td.len, (4u - (td.start & 3u)) & 3u);
+    const uint32_t nvec = (td.len - head) / 4;
+    for (uint32_t i = tid; i < head; i += kAggThreads) dense[td.start + i] = 0.0f;
+    float4* d4 = reinterpret_cast<float4*>(dense + td.start + head);
+    for (uint32_t v = tid; v < nvec; v += kAggThreads) d4[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (uint32_t i = head + 4 * nvec + tid; i < td.len; i += kAggThreads)
+      dense[td.start + i] = 0.0f;
+  }
   const uint32_t kend = ld.koff + ld.k;
   uint32_t cnt = 0;
   if (tid < (int)P) {
@@ -150,7 +160,7 @@ __global__ void __launch_bounds__(kAggThreads)
     for (uint32_t i = tid; i < total; i += kAggThreads) {
       const uint32_t x = sh.loc[i];
       if (x >= td.len) continue;
-      uint32_t p = 0, hi = P - 1;  // worker of staged pick i: last p with base[p] <= i
+      uint32_t p = 0, hi = P - 1;  // worker of staged pick i
       while (p < hi) {
         const uint32_t m = (p + hi + 1) >> 1;
         if (sh.base[m] <= i) p = m; else hi = m - 1;
@@ -168,33 +178,22 @@ __global__ void __launch_bounds__(kAggThreads)
           else s = __fadd_rn(s, sh.val[at]);
         }
       }
-      if (first_owner) sh.out[x] = __fdiv_rn(s, fP);
+      if (first_owner) dense[td.start + x] = __fdiv_rn(s, fP);
     }
-    __syncthreads();
   } else {
-    // many picks in this tile: accumulate worker by worker in shared memory
+    // many picks in this tile: accumulate worker by worker in the output
+    // itself (the zeros above), one barrier between workers
     for (uint32_t p = 0; p < P; ++p) {
       const uint32_t a = sh.rng[2 * p], b = sh.rng[2 * p + 1];
       for (uint32_t j = a + tid; j < b; j += kAggThreads) {
         const uint32_t x = idx[p * K + j] - td.start;
-        if (x < td.len) sh.out[x] = __fadd_rn(sh.out[x], val[p * K + j]);
+        if (x < td.len) dense[td.start + x] = __fadd_rn(dense[td.start + x], val[p * K + j]);
       }
       __syncthreads();
     }
-    for (uint32_t i = tid; i < td.len; i += kAggThreads) sh.out[i] = __fdiv_rn(sh.out[i], fP);
-    __syncthreads();
+    for (uint32_t i = tid; i < td.len; i += kAggThreads)
+      dense[td.start + i] = __fdiv_rn(dense[td.start + i], fP);
   }
-  // write the tile out, 16 bytes per store where the tile is aligned
-  const uint32_t head = min(td.len, (4u - (td.start & 3u)) & 3u);
-  for (uint32_t i = tid; i < head; i += kAggThreads) dense[td.start + i] = sh.out[i];
-  const uint32_t nvec = (td.len - head) / 4;
-  float4* d4 = reinterpret_cast<float4*>(dense + td.start + head);
-  for (uint32_t v = tid; v < nvec; v += kAggThreads) {
-    const uint32_t i = head + 4 * v;
-    __stcs(d4 + v, make_float4(sh.out[i], sh.out[i + 1], sh.out[i + 2], sh.out[i + 3]));
-  }
-  for (uint32_t i = head + 4 * nvec + tid; i < td.len; i += kAggThreads)
-    dense[td.start + i] = sh.out[i];
 }
 
 __global__ void __launch_bounds__(256) k_apply(uint32_t N, float* __restrict__ w,

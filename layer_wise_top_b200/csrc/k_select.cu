@@ -62,7 +62,6 @@ struct Cluster {
 
 struct SelectShared {
   uint32_t hist[kBins];          // this CTA's histogram (then the merged copy)
-  uint32_t merged[3][kBins];     // CTA 0: cluster-wide histograms, one per level
   uint32_t tpre[kSelectWindow + 1];
   uint32_t tmp[NT + NT / 32 + 4];
   uint32_t xch[4];               // read by the other CTAs of the cluster
@@ -72,13 +71,16 @@ struct SelectShared {
 
 template <int CL>
 __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const uint32_t* list,
+                                               uint32_t stage_cap,
                                                uint32_t* __restrict__ out_idx,
                                                float* __restrict__ out_val) {
   using C = Cluster<CL>;
   __shared__ SelectShared sh;
-  extern __shared__ __align__(16) uint32_t sel_stage[];  // kSelectStage idx, then values
+  // CTA 0 of a cluster: cluster-wide histograms, one per level
+  __shared__ uint32_t merged[CL > 1 ? 3 : 1][kBins];
+  extern __shared__ __align__(16) uint32_t sel_stage[];  // stage_cap indices, then values
   uint32_t* stage_idx = sel_stage;
-  float* stage_val = reinterpret_cast<float*>(sel_stage + kSelectStage);
+  float* stage_val = reinterpret_cast<float*>(sel_stage + stage_cap);
   const uint32_t rank = C::rank();
   const uint32_t layer = list[blockIdx.x / CL];
   const uint32_t p = blockIdx.y;
@@ -88,9 +90,8 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
 
   for (int i = tid; i < (int)kBins; i += NT) {
     sh.hist[i] = 0;
-    sh.merged[0][i] = 0;
-    sh.merged[1][i] = 0;
-    sh.merged[2][i] = 0;
+#pragma unroll
+    for (int q = 0; q < (CL > 1 ? 3 : 1); ++q) merged[q][i] = 0;
   }
 
   // ---- mode: candidate lists or exhaustive ----
@@ -175,7 +176,7 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
       __syncthreads();
     }
   };
-  const bool staged = fast && my <= kSelectStage;
+  const bool staged = fast && my <= stage_cap;
   if (staged) {
     // copy the share's candidates to shared memory in index order, 8 rounds of
     // loads in flight per thread
@@ -255,8 +256,18 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   // One radix level: histogram of digit (key >> dshift) & dmask over the keys
   // whose prefix key >> mshift equals mval (all keys when mshift == 32),
   // merged across the cluster into sh.hist.
+  // staged share: thread tid owns the contiguous positions [cb, ce)
+  const uint32_t chunk = (my + NT - 1) / NT;
+  const uint32_t cb = min(my, tid * chunk), ce = min(my, cb + chunk);
+
   auto hist_level = [&](int level, int mshift, uint32_t mval, int dshift, uint32_t dmask) {
-    traverse([&](bool valid, uint32_t, float val) {
+    if (staged) {
+      for (uint32_t i = cb; i < ce; ++i) {
+        const uint32_t key = mag_key(stage_val[i]);
+        if (mshift >= 32 || (key >> mshift) == mval)
+          atomicAdd(&sh.hist[(key >> dshift) & dmask], 1u);
+      }
+    } else traverse([&](bool valid, uint32_t, float val) {
       const uint32_t key = mag_key(val);
       const bool m = valid && (mshift >= 32 || (key >> mshift) == mval);
       const uint32_t dig = m ? ((key >> dshift) & dmask) : 0xFFFFFFFFu;
@@ -269,13 +280,13 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
     });
     __syncthreads();
     if constexpr (CL > 1) {
-      uint32_t* dst = C::remote(sh.merged[level], 0);
+      uint32_t* dst = C::remote(merged[level], 0);
       for (int i = tid; i < (int)kBins; i += NT) {
         const uint32_t h = sh.hist[i];
         if (h) atomicAdd(dst + i, h);
       }
       C::sync();
-      const uint32_t* src = C::remote(sh.merged[level], 0);
+      const uint32_t* src = C::remote(merged[level], 0);
       for (int i = tid; i < (int)kBins; i += NT) sh.hist[i] = src[i];
       __syncthreads();
     }
@@ -315,14 +326,27 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   const uint32_t need = rem;
 
   // ---- count strict picks and ties of this CTA, exchange prefixes ----
-  uint32_t na = 0, nb = 0;
-  traverse([&](bool valid, uint32_t, float val) {
-    const uint32_t s = mag_key(val) >> fshift;
-    na += valid && s > fpfx;
-    nb += valid && s == fpfx;
-  });
-  na = block_sum<NT>(na, sh.tmp);
-  nb = block_sum<NT>(nb, sh.tmp);
+  uint32_t na = 0, nb = 0, my_ex = 0;
+  if (staged) {
+    uint32_t ca = 0, ct = 0;
+    for (uint32_t i = cb; i < ce; ++i) {
+      const uint32_t s = mag_key(stage_val[i]) >> fshift;
+      ca += s > fpfx;
+      ct += s == fpfx;
+    }
+    uint32_t tot;  // per-CTA counts <= stage_cap < 2^16: pack strict | ties
+    my_ex = block_excl_scan<NT>((ca << 16) | ct, sh.tmp, &tot);
+    na = tot >> 16;
+    nb = tot & 0xFFFFu;
+  } else {
+    traverse([&](bool valid, uint32_t, float val) {
+      const uint32_t s = mag_key(val) >> fshift;
+      na += valid && s > fpfx;
+      nb += valid && s == fpfx;
+    });
+    na = block_sum<NT>(na, sh.tmp);
+    nb = block_sum<NT>(nb, sh.tmp);
+  }
   if (tid == 0) {
     sh.xch[2] = na;
     sh.xch[3] = nb;
@@ -335,54 +359,62 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
     b_run += x[3];
   }
 
-  // ---- ordered emission ----
+  // ---- ordered emission: pos = strict_before + min(need, ties_before) ----
   const uint64_t ob = (uint64_t)p * dp.K + ld.koff;
-  traverse([&](bool valid, uint32_t idx, float val) {
-    const uint32_t s = mag_key(val) >> fshift;
-    const bool st = valid && s > fpfx;
-    const bool ti = valid && s == fpfx;
-    uint32_t tot;
-    const uint32_t ex = block_excl_scan<NT>(((uint32_t)st << 16) | (uint32_t)ti, sh.tmp, &tot);
-    const uint32_t at = a_run + (ex >> 16), bt = b_run + (ex & 0xFFFFu);
-    bool emit = false;
-    uint32_t pos = 0;
-    if (st) {
-      emit = true;
-      pos = at + min(need, bt);
-    } else if (ti && bt < need) {
-      emit = true;
-      pos = at + bt;
+  auto emit = [&](uint32_t pos, uint32_t idx, float val) {
+    if (pos < ld.k) {
+      out_idx[ob + pos] = idx;
+      out_val[ob + pos] = val;
+      r[idx] = 0.0f;
+    } else {
+      atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
     }
-    if (emit) {
-      if (pos < ld.k) {
-        out_idx[ob + pos] = idx;
-        out_val[ob + pos] = val;
-        r[idx] = 0.0f;
-      } else {
-        atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
+  };
+  if (staged) {
+    uint32_t at = a_run + (my_ex >> 16), bt = b_run + (my_ex & 0xFFFFu);
+    for (uint32_t i = cb; i < ce; ++i) {
+      const float val = stage_val[i];
+      const uint32_t s = mag_key(val) >> fshift;
+      if (s > fpfx) {
+        emit(at + min(need, bt), stage_idx[i], val);
+        ++at;
+      } else if (s == fpfx) {
+        if (bt < need) emit(at + bt, stage_idx[i], val);
+        ++bt;
       }
     }
-    a_run += tot >> 16;
-    b_run += tot & 0xFFFFu;
-  });
+  } else {
+    traverse([&](bool valid, uint32_t idx, float val) {
+      const uint32_t s = mag_key(val) >> fshift;
+      const bool st = valid && s > fpfx;
+      const bool ti = valid && s == fpfx;
+      uint32_t tot;
+      const uint32_t ex = block_excl_scan<NT>(((uint32_t)st << 16) | (uint32_t)ti, sh.tmp, &tot);
+      const uint32_t at = a_run + (ex >> 16), bt = b_run + (ex & 0xFFFFu);
+      if (st) emit(at + min(need, bt), idx, val);
+      else if (ti && bt < need) emit(at + bt, idx, val);
+      a_run += tot >> 16;
+      b_run += tot & 0xFFFFu;
+    });
+  }
   C::sync();  // no CTA leaves while another may still read its shared memory
 }
 
-constexpr size_t kSelectDynSmem = 2 * kSelectStage * sizeof(uint32_t);
-
 cudaError_t configure_select() {
+  const int most = (int)(2 * kSelectStageMax * sizeof(uint32_t));
   cudaError_t e = cudaFuncSetAttribute(k_select<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSelectDynSmem);
+                                       most);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(k_select<kSelectCluster>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelectDynSmem);
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, most);
 }
 
 cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out_idx,
                           float* out_val, cudaStream_t s) {
   if (dp.n_small) {
     dim3 grid(dp.n_small, dp.P);
-    k_select<1><<<grid, NT, kSelectDynSmem, s>>>(dp, wp, dp.sel_small, out_idx, out_val);
+    const size_t smem = 2 * dp.stage_small * sizeof(uint32_t);
+    k_select<1><<<grid, NT, smem, s>>>(dp, wp, dp.sel_small, dp.stage_small, out_idx, out_val);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -390,7 +422,7 @@ cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(dp.n_large * kSelectCluster, dp.P);
     cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = kSelectDynSmem;
+    cfg.dynamicSmemBytes = 2 * dp.stage_large * sizeof(uint32_t);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -400,7 +432,7 @@ cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, k_select<kSelectCluster>, dp, wp, dp.sel_large,
-                                       out_idx, out_val);
+                                       dp.stage_large, out_idx, out_val);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }

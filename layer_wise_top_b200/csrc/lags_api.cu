@@ -16,6 +16,7 @@
 namespace lags {
 cudaError_t configure_estimate();
 cudaError_t configure_select();
+cudaError_t configure_ef_stream();
 cudaError_t configure_aggregate();
 }  // namespace lags
 
@@ -42,13 +43,14 @@ uint32_t slot_capacity(uint64_t d, uint64_t k) {
   return (uint32_t)(c < kTile ? c : kTile);
 }
 
-// Sample rank r* for a sample of m entries out of d, k picks: 1.5x the
-// expected number of sampled entries above the k-th largest, plus four
-// standard deviations and a floor of 8.  A whole-layer sample uses r* = k.
+// Sample rank r* for a sample of m entries out of d, k picks: the expected
+// number mu of sampled entries above the k-th largest, plus four standard
+// deviations and a floor of 6, so the threshold it sets keeps the k largest
+// entries with overwhelming probability.  A whole-layer sample uses r* = k.
 uint32_t sample_rank(uint64_t m, uint64_t d, uint64_t k) {
   if (m == d) return (uint32_t)k;
   double mu = (double)m * (double)k / (double)d;
-  double r = std::ceil(1.5 * mu + 4.0 * std::sqrt(mu) + 8.0);
+  double r = std::ceil(mu + 4.0 * std::sqrt(mu) + 6.0);
   if (r > (double)m) r = (double)m;
   if (r < 1.0) r = 1.0;
   return (uint32_t)r;
@@ -138,6 +140,21 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
     off += (uint64_t)d;
     koff += k;
   }
+  // staging capacity of each select launch: 1.5x the largest expected
+  // candidate count of one CTA (the sample rank scaled to the layer) plus 512
+  auto stage_for = [plan](const std::vector<uint32_t>& list, uint32_t ctas) {
+    double most = 0.0;
+    for (uint32_t l : list) {
+      const LayerDesc& ld = plan->layers[l];
+      const double c = ld.sample == ld.d ? (double)ld.k
+                                         : std::ceil((double)ld.rank * ld.d / ld.sample);
+      most = std::max(most, c / ctas);
+    }
+    uint64_t cap = ((uint64_t)std::ceil(1.5 * most + 512.0) + 255) / 256 * 256;
+    return (uint32_t)std::min<uint64_t>(std::max<uint64_t>(cap, kSelectStageMin), kSelectStageMax);
+  };
+  plan->stage_small = stage_for(plan->sel_small, 1);
+  plan->stage_large = stage_for(plan->sel_large, kSelectCluster);
   // select the layers with the most picks first, so the longest CTAs start early
   auto by_k_desc = [plan](uint32_t a, uint32_t b) {
     return plan->layers[a].k != plan->layers[b].k ? plan->layers[a].k > plan->layers[b].k : a < b;
@@ -202,6 +219,7 @@ lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t byt
     return LAGS_ERR_CUDA;
   if (major != 10 || minor != 0) return LAGS_ERR_UNSUPPORTED_DEVICE;
   if (configure_estimate() != cudaSuccess || configure_select() != cudaSuccess ||
+      configure_ef_stream() != cudaSuccess ||
       configure_aggregate() != cudaSuccess)
     return LAGS_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
@@ -237,7 +255,7 @@ lags_status lags_sparsify(lags_plan* plan, const float* const* grads, float* con
   const bool timed = plan->ev_before && plan->ev_after;
   cudaError_t e = launch_estimate(plan->dp, wp, lr, s);
   if (e == cudaSuccess && timed) e = cudaEventRecord(plan->ev_before, s);
-  if (e == cudaSuccess) e = launch_ef_capture(plan->dp, wp, lr, out_idx, out_val, s);
+  if (e == cudaSuccess) e = launch_ef(plan->dp, wp, lr, out_idx, out_val, s);
   if (e == cudaSuccess && timed) e = cudaEventRecord(plan->ev_after, s);
   if (e == cudaSuccess) e = launch_select(plan->dp, wp, out_idx, out_val, s);
   return cuda_status(e);

@@ -25,7 +25,11 @@ constexpr uint32_t kEstThreads = 512;
 constexpr int kSelectCluster = 8;
 constexpr uint32_t kSelectThreads = 512;
 constexpr uint32_t kSelectWindow = 2048;  // tiles whose prefix sits in smem at once
-constexpr uint32_t kSelectStage = 8192;   // candidates per CTA copied to smem
+// Candidates one selection CTA copies to shared memory (sized per launch from
+// the expected candidate counts, at most kSelectStageMax); a CTA with more
+// reads them from global memory on every pass instead.
+constexpr uint32_t kSelectStageMin = 1024;
+constexpr uint32_t kSelectStageMax = 11264;
 constexpr uint32_t kLargeK = 4096;  // k_l at or above: clustered select
 
 // Radix digits of the magnitude key (bits 30..0 of the fp32 pattern).
@@ -84,18 +88,31 @@ struct DevPlan {
   uint32_t N;
   uint64_t K;
   uint64_t C;  // candidate slots per worker
+  uint32_t stage_small, stage_large;  // shared-memory staging capacity per select launch
 };
 
 // Launchers (each returns the launch's cudaError_t).
 cudaError_t launch_estimate(const DevPlan& dp, const WorkerPtrs& wp, float lr, cudaStream_t s);
 cudaError_t launch_ef_capture(const DevPlan& dp, const WorkerPtrs& wp, float lr,
                               uint32_t* out_idx, float* out_val, cudaStream_t s);
+cudaError_t launch_ef_stream(const DevPlan& dp, const WorkerPtrs& wp, float lr,
+                             uint32_t* out_idx, float* out_val, cudaStream_t s);
 cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out_idx,
                           float* out_val, cudaStream_t s);
 cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStream_t s);
 cudaError_t launch_aggregate(const DevPlan& dp, const uint32_t* idx, const float* val,
                              float* dense, cudaStream_t s);
 cudaError_t launch_apply(uint32_t N, float* w, const float* dense, cudaStream_t s);
+
+// The fused error-feedback pass used by lags_sparsify.
+inline cudaError_t launch_ef(const DevPlan& dp, const WorkerPtrs& wp, float lr, uint32_t* out_idx,
+                             float* out_val, cudaStream_t s) {
+#ifdef LAGS_EF_BULK_COPY
+  return launch_ef_stream(dp, wp, lr, out_idx, out_val, s);
+#else
+  return launch_ef_capture(dp, wp, lr, out_idx, out_val, s);
+#endif
+}
 
 // ------------------------------------------------------------------ helpers
 __device__ __forceinline__ uint32_t mag_key(float x) {

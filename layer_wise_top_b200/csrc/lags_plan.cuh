@@ -22,6 +22,7 @@ struct lags_plan {
   void* ws = nullptr;
   int device = -1;
   cudaEvent_t ev_before = nullptr, ev_after = nullptr;
+  uint32_t stage_small = 0, stage_large = 0;  // select staging capacity per launch
   lags::DevPlan dp{};  // device view once a workspace is bound
 };
 
@@ -51,4 +52,6 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.N = (uint32_t)plan->N;
   dp.K = plan->K;
   dp.C = plan->C;
+  dp.stage_small = plan->stage_small;
+  dp.stage_large = plan->stage_large;
 }

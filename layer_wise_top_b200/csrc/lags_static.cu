@@ -32,6 +32,7 @@
 namespace lags {
 cudaError_t configure_estimate();
 cudaError_t configure_select();
+cudaError_t configure_ef_stream();
 }  // namespace lags
 
 using namespace lags;
@@ -64,7 +65,8 @@ lags_status scratch_for_current_device(char** out) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr)
       return LAGS_ERR_CUDA;
-    if (configure_estimate() != cudaSuccess || configure_select() != cudaSuccess)
+    if (configure_estimate() != cudaSuccess || configure_select() != cudaSuccess ||
+      configure_ef_stream() != cudaSuccess)
       return LAGS_ERR_CUDA;
     g_scratch_dev[dev] = (char*)ptr;
   }
@@ -109,7 +111,7 @@ extern "C" lags_status lags_sparsify_static(lags_plan* plan, const float* const*
   DevPlan dp;
   bind_dev_plan(plan, base, &dp);
   e = launch_estimate(dp, wp, lr, s);
-  if (e == cudaSuccess) e = launch_ef_capture(dp, wp, lr, out_idx, out_val, s);
+  if (e == cudaSuccess) e = launch_ef(dp, wp, lr, out_idx, out_val, s);
   if (e == cudaSuccess) e = launch_select(dp, wp, out_idx, out_val, s);
   return e == cudaSuccess ? LAGS_OK : LAGS_ERR_CUDA;
 }
