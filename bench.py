@@ -229,15 +229,12 @@ def run_ours(args):
     weights = torch.zeros(N, dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
 
-    n_sparse = sum(1 for l, d in enumerate(w.sizes) if plan.layers[l][1] < d)
-    n_large = sum(1 for l, d in enumerate(w.sizes) if d > plan.layers[l][1] >= 4096)
-    launches_per_step = (1 if n_sparse else 0) + 1 + (1 if n_sparse - n_large else 0) + \
-        (1 if n_large else 0) + 3
+    n_sparsify, n_aggregate, _ = plan.kernel_launches()
+    launches_per_step = n_sparsify + n_aggregate
 
     def step(i):
         plan.sparsify(grads[i % pool], res, w.lr, idx, val)
-        plan.aggregate(idx, val, dense)
-        plan.apply(weights, dense)
+        plan.aggregate_apply(idx, val, dense, weights)
 
     for i in range(args.warmup):
         step(i)
@@ -290,8 +287,7 @@ def run_ours(args):
             for p in range(P):
                 dev_g[p].copy_(host[p], non_blocking=True)
             plan.sparsify(dev_g, res, w.lr, idx, val)
-            plan.aggregate(idx, val, dense)
-            plan.apply(weights, dense)
+            plan.aggregate_apply(idx, val, dense, weights)
             w_host.copy_(weights, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
@@ -330,7 +326,7 @@ def run_ours(args):
             w, parallelism=f"replicas x{world}", grad_pool_steps=pool,
             l2=f"inputs larger than L2: {12 * P * N / 1e9:.2f} GB streamed per step vs "
                f"{L2_BYTES / 1e6:.0f} MB L2",
-            step="lags_sparsify + lags_aggregate + lags_apply"),
+            step="lags_sparsify + lags_aggregate_apply (aggregate and apply fused)"),
         "roofline": {"kernel": "k_ef_capture", "bound": "hbm", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": None,

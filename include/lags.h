@@ -151,6 +151,17 @@ LAGS_API lags_status lags_aggregate(lags_plan* plan, const uint32_t* idx, const 
                            float* dense_out, void* stream);
 
 /*
+ * lags_aggregate_apply - lags_aggregate followed by lags_apply in one pass
+ * over the update: dense_out is written exactly as lags_aggregate writes it and
+ * weights end exactly as lags_apply leaves them (entries no worker picked
+ * keep their weight, since w - (+0) == w), without reading dense_out back.
+ *   weights    device float[N], 16-byte aligned, updated in place.
+ * Other arguments, layout and errors: as lags_aggregate.
+ */
+LAGS_API lags_status lags_aggregate_apply(lags_plan* plan, const uint32_t* idx, const float* val,
+                                          float* dense_out, float* weights, void* stream);
+
+/*
  * lags_apply - weights <- weights - dense_out over the plan's N elements.
  *   weights    device float[N], 16-byte aligned, updated in place.
  *   dense_out  device float[N], 16-byte aligned.
@@ -203,6 +214,14 @@ LAGS_API lags_status lags_sparsify_static(lags_plan* plan, const float* const* g
  * NULL, NULL to stop.  The events stay the caller's.
  */
 LAGS_API lags_status lags_plan_set_events(lags_plan* plan, void* before, void* after);
+
+/*
+ * lags_plan_kernel_launches - how many kernels one lags_sparsify, one
+ * lags_aggregate (or lags_aggregate_apply) and one lags_apply call enqueue for
+ * this plan (any output pointer may be NULL).
+ */
+LAGS_API lags_status lags_plan_kernel_launches(const lags_plan* plan, int32_t* sparsify,
+                                               int32_t* aggregate, int32_t* apply);
 
 /* Static, human-readable text for a status code. */
 LAGS_API const char* lags_error_string(lags_status status);

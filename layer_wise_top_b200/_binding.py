@@ -25,7 +25,7 @@ LAGS_FLAG_TIMEOUT = 0x4
 EXPORTED = ("lags_plan_create", "lags_plan_destroy", "lags_plan_info", "lags_plan_layer",
             "lags_plan_set_workspace", "lags_sparsify", "lags_aggregate", "lags_apply",
             "lags_status_poll", "lags_plan_set_events", "lags_sparsify_static",
-            "lags_error_string")
+            "lags_aggregate_apply", "lags_plan_kernel_launches", "lags_error_string")
 
 
 class LagsError(RuntimeError):
@@ -52,6 +52,9 @@ def _load() -> ctypes.CDLL:
                                   vp, vp, vp]
     lib.lags_aggregate.argtypes = [vp, vp, vp, vp, vp]
     lib.lags_apply.argtypes = [vp, vp, vp, vp]
+    lib.lags_aggregate_apply.argtypes = [vp, vp, vp, vp, vp, vp]
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    lib.lags_plan_kernel_launches.argtypes = [vp, i32p, i32p, i32p]
     lib.lags_status_poll.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32),
                                      ctypes.POINTER(ctypes.c_uint32), vp]
     lib.lags_plan_set_events.argtypes = [vp, vp, vp]
@@ -142,6 +145,20 @@ def lags_aggregate(plan, idx: int, val: int, dense_out: int, stream: int = 0) ->
     _check(_LIB.lags_aggregate(plan, ctypes.c_void_p(idx), ctypes.c_void_p(val),
                                ctypes.c_void_p(dense_out), ctypes.c_void_p(stream)),
            "lags_aggregate")
+
+
+def lags_aggregate_apply(plan, idx: int, val: int, dense_out: int, weights: int,
+                         stream: int = 0) -> None:
+    _check(_LIB.lags_aggregate_apply(plan, ctypes.c_void_p(idx), ctypes.c_void_p(val),
+                                     ctypes.c_void_p(dense_out), ctypes.c_void_p(weights),
+                                     ctypes.c_void_p(stream)), "lags_aggregate_apply")
+
+
+def lags_plan_kernel_launches(plan) -> Tuple[int, int, int]:
+    a, b, c = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(_LIB.lags_plan_kernel_launches(plan, ctypes.byref(a), ctypes.byref(b),
+                                          ctypes.byref(c)), "lags_plan_kernel_launches")
+    return a.value, b.value, c.value
 
 
 def lags_apply(plan, weights: int, dense_out: int, stream: int = 0) -> None:

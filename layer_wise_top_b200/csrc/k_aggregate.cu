@@ -3,15 +3,12 @@
 // Sparsified S-SGD ("Layer-wise Adaptive Gradient Sparsification ..." review,
 // abstract) sums the workers' sparse sets into one averaged dense update:
 // dense_j = ((+0 + v_0j) + v_1j + ... + v_(P-1)j) / P, workers in order, one
-// rounding per add, a correctly rounded division.  Every CTA owns one tile of
-// the flattened buffer and builds that tile of the update in shared memory.
-// It stages all workers' picks of the tile (each worker's list ascending);
-// for every position, the thread holding the lowest worker's pick of it finds
-// the other workers' picks by binary search and adds them in worker order.
-// Positions nobody picked stay +0.  Tiles with more picks than fit in shared
-// memory (layers sent at high density) accumulate worker by worker with a
-// barrier in between.  No atomics: the result is bit-identical however the
-// grid is scheduled.
+// rounding per add, a correctly rounded division; positions no worker picked
+// are +0.  One CTA per tile of the flattened buffer: it stages all workers'
+// picks of the tile in shared memory, then each thread sums its own span of
+// positions worker by worker.  No atomics and no cross-thread reduction, so the
+// result is bit-identical however the grid is scheduled.  With a weights
+// pointer the same kernel also applies the SGD update (weights -= dense).
 //
 // k_pick_bounds first turns each worker's ascending pick list into the slot of
 // the first pick of every tile, so each aggregation CTA reads only its own
@@ -28,15 +25,22 @@ __device__ __forceinline__ uint32_t tile_of(const LayerDesc& ld, uint32_t x) {
 }
 
 __global__ void __launch_bounds__(256) k_pick_bounds(DevPlan dp, const uint32_t* __restrict__ idx) {
-  const uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  __shared__ uint32_t s_layer0;
+  const uint64_t i0 = (uint64_t)blockIdx.x * blockDim.x;
+  const uint64_t i = i0 + threadIdx.x;
   const uint32_t p = blockIdx.y;
-  if (i >= dp.K) return;
-  // layer holding pick slot i: the last layer with koff <= i
-  uint32_t lo = 0, hi = dp.L - 1;
-  while (lo < hi) {
-    const uint32_t mid = (lo + hi + 1) >> 1;
-    if (dp.layers[mid].koff <= i) lo = mid; else hi = mid - 1;
+  if (threadIdx.x == 0) {  // layer holding the block's first slot: last layer with koff <= i0
+    uint32_t lo = 0, hi = dp.L - 1;
+    while (lo < hi) {
+      const uint32_t mid = (lo + hi + 1) >> 1;
+      if (dp.layers[mid].koff <= i0) lo = mid; else hi = mid - 1;
+    }
+    s_layer0 = lo;
   }
+  __syncthreads();
+  if (i >= dp.K) return;
+  uint32_t lo = s_layer0;  // slots are consecutive: step forward to this slot's layer
+  while (lo + 1 < dp.L && dp.layers[lo + 1].koff <= i) ++lo;
   const LayerDesc ld = dp.layers[lo];
   if (ld.k == ld.d) return;  // dense layer: slot of element e is koff + e - off
   const uint32_t* pi = idx + (uint64_t)p * dp.K;
@@ -64,33 +68,33 @@ __global__ void __launch_bounds__(256) k_pick_bounds(DevPlan dp, const uint32_t*
     for (uint32_t t = ti + 1; t < ld.tile_end; ++t) first[t] = ld.koff + ld.k;
 }
 
-// Picks of one tile that fit in shared memory at once; a tile with more picks
-// (layers sent at high density) is summed worker by worker instead.
+// Picks of one tile staged in shared memory; a tile with more picks (layers
+// sent at high density by many workers) reads them from global memory.
 constexpr uint32_t kAggPickCap = 4096;
+// Up to this many picks in a tile, the thread holding a position's first pick
+// looks the position up in the other workers' lists (binary search); above it,
+// and when the launch has room for a tile accumulator, the CTA adds the
+// workers' picks into shared memory one worker at a time instead.
+constexpr uint32_t kAggOwnerMax = 512;
 
 struct AggShared {
-  uint16_t loc[kAggPickCap];      // pick position inside the tile, per worker ascending
+  uint16_t loc[kAggPickCap];             // pick position inside the tile, per worker ascending
   float val[kAggPickCap];
-  uint32_t base[LAGS_MAX_WORKERS + 1];  // first staged pick of each worker
+  uint32_t base[LAGS_MAX_WORKERS + 1];   // first staged pick of each worker
   uint32_t rng[2 * LAGS_MAX_WORKERS];
   uint32_t warp[kAggThreads / 32];
 };
-
-// Lower bound of x in the ascending loc[a, b).
-__device__ __forceinline__ uint32_t lower_bound_loc(const uint16_t* loc, uint32_t a, uint32_t b,
-                                                    uint32_t x) {
-  while (a < b) {
-    const uint32_t m = (a + b) >> 1;
-    if (loc[m] < x) a = m + 1; else b = m;
-  }
-  return a;
-}
+struct AggTileAcc {                      // only in launches that may need it
+  float acc[kTile];
+  uint32_t hit[kTile / 32];              // bit i of word w: position 32 w + i was picked
+};
 
 __global__ void __launch_bounds__(kAggThreads)
     k_aggregate(DevPlan dp, const uint32_t* __restrict__ idx, const float* __restrict__ val,
-                float* __restrict__ dense) {
+                float* __restrict__ dense, float* __restrict__ weights, bool have_acc) {
   extern __shared__ __align__(16) unsigned char agg_smem[];
   AggShared& sh = *reinterpret_cast<AggShared*>(agg_smem);
+  AggTileAcc& ta = *reinterpret_cast<AggTileAcc*>(agg_smem + sizeof(AggShared));
   const uint32_t t = blockIdx.x;
   const TileDesc td = dp.tiles[t];
   const LayerDesc ld = dp.layers[td.layer];
@@ -105,23 +109,13 @@ __global__ void __launch_bounds__(kAggThreads)
     for (uint32_t i = tid; i < td.len; i += kAggThreads) {
       float s = 0.0f;
       for (uint32_t p = 0; p < P; ++p) s = __fadd_rn(s, val[p * K + s0 + i]);
-      dense[td.start + i] = __fdiv_rn(s, fP);
+      const float dv = __fdiv_rn(s, fP);
+      dense[td.start + i] = dv;
+      if (weights) weights[td.start + i] = __fsub_rn(weights[td.start + i], dv);
     }
     return;
   }
 
-  // positions nobody picked are +0: write the whole tile as zeros first
-  // (16-byte stores where aligned); picked positions are overwritten below
-  // after a barrier, which orders the two writes
-  {
-    const uint32_t head = min(td.len, (4u - (td.start & 3u)) & 3u);
-    const uint32_t nvec = (td.len - head) / 4;
-    for (uint32_t i = tid; i < head; i += kAggThreads) dense[td.start + i] = 0.0f;
-    float4* d4 = reinterpret_cast<float4*>(dense + td.start + head);
-    for (uint32_t v = tid; v < nvec; v += kAggThreads) d4[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (uint32_t i = head + 4 * nvec + tid; i < td.len; i += kAggThreads)
-      dense[td.start + i] = 0.0f;
-  }
   const uint32_t kend = ld.koff + ld.k;
   uint32_t cnt = 0;
   if (tid < (int)P) {
@@ -139,32 +133,38 @@ __global__ void __launch_bounds__(kAggThreads)
   if (tid < (int)P) sh.base[tid] = before;
   if (tid == 0) sh.base[P] = total;
   __syncthreads();
-
-  if (total <= kAggPickCap) {
-    // stage every worker's picks of this tile (each list ascending); staged
-    // pick i belongs to the last worker p with base[p] <= i
+  auto worker_of = [&](uint32_t i) {  // staged pick i: last worker p with base[p] <= i
+    uint32_t p = 0, hi = P - 1;
+    while (p < hi) {
+      const uint32_t m = (p + hi + 1) >> 1;
+      if (sh.base[m] <= i) p = m; else hi = m - 1;
+    }
+    return p;
+  };
+  const bool staged = total <= kAggPickCap;
+  if (staged) {
     for (uint32_t i = tid; i < total; i += kAggThreads) {
-      uint32_t p = 0, hi = P - 1;
-      while (p < hi) {
-        const uint32_t m = (p + hi + 1) >> 1;
-        if (sh.base[m] <= i) p = m; else hi = m - 1;
-      }
+      const uint32_t p = worker_of(i);
       const uint64_t slot = p * K + sh.rng[2 * p] + (i - sh.base[p]);
       const uint32_t x = idx[slot] - td.start;
       sh.loc[i] = (uint16_t)(x < td.len ? x : 0xFFFFu);
       sh.val[i] = val[slot];
     }
-    __syncthreads();
-    // the first worker that picked a position sums all workers' values for it
-    // in worker order, then divides by P
+  }
+  const uint32_t head = min(td.len, (4u - (td.start & 3u)) & 3u);
+  const uint32_t nvec = (td.len - head) / 4;
+
+  if (staged && (total <= kAggOwnerMax || !have_acc)) {
+    // ---- few picks: zeros everywhere, then each position's first owner ----
+    for (uint32_t i = tid; i < head; i += kAggThreads) dense[td.start + i] = 0.0f;
+    float4* d4 = reinterpret_cast<float4*>(dense + td.start + head);
+    for (uint32_t v = tid; v < nvec; v += kAggThreads) __stcs(d4 + v, make_float4(0.f, 0.f, 0.f, 0.f));
+    for (uint32_t i = head + 4 * nvec + tid; i < td.len; i += kAggThreads) dense[td.start + i] = 0.0f;
+    __syncthreads();  // orders the zeros before the sums written below
     for (uint32_t i = tid; i < total; i += kAggThreads) {
       const uint32_t x = sh.loc[i];
       if (x >= td.len) continue;
-      uint32_t p = 0, hi = P - 1;  // worker of staged pick i
-      while (p < hi) {
-        const uint32_t m = (p + hi + 1) >> 1;
-        if (sh.base[m] <= i) p = m; else hi = m - 1;
-      }
+      const uint32_t p = worker_of(i);
       bool first_owner = true;
       float s = 0.0f;
       for (uint32_t q = 0; q < P && first_owner; ++q) {
@@ -172,27 +172,100 @@ __global__ void __launch_bounds__(kAggThreads)
           s = __fadd_rn(s, sh.val[i]);
           continue;
         }
-        const uint32_t at = lower_bound_loc(sh.loc, sh.base[q], sh.base[q + 1], x);
-        if (at < sh.base[q + 1] && sh.loc[at] == x) {
+        uint32_t a = sh.base[q], b = sh.base[q + 1];
+        while (a < b) {  // lower bound of x in worker q's staged picks
+          const uint32_t m = (a + b) >> 1;
+          if (sh.loc[m] < x) a = m + 1; else b = m;
+        }
+        if (a < sh.base[q + 1] && sh.loc[a] == x) {
           if (q < p) first_owner = false;
-          else s = __fadd_rn(s, sh.val[at]);
+          else s = __fadd_rn(s, sh.val[a]);
         }
       }
-      if (first_owner) dense[td.start + x] = __fdiv_rn(s, fP);
+      if (first_owner) {
+        const float dv = __fdiv_rn(s, fP);
+        dense[td.start + x] = dv;
+        if (weights) weights[td.start + x] = __fsub_rn(weights[td.start + x], dv);
+      }
     }
-  } else {
-    // many picks in this tile: accumulate worker by worker in the output
-    // itself (the zeros above), one barrier between workers
+    return;
+  }
+
+  if (have_acc) {
+    // ---- many picks: worker-ordered accumulation in a shared tile ----
+    for (uint32_t i = tid; i < kTile; i += kAggThreads) ta.acc[i] = 0.0f;
+    for (uint32_t i = tid; i < kTile / 32; i += kAggThreads) ta.hit[i] = 0;
+    __syncthreads();
     for (uint32_t p = 0; p < P; ++p) {
-      const uint32_t a = sh.rng[2 * p], b = sh.rng[2 * p + 1];
-      for (uint32_t j = a + tid; j < b; j += kAggThreads) {
-        const uint32_t x = idx[p * K + j] - td.start;
-        if (x < td.len) dense[td.start + x] = __fadd_rn(dense[td.start + x], val[p * K + j]);
+      if (staged) {
+        for (uint32_t j = sh.base[p] + tid; j < sh.base[p + 1]; j += kAggThreads) {
+          const uint32_t x = sh.loc[j];
+          if (x >= td.len) continue;
+          ta.acc[x] = __fadd_rn(ta.acc[x], sh.val[j]);
+          atomicOr(&ta.hit[x / 32], 1u << (x % 32));
+        }
+      } else {
+        const uint64_t row = p * K;
+        for (uint32_t j = sh.rng[2 * p] + tid; j < sh.rng[2 * p + 1]; j += kAggThreads) {
+          const uint32_t x = idx[row + j] - td.start;
+          if (x >= td.len) continue;
+          ta.acc[x] = __fadd_rn(ta.acc[x], val[row + j]);
+          atomicOr(&ta.hit[x / 32], 1u << (x % 32));
+        }
       }
       __syncthreads();
     }
-    for (uint32_t i = tid; i < td.len; i += kAggThreads)
-      dense[td.start + i] = __fdiv_rn(dense[td.start + i], fP);
+    auto picked = [&](uint32_t i) -> bool { return (ta.hit[i / 32] >> (i % 32)) & 1u; };
+    auto value_at = [&](uint32_t i) -> float {
+      return picked(i) ? __fdiv_rn(ta.acc[i], fP) : 0.0f;
+    };
+    for (uint32_t i = tid; i < head; i += kAggThreads) {
+      const float q = value_at(i);
+      dense[td.start + i] = q;
+      if (weights && picked(i)) weights[td.start + i] = __fsub_rn(weights[td.start + i], q);
+    }
+    float4* d4 = reinterpret_cast<float4*>(dense + td.start + head);
+    float4* w4 = weights ? reinterpret_cast<float4*>(weights + td.start + head) : nullptr;
+    for (uint32_t v = tid; v < nvec; v += kAggThreads) {
+      const uint32_t i = head + 4 * v;
+      const float4 q = make_float4(value_at(i), value_at(i + 1), value_at(i + 2), value_at(i + 3));
+      __stcs(d4 + v, q);
+      if (w4 && (picked(i) || picked(i + 1) || picked(i + 2) || picked(i + 3))) {
+        float4 wv = w4[v];  // 16-byte aligned: weights and dense share the layout
+        if (picked(i)) wv.x = __fsub_rn(wv.x, q.x);
+        if (picked(i + 1)) wv.y = __fsub_rn(wv.y, q.y);
+        if (picked(i + 2)) wv.z = __fsub_rn(wv.z, q.z);
+        if (picked(i + 3)) wv.w = __fsub_rn(wv.w, q.w);
+        w4[v] = wv;
+      }
+    }
+    for (uint32_t i = head + 4 * nvec + tid; i < td.len; i += kAggThreads) {
+      const float q = value_at(i);
+      dense[td.start + i] = q;
+      if (weights && picked(i)) weights[td.start + i] = __fsub_rn(weights[td.start + i], q);
+    }
+    return;
+  }
+
+  // ---- more picks than the stage holds and no tile accumulator: accumulate
+  // worker by worker in the output itself, a barrier between workers ----
+  for (uint32_t i = tid; i < td.len; i += kAggThreads) dense[td.start + i] = 0.0f;
+  __syncthreads();
+  for (uint32_t p = 0; p < P; ++p) {
+    const uint64_t row = p * K;
+    for (uint32_t j = sh.rng[2 * p] + tid; j < sh.rng[2 * p + 1]; j += kAggThreads) {
+      const uint32_t x = idx[row + j] - td.start;
+      if (x < td.len) dense[td.start + x] = __fadd_rn(dense[td.start + x], val[row + j]);
+    }
+    __syncthreads();
+  }
+  for (uint32_t i = tid; i < td.len; i += kAggThreads) {
+    const float s = dense[td.start + i];
+    if (s != 0.0f) {  // +0 stays +0 (0 / P), and w - (+0) == w
+      const float dv = __fdiv_rn(s, fP);
+      dense[td.start + i] = dv;
+      if (weights) weights[td.start + i] = __fsub_rn(weights[td.start + i], dv);
+    }
   }
 }
 
@@ -223,12 +296,13 @@ cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStrea
 
 cudaError_t configure_aggregate() {
   return cudaFuncSetAttribute(k_aggregate, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)sizeof(AggShared));
+                              (int)(sizeof(AggShared) + sizeof(AggTileAcc)));
 }
 
 cudaError_t launch_aggregate(const DevPlan& dp, const uint32_t* idx, const float* val,
-                             float* dense, cudaStream_t s) {
-  k_aggregate<<<dp.T, kAggThreads, sizeof(AggShared), s>>>(dp, idx, val, dense);
+                             float* dense, float* weights, cudaStream_t s) {
+  const size_t smem = sizeof(AggShared) + (dp.agg_tile_acc ? sizeof(AggTileAcc) : 0);
+  k_aggregate<<<dp.T, kAggThreads, smem, s>>>(dp, idx, val, dense, weights, dp.agg_tile_acc != 0);
   return cudaGetLastError();
 }
 

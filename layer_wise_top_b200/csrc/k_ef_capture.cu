@@ -19,7 +19,12 @@
 
 namespace lags {
 
-__device__ __forceinline__ float4 ld_stream(const float* p) {
+// Streaming (evict-first) loads and stores: each byte is touched once.  Plain
+// loads/stores measured 13% slower and L2 256-byte prefetch hints no faster.
+__device__ __forceinline__ float4 ld_grad(const float* p) {
+  return __ldcs(reinterpret_cast<const float4*>(p));
+}
+__device__ __forceinline__ float4 ld_resid(const float* p) {
   return __ldcs(reinterpret_cast<const float4*>(p));
 }
 __device__ __forceinline__ void st_stream(float* p, float4 v) {
@@ -29,7 +34,10 @@ __device__ __forceinline__ float comp(const float4& v, int j) {
   return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
 }
 
-__global__ void __launch_bounds__(kEfThreads) k_ef_capture(DevPlan dp, WorkerPtrs wp, float lr,
+// Three CTAs per SM: the 16 float4 loads of a thread stay in flight together
+// (about 80 registers), which measured 1.2x faster than four CTAs with loads
+// interleaved with arithmetic and than two CTAs with all loads in flight.
+__global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, WorkerPtrs wp, float lr,
                                                            uint32_t* __restrict__ out_idx,
                                                            float* __restrict__ out_val) {
   constexpr int V = kEfVecPerThread;
@@ -49,25 +57,31 @@ __global__ void __launch_bounds__(kEfThreads) k_ef_capture(DevPlan dp, WorkerPtr
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
   float4 a[V];
+  float4 gv[V];
+  // every load of the tile is issued before any arithmetic
 #pragma unroll
   for (int v = 0; v < V; ++v) {
     const uint32_t e0 = base + 4u * (v * kEfThreads + threadIdx.x);
-    float4 gv = make_float4(0.f, 0.f, 0.f, 0.f), rv = gv;
+    gv[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    a[v] = gv[v];
     if (e0 < end) {
       if (e0 + 4 <= N) {
-        gv = ld_stream(g + e0);
-        rv = ld_stream(r + e0);
+        gv[v] = ld_grad(g + e0);
+        a[v] = ld_resid(r + e0);
       } else {
-        gv.x = g[e0];
-        rv.x = r[e0];
-        if (e0 + 1 < N) { gv.y = g[e0 + 1]; rv.y = r[e0 + 1]; }
-        if (e0 + 2 < N) { gv.z = g[e0 + 2]; rv.z = r[e0 + 2]; }
+        gv[v].x = g[e0];
+        a[v].x = r[e0];
+        if (e0 + 1 < N) { gv[v].y = g[e0 + 1]; a[v].y = r[e0 + 1]; }
+        if (e0 + 2 < N) { gv[v].z = g[e0 + 2]; a[v].z = r[e0 + 2]; }
       }
     }
-    a[v].x = __fadd_rn(rv.x, __fmul_rn(lr, gv.x));
-    a[v].y = __fadd_rn(rv.y, __fmul_rn(lr, gv.y));
-    a[v].z = __fadd_rn(rv.z, __fmul_rn(lr, gv.z));
-    a[v].w = __fadd_rn(rv.w, __fmul_rn(lr, gv.w));
+  }
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    a[v].x = __fadd_rn(a[v].x, __fmul_rn(lr, gv[v].x));
+    a[v].y = __fadd_rn(a[v].y, __fmul_rn(lr, gv[v].y));
+    a[v].z = __fadd_rn(a[v].z, __fmul_rn(lr, gv[v].z));
+    a[v].w = __fadd_rn(a[v].w, __fmul_rn(lr, gv[v].w));
   }
 
   if (ld.k == ld.d) {

@@ -78,9 +78,7 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   __shared__ SelectShared sh;
   // CTA 0 of a cluster: cluster-wide histograms, one per level
   __shared__ uint32_t merged[CL > 1 ? 3 : 1][kBins];
-  extern __shared__ __align__(16) uint32_t sel_stage[];  // stage_cap indices, then values
-  uint32_t* stage_idx = sel_stage;
-  float* stage_val = reinterpret_cast<float*>(sel_stage + stage_cap);
+  extern __shared__ __align__(16) float stage_val[];  // stage_cap candidate values
   const uint32_t rank = C::rank();
   const uint32_t layer = list[blockIdx.x / CL];
   const uint32_t p = blockIdx.y;
@@ -176,72 +174,59 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
       __syncthreads();
     }
   };
-  const bool staged = fast && my <= stage_cap;
+  // Staged share: the values of this CTA's candidates, in index order, copied
+  // once to shared memory (the tile prefix sums stay in sh.tpre, so a staged
+  // position maps back to its candidate slot for the index at emission).
+  const bool staged = fast && my <= stage_cap && tb - ta <= kSelectWindow;
   if (staged) {
-    // copy the share's candidates to shared memory in index order, 8 rounds of
-    // loads in flight per thread
-    uint32_t seen = 0;
-    for (uint32_t w0 = ta; w0 < tb; w0 += kSelectWindow) {
-      const uint32_t nw = min(kSelectWindow, tb - w0);
-      constexpr int PER = kSelectWindow / NT;
-      uint32_t c[PER], sum = 0;
+    const uint32_t nw = tb - ta;
+    constexpr int PER = kSelectWindow / NT;
+    uint32_t c[PER], sum = 0;
 #pragma unroll
-      for (int i = 0; i < PER; ++i) {
-        const uint32_t q = tid * PER + i;
-        c[i] = q < nw ? cnt[w0 + q] : 0u;
-        sum += c[i];
-      }
-      uint32_t wtotal;
-      uint32_t ex = block_excl_scan<NT>(sum, sh.tmp, &wtotal);
-#pragma unroll
-      for (int i = 0; i < PER; ++i) {
-        const uint32_t q = tid * PER + i;
-        if (q < nw) sh.tpre[q] = ex;
-        ex += c[i];
-      }
-      __syncthreads();
-      constexpr uint32_t U = 8;
-      for (uint32_t b = 0; b < wtotal; b += NT * U) {
-        uint32_t iv[U];
-        float fv[U];
-#pragma unroll
-        for (uint32_t u = 0; u < U; ++u) {
-          const uint32_t v = b + u * NT + tid;
-          iv[u] = 0;
-          fv[u] = 0.f;
-          if (v < wtotal) {
-            uint32_t lo = 0, hi = nw - 1;
-            while (lo < hi) {
-              const uint32_t mid = (lo + hi + 1) >> 1;
-              if (sh.tpre[mid] <= v) lo = mid; else hi = mid - 1;
-            }
-            const uint64_t slot =
-                cbase + (uint64_t)(w0 + lo - ld.tile_begin) * cap + (v - sh.tpre[lo]);
-            iv[u] = dp.cand_idx[slot];
-            fv[u] = dp.cand_val[slot];
-          }
-        }
-#pragma unroll
-        for (uint32_t u = 0; u < U; ++u) {
-          const uint32_t v = b + u * NT + tid;
-          if (v < wtotal) {
-            stage_idx[seen + v] = iv[u];
-            stage_val[seen + v] = fv[u];
-          }
-        }
-      }
-      seen += wtotal;
-      __syncthreads();
+    for (int i = 0; i < PER; ++i) {
+      const uint32_t q = tid * PER + i;
+      c[i] = q < nw ? cnt[ta + q] : 0u;
+      sum += c[i];
     }
-  }
-  auto traverse = [&](auto&& fn) {
-    if (staged) {
-      for (uint32_t b = 0; b < my; b += NT) {
-        const uint32_t v = b + tid;
-        const bool valid = v < my;
-        fn(valid, valid ? stage_idx[v] : 0u, valid ? stage_val[v] : 0.f);
+    uint32_t wtotal;
+    uint32_t ex = block_excl_scan<NT>(sum, sh.tmp, &wtotal);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const uint32_t q = tid * PER + i;
+      if (q < nw) sh.tpre[q] = ex;
+      ex += c[i];
+    }
+    if (tid == 0) sh.tpre[nw] = wtotal;
+    __syncthreads();
+    constexpr uint32_t U = 8;  // loads in flight per thread
+    for (uint32_t b = 0; b < wtotal; b += NT * U) {
+      float fv[U];
+#pragma unroll
+      for (uint32_t u = 0; u < U; ++u) {
+        const uint32_t v = b + u * NT + tid;
+        fv[u] = 0.f;
+        if (v < wtotal) {
+          uint32_t lo = 0, hi = nw - 1;
+          while (lo < hi) {
+            const uint32_t mid = (lo + hi + 1) >> 1;
+            if (sh.tpre[mid] <= v) lo = mid; else hi = mid - 1;
+          }
+          fv[u] = dp.cand_val[cbase + (uint64_t)(ta + lo - ld.tile_begin) * cap +
+                              (v - sh.tpre[lo])];
+        }
       }
-    } else if (fast) {
+#pragma unroll
+      for (uint32_t u = 0; u < U; ++u) {
+        const uint32_t v = b + u * NT + tid;
+        if (v < wtotal) stage_val[v] = fv[u];
+      }
+    }
+    __syncthreads();
+  }
+  // Unstaged shares: every pass walks the candidates (or, on the exhaustive
+  // path, the layer's acc) from global memory.
+  auto traverse = [&](auto&& fn) {
+    if (fast) {
       stream_candidates([&](bool valid, uint32_t, uint32_t idx, float val) { fn(valid, idx, val); });
     } else {
       for (uint32_t b = ea; b < eb; b += NT) {
@@ -372,16 +357,26 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   };
   if (staged) {
     uint32_t at = a_run + (my_ex >> 16), bt = b_run + (my_ex & 0xFFFFu);
+    uint32_t tl = 0;  // tile (relative to ta) holding staged position cb
+    {
+      uint32_t hi = tb - ta - 1;
+      while (tl < hi) {
+        const uint32_t mid = (tl + hi + 1) >> 1;
+        if (sh.tpre[mid] <= cb) tl = mid; else hi = mid - 1;
+      }
+    }
     for (uint32_t i = cb; i < ce; ++i) {
+      while (sh.tpre[tl + 1] <= i) ++tl;
       const float val = stage_val[i];
       const uint32_t s = mag_key(val) >> fshift;
-      if (s > fpfx) {
-        emit(at + min(need, bt), stage_idx[i], val);
-        ++at;
-      } else if (s == fpfx) {
-        if (bt < need) emit(at + bt, stage_idx[i], val);
-        ++bt;
+      const bool st = s > fpfx, ti = s == fpfx && bt < need;
+      if (st || ti) {
+        const uint32_t idx =
+            dp.cand_idx[cbase + (uint64_t)(ta + tl - ld.tile_begin) * cap + (i - sh.tpre[tl])];
+        emit(st ? at + min(need, bt) : at + bt, idx, val);
       }
+      at += st;
+      bt += s == fpfx;
     }
   } else {
     traverse([&](bool valid, uint32_t idx, float val) {
@@ -401,7 +396,7 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
 }
 
 cudaError_t configure_select() {
-  const int most = (int)(2 * kSelectStageMax * sizeof(uint32_t));
+  const int most = (int)(kSelectStageMax * sizeof(float));
   cudaError_t e = cudaFuncSetAttribute(k_select<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        most);
   if (e != cudaSuccess) return e;
@@ -413,7 +408,7 @@ cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out
                           float* out_val, cudaStream_t s) {
   if (dp.n_small) {
     dim3 grid(dp.n_small, dp.P);
-    const size_t smem = 2 * dp.stage_small * sizeof(uint32_t);
+    const size_t smem = dp.stage_small * sizeof(float);
     k_select<1><<<grid, NT, smem, s>>>(dp, wp, dp.sel_small, dp.stage_small, out_idx, out_val);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -422,7 +417,7 @@ cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(dp.n_large * kSelectCluster, dp.P);
     cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = 2 * dp.stage_large * sizeof(uint32_t);
+    cfg.dynamicSmemBytes = dp.stage_large * sizeof(float);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;

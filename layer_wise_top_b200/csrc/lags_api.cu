@@ -56,6 +56,13 @@ uint32_t sample_rank(uint64_t m, uint64_t d, uint64_t k) {
   return (uint32_t)r;
 }
 
+// Candidates the fused pass is expected to keep for a layer: its sample rank
+// scaled from the sample to the layer (exactly k when the sample is the layer).
+double expected_candidates(const LayerDesc& ld) {
+  if (ld.sample == ld.d) return (double)ld.k;
+  return std::ceil((double)ld.rank * ld.d / ld.sample);
+}
+
 lags_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LAGS_OK : LAGS_ERR_CUDA; }
 
 bool fill_workers(const lags_plan* plan, const float* const* grads, float* const* residuals,
@@ -127,7 +134,11 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
       ld.sample = (uint32_t)((uint64_t)d < kSampleMax ? d : kSampleMax);
       ld.rank = sample_rank(ld.sample, d, k);
       plan->sparse.push_back((uint32_t)l);
-      (k >= kLargeK ? plan->sel_large : plan->sel_small).push_back((uint32_t)l);
+      // one CTA when its shared memory can stage the expected candidates with
+      // a third to spare, else an 8-CTA cluster
+      const double expect = expected_candidates(ld);
+      (1.33 * expect + 512.0 <= (double)kSelectStageMax ? plan->sel_small : plan->sel_large)
+          .push_back((uint32_t)l);
     }
     if (slots >= (1ull << 32) || koff + k >= (1ull << 32)) {
       delete plan;
@@ -144,15 +155,18 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
   // candidate count of one CTA (the sample rank scaled to the layer) plus 512
   auto stage_for = [plan](const std::vector<uint32_t>& list, uint32_t ctas) {
     double most = 0.0;
-    for (uint32_t l : list) {
-      const LayerDesc& ld = plan->layers[l];
-      const double c = ld.sample == ld.d ? (double)ld.k
-                                         : std::ceil((double)ld.rank * ld.d / ld.sample);
-      most = std::max(most, c / ctas);
-    }
+    for (uint32_t l : list) most = std::max(most, expected_candidates(plan->layers[l]) / ctas);
     uint64_t cap = ((uint64_t)std::ceil(1.5 * most + 512.0) + 255) / 256 * 256;
     return (uint32_t)std::min<uint64_t>(std::max<uint64_t>(cap, kSelectStageMin), kSelectStageMax);
   };
+  // aggregation: a tile of a sparse layer is expected to hold P * k * kTile / d
+  // picks; past a few hundred, worker-ordered accumulation in a shared tile
+  // beats looking each position up in every worker's list
+  for (uint32_t l : plan->sparse) {
+    const LayerDesc& ld = plan->layers[l];
+    if ((double)num_workers * ld.k * std::min<double>(kTile, ld.d) / ld.d > 256.0)
+      plan->agg_tile_acc = 1;
+  }
   plan->stage_small = stage_for(plan->sel_small, 1);
   plan->stage_large = stage_for(plan->sel_large, kSelectCluster);
   // select the layers with the most picks first, so the longest CTAs start early
@@ -268,8 +282,32 @@ lags_status lags_aggregate(lags_plan* plan, const uint32_t* idx, const float* va
   if (!aligned(idx, 4) || !aligned(val, 4) || !aligned(dense_out, 16)) return LAGS_ERR_ALIGNMENT;
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = launch_pick_bounds(plan->dp, idx, s);
-  if (e == cudaSuccess) e = launch_aggregate(plan->dp, idx, val, dense_out, s);
+  if (e == cudaSuccess) e = launch_aggregate(plan->dp, idx, val, dense_out, nullptr, s);
   return cuda_status(e);
+}
+
+lags_status lags_aggregate_apply(lags_plan* plan, const uint32_t* idx, const float* val,
+                                 float* dense_out, float* weights, void* stream) {
+  if (!plan || !idx || !val || !dense_out || !weights) return LAGS_ERR_INVALID_ARG;
+  if (!plan->ws) return LAGS_ERR_WORKSPACE;
+  if (!aligned(idx, 4) || !aligned(val, 4) || !aligned(dense_out, 16) || !aligned(weights, 16))
+    return LAGS_ERR_ALIGNMENT;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_pick_bounds(plan->dp, idx, s);
+  if (e == cudaSuccess) e = launch_aggregate(plan->dp, idx, val, dense_out, weights, s);
+  return cuda_status(e);
+}
+
+lags_status lags_plan_kernel_launches(const lags_plan* plan, int32_t* sparsify,
+                                      int32_t* aggregate, int32_t* apply) {
+  if (!plan) return LAGS_ERR_INVALID_ARG;
+  const bool any_sparse = !plan->sparse.empty();
+  if (sparsify)
+    *sparsify = (any_sparse ? 1 : 0) + 1 + (plan->sel_small.empty() ? 0 : 1) +
+                (plan->sel_large.empty() ? 0 : 1);
+  if (aggregate) *aggregate = 2;
+  if (apply) *apply = 1;
+  return LAGS_OK;
 }
 
 lags_status lags_apply(const lags_plan* plan, float* weights, const float* dense_out,

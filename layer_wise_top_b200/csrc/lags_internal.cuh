@@ -21,7 +21,8 @@ constexpr uint32_t kSampleMax = 16384;
 constexpr uint32_t kSampleChunk = 64;  // contiguous elements per sample chunk
 constexpr uint32_t kEstThreads = 512;
 
-// Cluster size used to select the large layers; small layers use one CTA.
+// Cluster size used to select layers whose expected candidates exceed what one
+// CTA stages in shared memory; the other layers use one CTA.
 constexpr int kSelectCluster = 8;
 constexpr uint32_t kSelectThreads = 512;
 constexpr uint32_t kSelectWindow = 2048;  // tiles whose prefix sits in smem at once
@@ -29,8 +30,8 @@ constexpr uint32_t kSelectWindow = 2048;  // tiles whose prefix sits in smem at 
 // the expected candidate counts, at most kSelectStageMax); a CTA with more
 // reads them from global memory on every pass instead.
 constexpr uint32_t kSelectStageMin = 1024;
-constexpr uint32_t kSelectStageMax = 11264;
-constexpr uint32_t kLargeK = 4096;  // k_l at or above: clustered select
+constexpr uint32_t kSelectStageMax = 22528;
+
 
 // Radix digits of the magnitude key (bits 30..0 of the fp32 pattern).
 constexpr int kDigitShift0 = 20;  // level 0: bits 30..20, 2048 bins
@@ -89,6 +90,7 @@ struct DevPlan {
   uint64_t K;
   uint64_t C;  // candidate slots per worker
   uint32_t stage_small, stage_large;  // shared-memory staging capacity per select launch
+  uint32_t agg_tile_acc;  // aggregation launches carry a shared tile accumulator
 };
 
 // Launchers (each returns the launch's cudaError_t).
@@ -101,7 +103,7 @@ cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out
                           float* out_val, cudaStream_t s);
 cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStream_t s);
 cudaError_t launch_aggregate(const DevPlan& dp, const uint32_t* idx, const float* val,
-                             float* dense, cudaStream_t s);
+                             float* dense, float* weights, cudaStream_t s);
 cudaError_t launch_apply(uint32_t N, float* w, const float* dense, cudaStream_t s);
 
 // The fused error-feedback pass used by lags_sparsify.

@@ -23,6 +23,7 @@ struct lags_plan {
   int device = -1;
   cudaEvent_t ev_before = nullptr, ev_after = nullptr;
   uint32_t stage_small = 0, stage_large = 0;  // select staging capacity per launch
+  uint32_t agg_tile_acc = 0;  // some tile expects more picks than the owner search handles
   lags::DevPlan dp{};  // device view once a workspace is bound
 };
 
@@ -54,4 +55,5 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.C = plan->C;
   dp.stage_small = plan->stage_small;
   dp.stage_large = plan->stage_large;
+  dp.agg_tile_acc = plan->agg_tile_acc;
 }

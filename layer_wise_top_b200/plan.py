@@ -77,6 +77,19 @@ class Plan:
         B.lags_aggregate(self.handle, idx.data_ptr(), val.data_ptr(), dense_out.data_ptr(),
                          _stream(stream, self.device))
 
+    def aggregate_apply(self, idx: torch.Tensor, val: torch.Tensor, dense_out: torch.Tensor,
+                        weights: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> None:
+        _need(idx, torch.int32, self.P * self.K, "idx")
+        _need(val, torch.float32, self.P * self.K, "val")
+        _need(dense_out, torch.float32, self.N, "dense_out")
+        _need(weights, torch.float32, self.N, "weights")
+        B.lags_aggregate_apply(self.handle, idx.data_ptr(), val.data_ptr(), dense_out.data_ptr(),
+                               weights.data_ptr(), _stream(stream, self.device))
+
+    def kernel_launches(self):
+        """Kernels enqueued by one sparsify, aggregate and apply call."""
+        return B.lags_plan_kernel_launches(self.handle)
+
     def apply(self, weights: torch.Tensor, dense_out: torch.Tensor,
               stream: Optional[torch.cuda.Stream] = None) -> None:
         _need(weights, torch.float32, self.N, "weights")

@@ -35,12 +35,17 @@ class GpuRun:
         self.keep_prev = keep_prev
         self.prev: Optional[List[torch.Tensor]] = None
 
-    def step(self) -> None:
+    def step(self, fused: bool = False) -> None:
+        """One step; `fused` uses lags_aggregate_apply instead of
+        lags_aggregate + lags_apply (the results must be identical)."""
         if self.keep_prev:
             self.prev = [r.clone() for r in self.res]
         self.plan.sparsify(self.grads, self.res, self.lr, self.idx, self.val)
-        self.plan.aggregate(self.idx, self.val, self.dense)
-        self.plan.apply(self.weights, self.dense)
+        if fused:
+            self.plan.aggregate_apply(self.idx, self.val, self.dense, self.weights)
+        else:
+            self.plan.aggregate(self.idx, self.val, self.dense)
+            self.plan.apply(self.weights, self.dense)
 
 
 def oracle_layer_steps(off: int, d: int, k: int, P: int, lr: float, steps: int,

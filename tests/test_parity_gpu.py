@@ -40,7 +40,7 @@ def run_full_compare(sizes, densities, P, lr, steps, grad_fn, expect_fallbacks=N
     for s in range(steps):
         for p in range(P):
             run.grads[p].copy_(torch.from_numpy(grad_fn(p, s)))
-        run.step()
+        run.step(fused=s % 2 == 1)  # odd steps: lags_aggregate_apply
         flags, fb = run.plan.poll()
         assert flags == 0
         total_fb += fb
@@ -116,9 +116,11 @@ def test_integer_ties_force_exact_path():
 
 
 def test_all_zero_gradients():
-    sizes = [100, 8192, 30000, 1_048_576, 600_000]
+    # all picks tie at 0 and go to the lowest indices: the first tile of the
+    # 1M layer at 0.005 receives 2 x 5243 picks, more than aggregation stages
+    sizes = [100, 8192, 30000, 1_048_576, 600_000, 1_000_000]
     fn = _np_grads(lambda n: np.zeros(n, dtype=F32), sizes, 2, 2)
-    run_full_compare(sizes, [0.01, 0.001, 0.5, 0.001, 0.01], 2, 0.1, 2, fn)
+    run_full_compare(sizes, [0.01, 0.001, 0.5, 0.001, 0.01, 0.005], 2, 0.1, 2, fn)
 
 
 def test_signed_zero_denormal_inf():
@@ -191,7 +193,7 @@ def _full_size(name, steps, inv_workers):
     for s in range(steps):
         for p in range(w.P):
             synth.worker_grads_device(w, p, s, run.grads[p])
-        run.step()
+        run.step(fused=s % 2 == 1)
         flags, fb = run.plan.poll()
         assert flags == 0
         fallbacks += fb
