@@ -10,6 +10,9 @@
 // result is bit-identical however the grid is scheduled.  With a weights
 // pointer the same kernel also applies the SGD update (weights -= dense).
 //
+// Pick lists are read through the read-only path (they are inputs; plain
+// loads would be ordered behind the kernels' own scattered stores).
+//
 // k_pick_bounds first turns each worker's ascending pick list into the slot of
 // the first pick of every tile, so each aggregation CTA reads only its own
 // picks.  It also checks that the lists are ascending and inside their layer.
@@ -25,26 +28,15 @@ __device__ __forceinline__ uint32_t tile_of(const LayerDesc& ld, uint32_t x) {
 }
 
 __global__ void __launch_bounds__(256) k_pick_bounds(DevPlan dp, const uint32_t* __restrict__ idx) {
-  __shared__ uint32_t s_layer0;
-  const uint64_t i0 = (uint64_t)blockIdx.x * blockDim.x;
-  const uint64_t i = i0 + threadIdx.x;
+  // one block per (chunk of 256 pick slots of a sparse layer, worker)
+  const uint2 ch = dp.pick_chunks[blockIdx.x];  // (layer, first slot within the layer)
   const uint32_t p = blockIdx.y;
-  if (threadIdx.x == 0) {  // layer holding the block's first slot: last layer with koff <= i0
-    uint32_t lo = 0, hi = dp.L - 1;
-    while (lo < hi) {
-      const uint32_t mid = (lo + hi + 1) >> 1;
-      if (dp.layers[mid].koff <= i0) lo = mid; else hi = mid - 1;
-    }
-    s_layer0 = lo;
-  }
-  __syncthreads();
-  if (i >= dp.K) return;
-  uint32_t lo = s_layer0;  // slots are consecutive: step forward to this slot's layer
-  while (lo + 1 < dp.L && dp.layers[lo + 1].koff <= i) ++lo;
-  const LayerDesc ld = dp.layers[lo];
-  if (ld.k == ld.d) return;  // dense layer: slot of element e is koff + e - off
+  const LayerDesc ld = dp.layers[ch.x];
+  const uint32_t j = ch.y + threadIdx.x;
+  if (j >= ld.k) return;
+  const uint64_t i = (uint64_t)ld.koff + j;
   const uint32_t* pi = idx + (uint64_t)p * dp.K;
-  const uint32_t x = pi[i];
+  const uint32_t x = __ldg(pi + i);
   const uint32_t lend = ld.off + ld.d;
   if (x < ld.off || x >= lend) {
     atomicOr(dp.status + kStatusFlags, LAGS_FLAG_BAD_PICKS);
@@ -55,7 +47,7 @@ __global__ void __launch_bounds__(256) k_pick_bounds(DevPlan dp, const uint32_t*
   if (i == ld.koff) {
     tprev = ld.tile_begin - 1;  // wraps for tile_begin == 0; only used as tprev + 1
   } else {
-    const uint32_t xp = pi[i - 1];
+    const uint32_t xp = __ldg(pi + i - 1);
     if (xp < ld.off || xp >= x) {
       atomicOr(dp.status + kStatusFlags, LAGS_FLAG_BAD_PICKS);
       return;
@@ -70,7 +62,7 @@ __global__ void __launch_bounds__(256) k_pick_bounds(DevPlan dp, const uint32_t*
 
 // Picks of one tile staged in shared memory; a tile with more picks (layers
 // sent at high density by many workers) reads them from global memory.
-constexpr uint32_t kAggPickCap = 4096;
+constexpr uint32_t kAggPickCap = 2048;
 // Up to this many picks in a tile, the thread holding a position's first pick
 // looks the position up in the other workers' lists (binary search); above it,
 // and when the launch has room for a tile accumulator, the CTA adds the
@@ -84,17 +76,23 @@ struct AggShared {
   uint32_t rng[2 * LAGS_MAX_WORKERS];
   uint32_t warp[kAggThreads / 32];
 };
-struct AggTileAcc {                      // only in launches that may need it
+// Tile accumulator, only in launches that may need it.  A sum that started at
+// +0 is never -0, so acc != 0 tells exactly which positions need the division
+// and the weight update (0 / P == +0 and w - (+0) == w).
+struct AggTileAcc {
   float acc[kTile];
-  uint32_t hit[kTile / 32];              // bit i of word w: position 32 w + i was picked
 };
+// The accumulator follows AggShared in dynamic shared memory and is cleared
+// with 16-byte stores, so it starts on a 128-byte boundary.
+constexpr size_t kAggAccOffset = (sizeof(AggShared) + 127) / 128 * 128;
+static_assert(kAggAccOffset % 16 == 0, "tile accumulator alignment");
 
 __global__ void __launch_bounds__(kAggThreads)
     k_aggregate(DevPlan dp, const uint32_t* __restrict__ idx, const float* __restrict__ val,
                 float* __restrict__ dense, float* __restrict__ weights, bool have_acc) {
   extern __shared__ __align__(16) unsigned char agg_smem[];
   AggShared& sh = *reinterpret_cast<AggShared*>(agg_smem);
-  AggTileAcc& ta = *reinterpret_cast<AggTileAcc*>(agg_smem + sizeof(AggShared));
+  AggTileAcc& ta = *reinterpret_cast<AggTileAcc*>(agg_smem + kAggAccOffset);
   const uint32_t t = blockIdx.x;
   const TileDesc td = dp.tiles[t];
   const LayerDesc ld = dp.layers[td.layer];
@@ -108,7 +106,7 @@ __global__ void __launch_bounds__(kAggThreads)
     const uint64_t s0 = ld.koff + (td.start - ld.off);
     for (uint32_t i = tid; i < td.len; i += kAggThreads) {
       float s = 0.0f;
-      for (uint32_t p = 0; p < P; ++p) s = __fadd_rn(s, val[p * K + s0 + i]);
+      for (uint32_t p = 0; p < P; ++p) s = __fadd_rn(s, __ldg(val + p * K + s0 + i));
       const float dv = __fdiv_rn(s, fP);
       dense[td.start + i] = dv;
       if (weights) weights[td.start + i] = __fsub_rn(weights[td.start + i], dv);
@@ -120,8 +118,8 @@ __global__ void __launch_bounds__(kAggThreads)
   uint32_t cnt = 0;
   if (tid < (int)P) {
     const uint32_t* first = dp.pick_first + (size_t)tid * dp.T;
-    uint32_t a = first[t];
-    uint32_t b = (t + 1 < ld.tile_end) ? first[t + 1] : kend;
+    uint32_t a = __ldg(first + t);
+    uint32_t b = (t + 1 < ld.tile_end) ? __ldg(first + t + 1) : kend;
     a = min(max(a, ld.koff), kend);  // keeps a bad pick list inside the layer
     b = min(max(b, a), kend);
     sh.rng[2 * tid] = a;
@@ -146,9 +144,9 @@ __global__ void __launch_bounds__(kAggThreads)
     for (uint32_t i = tid; i < total; i += kAggThreads) {
       const uint32_t p = worker_of(i);
       const uint64_t slot = p * K + sh.rng[2 * p] + (i - sh.base[p]);
-      const uint32_t x = idx[slot] - td.start;
+      const uint32_t x = __ldg(idx + slot) - td.start;
       sh.loc[i] = (uint16_t)(x < td.len ? x : 0xFFFFu);
-      sh.val[i] = val[slot];
+      sh.val[i] = __ldg(val + slot);
     }
   }
   const uint32_t head = min(td.len, (4u - (td.start & 3u)) & 3u);
@@ -193,56 +191,68 @@ __global__ void __launch_bounds__(kAggThreads)
 
   if (have_acc) {
     // ---- many picks: worker-ordered accumulation in a shared tile ----
-    for (uint32_t i = tid; i < kTile; i += kAggThreads) ta.acc[i] = 0.0f;
-    for (uint32_t i = tid; i < kTile / 32; i += kAggThreads) ta.hit[i] = 0;
+    float4* acc4 = reinterpret_cast<float4*>(ta.acc);
+    for (uint32_t i = tid; i < kTile / 4; i += kAggThreads) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();
     for (uint32_t p = 0; p < P; ++p) {
       if (staged) {
         for (uint32_t j = sh.base[p] + tid; j < sh.base[p + 1]; j += kAggThreads) {
           const uint32_t x = sh.loc[j];
-          if (x >= td.len) continue;
-          ta.acc[x] = __fadd_rn(ta.acc[x], sh.val[j]);
-          atomicOr(&ta.hit[x / 32], 1u << (x % 32));
+          if (x < td.len) ta.acc[x] = __fadd_rn(ta.acc[x], sh.val[j]);
         }
       } else {
         const uint64_t row = p * K;
         for (uint32_t j = sh.rng[2 * p] + tid; j < sh.rng[2 * p + 1]; j += kAggThreads) {
-          const uint32_t x = idx[row + j] - td.start;
-          if (x >= td.len) continue;
-          ta.acc[x] = __fadd_rn(ta.acc[x], val[row + j]);
-          atomicOr(&ta.hit[x / 32], 1u << (x % 32));
+          const uint32_t x = __ldg(idx + row + j) - td.start;
+          if (x < td.len) ta.acc[x] = __fadd_rn(ta.acc[x], __ldg(val + row + j));
         }
       }
       __syncthreads();
     }
-    auto picked = [&](uint32_t i) -> bool { return (ta.hit[i / 32] >> (i % 32)) & 1u; };
     auto value_at = [&](uint32_t i) -> float {
-      return picked(i) ? __fdiv_rn(ta.acc[i], fP) : 0.0f;
+      const float a = ta.acc[i];
+      return a != 0.0f ? __fdiv_rn(a, fP) : 0.0f;
     };
     for (uint32_t i = tid; i < head; i += kAggThreads) {
       const float q = value_at(i);
       dense[td.start + i] = q;
-      if (weights && picked(i)) weights[td.start + i] = __fsub_rn(weights[td.start + i], q);
+      if (weights && __float_as_uint(q) != 0u)  // skip only +0: w - (-0) may differ from w
+        weights[td.start + i] = __fsub_rn(weights[td.start + i], q);
     }
     float4* d4 = reinterpret_cast<float4*>(dense + td.start + head);
     float4* w4 = weights ? reinterpret_cast<float4*>(weights + td.start + head) : nullptr;
-    for (uint32_t v = tid; v < nvec; v += kAggThreads) {
-      const uint32_t i = head + 4 * v;
+    // a thread's weight loads all go out before its first store (a load
+    // issued after stores waits for them)
+    constexpr uint32_t GV = (kTile / 4 + kAggThreads - 1) / kAggThreads;
+    float4 wv[GV];
+    bool upd[GV];
+#pragma unroll
+    for (uint32_t j = 0; j < GV; ++j) {
+      const uint32_t v = tid + j * kAggThreads, i = head + 4 * v;
+      upd[j] = w4 && v < nvec &&
+               (ta.acc[i] != 0.f || ta.acc[i + 1] != 0.f || ta.acc[i + 2] != 0.f ||
+                ta.acc[i + 3] != 0.f);
+      if (upd[j]) wv[j] = w4[v];  // 16-byte aligned: weights and dense share the layout
+    }
+#pragma unroll
+    for (uint32_t j = 0; j < GV; ++j) {
+      const uint32_t v = tid + j * kAggThreads, i = head + 4 * v;
+      if (v >= nvec) continue;
       const float4 q = make_float4(value_at(i), value_at(i + 1), value_at(i + 2), value_at(i + 3));
       __stcs(d4 + v, q);
-      if (w4 && (picked(i) || picked(i + 1) || picked(i + 2) || picked(i + 3))) {
-        float4 wv = w4[v];  // 16-byte aligned: weights and dense share the layout
-        if (picked(i)) wv.x = __fsub_rn(wv.x, q.x);
-        if (picked(i + 1)) wv.y = __fsub_rn(wv.y, q.y);
-        if (picked(i + 2)) wv.z = __fsub_rn(wv.z, q.z);
-        if (picked(i + 3)) wv.w = __fsub_rn(wv.w, q.w);
-        w4[v] = wv;
+      if (upd[j]) {
+        wv[j].x = __fsub_rn(wv[j].x, q.x);
+        wv[j].y = __fsub_rn(wv[j].y, q.y);
+        wv[j].z = __fsub_rn(wv[j].z, q.z);
+        wv[j].w = __fsub_rn(wv[j].w, q.w);
+        w4[v] = wv[j];
       }
     }
     for (uint32_t i = head + 4 * nvec + tid; i < td.len; i += kAggThreads) {
       const float q = value_at(i);
       dense[td.start + i] = q;
-      if (weights && picked(i)) weights[td.start + i] = __fsub_rn(weights[td.start + i], q);
+      if (weights && __float_as_uint(q) != 0u)  // skip only +0: w - (-0) may differ from w
+        weights[td.start + i] = __fsub_rn(weights[td.start + i], q);
     }
     return;
   }
@@ -254,8 +264,8 @@ __global__ void __launch_bounds__(kAggThreads)
   for (uint32_t p = 0; p < P; ++p) {
     const uint64_t row = p * K;
     for (uint32_t j = sh.rng[2 * p] + tid; j < sh.rng[2 * p + 1]; j += kAggThreads) {
-      const uint32_t x = idx[row + j] - td.start;
-      if (x < td.len) dense[td.start + x] = __fadd_rn(dense[td.start + x], val[row + j]);
+      const uint32_t x = __ldg(idx + row + j) - td.start;
+      if (x < td.len) dense[td.start + x] = __fadd_rn(dense[td.start + x], __ldg(val + row + j));
     }
     __syncthreads();
   }
@@ -289,19 +299,20 @@ __global__ void __launch_bounds__(256) k_apply(uint32_t N, float* __restrict__ w
 }
 
 cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStream_t s) {
-  dim3 grid((unsigned)((dp.K + 255) / 256), dp.P);
+  if (dp.n_chunks == 0) return cudaSuccess;
+  dim3 grid(dp.n_chunks, dp.P);
   k_pick_bounds<<<grid, 256, 0, s>>>(dp, idx);
   return cudaGetLastError();
 }
 
 cudaError_t configure_aggregate() {
   return cudaFuncSetAttribute(k_aggregate, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)(sizeof(AggShared) + sizeof(AggTileAcc)));
+                              (int)(kAggAccOffset + sizeof(AggTileAcc)));
 }
 
 cudaError_t launch_aggregate(const DevPlan& dp, const uint32_t* idx, const float* val,
                              float* dense, float* weights, cudaStream_t s) {
-  const size_t smem = sizeof(AggShared) + (dp.agg_tile_acc ? sizeof(AggTileAcc) : 0);
+  const size_t smem = dp.agg_tile_acc ? kAggAccOffset + sizeof(AggTileAcc) : sizeof(AggShared);
   k_aggregate<<<dp.T, kAggThreads, smem, s>>>(dp, idx, val, dense, weights, dp.agg_tile_acc != 0);
   return cudaGetLastError();
 }

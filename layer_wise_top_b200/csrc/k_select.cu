@@ -32,8 +32,6 @@ namespace lags {
 
 namespace {
 
-constexpr int NT = kSelectThreads;
-
 template <int CL>
 struct Cluster {
   __device__ __forceinline__ static void sync() {
@@ -60,6 +58,13 @@ struct Cluster {
   }
 };
 
+// First element of tile t of layer ld: tiles start on multiples of kTile in
+// the flattened buffer, except a layer's first tile, which starts at the layer.
+__device__ __forceinline__ uint32_t tile_start(const LayerDesc& ld, uint32_t t) {
+  return t == ld.tile_begin ? ld.off : (ld.off / kTile + (t - ld.tile_begin)) * kTile;
+}
+
+template <int NT>
 struct SelectShared {
   uint32_t hist[kBins];          // this CTA's histogram (then the merged copy)
   uint32_t tpre[kSelectWindow + 1];
@@ -69,16 +74,19 @@ struct SelectShared {
 
 }  // namespace
 
-template <int CL>
+template <int CL, int NT>
 __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const uint32_t* list,
                                                uint32_t stage_cap,
                                                uint32_t* __restrict__ out_idx,
                                                float* __restrict__ out_val) {
   using C = Cluster<CL>;
-  __shared__ SelectShared sh;
+  __shared__ SelectShared<NT> sh;
   // CTA 0 of a cluster: cluster-wide histograms, one per level
   __shared__ uint32_t merged[CL > 1 ? 3 : 1][kBins];
-  extern __shared__ __align__(16) float stage_val[];  // stage_cap candidate values
+  // staged candidates: stage_cap values, then stage_cap 16-bit offsets inside
+  // their tile (the index is tile_start + offset)
+  extern __shared__ __align__(16) float stage_val[];
+  uint16_t* stage_off = reinterpret_cast<uint16_t*>(stage_val + stage_cap);
   const uint32_t rank = C::rank();
   const uint32_t layer = list[blockIdx.x / CL];
   const uint32_t p = blockIdx.y;
@@ -100,7 +108,7 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   const uint32_t* cnt = dp.tile_cnt + (size_t)p * dp.T;
   uint32_t my = 0, ovf = 0;
   for (uint32_t t = ta + tid; t < tb; t += NT) {
-    const uint32_t c = cnt[t];
+    const uint32_t c = __ldg(cnt + t);
     my += c;
     ovf |= c > cap;
   }
@@ -140,7 +148,7 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
         const uint32_t q = tid * PER + i;
-        c[i] = q < nw ? cnt[w0 + q] : 0u;
+        c[i] = q < nw ? __ldg(cnt + w0 + q) : 0u;
         sum += c[i];
       }
       uint32_t wtotal;
@@ -165,8 +173,8 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
           }
           const uint64_t slot =
               cbase + (uint64_t)(w0 + lo - ld.tile_begin) * cap + (v - sh.tpre[lo]);
-          idx = dp.cand_idx[slot];
-          val = dp.cand_val[slot];
+          idx = __ldg(dp.cand_idx + slot);
+          val = __ldg(dp.cand_val + slot);
         }
         fn(valid, seen + v, idx, val);
       }
@@ -185,7 +193,7 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const uint32_t q = tid * PER + i;
-      c[i] = q < nw ? cnt[ta + q] : 0u;
+      c[i] = q < nw ? __ldg(cnt + ta + q) : 0u;
       sum += c[i];
     }
     uint32_t wtotal;
@@ -198,31 +206,40 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
     }
     if (tid == 0) sh.tpre[nw] = wtotal;
     __syncthreads();
-    constexpr uint32_t U = 8;  // loads in flight per thread
+    constexpr uint32_t U = 8;  // candidates per thread with loads in flight
     for (uint32_t b = 0; b < wtotal; b += NT * U) {
       float fv[U];
+      uint32_t iv[U];
 #pragma unroll
       for (uint32_t u = 0; u < U; ++u) {
         const uint32_t v = b + u * NT + tid;
         fv[u] = 0.f;
+        iv[u] = 0;
         if (v < wtotal) {
           uint32_t lo = 0, hi = nw - 1;
           while (lo < hi) {
             const uint32_t mid = (lo + hi + 1) >> 1;
             if (sh.tpre[mid] <= v) lo = mid; else hi = mid - 1;
           }
-          fv[u] = dp.cand_val[cbase + (uint64_t)(ta + lo - ld.tile_begin) * cap +
-                              (v - sh.tpre[lo])];
+          const uint64_t slot = cbase + (uint64_t)(ta + lo - ld.tile_begin) * cap + (v - sh.tpre[lo]);
+          fv[u] = __ldg(dp.cand_val + slot);
+          iv[u] = __ldg(dp.cand_idx + slot) - tile_start(ld, ta + lo);
         }
       }
 #pragma unroll
       for (uint32_t u = 0; u < U; ++u) {
         const uint32_t v = b + u * NT + tid;
-        if (v < wtotal) stage_val[v] = fv[u];
+        if (v < wtotal) {
+          stage_val[v] = fv[u];
+          stage_off[v] = (uint16_t)iv[u];
+        }
       }
     }
     __syncthreads();
   }
+  // (Candidate lists and counts are read through the read-only path: nothing
+  // writes them during this kernel, and plain loads would be ordered behind the
+  // emission's scattered stores, which measured 6x slower.)
   // Unstaged shares: every pass walks the candidates (or, on the exhaustive
   // path, the layer's acc) from global memory.
   auto traverse = [&](auto&& fn) {
@@ -241,13 +258,17 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   // One radix level: histogram of digit (key >> dshift) & dmask over the keys
   // whose prefix key >> mshift equals mval (all keys when mshift == 32),
   // merged across the cluster into sh.hist.
-  // staged share: thread tid owns the contiguous positions [cb, ce)
-  const uint32_t chunk = (my + NT - 1) / NT;
-  const uint32_t cb = min(my, tid * chunk), ce = min(my, cb + chunk);
+  // staged share, for the ordered emission: warp w owns the contiguous
+  // positions [wb, we) and walks them 32 at a time
+  constexpr uint32_t NW = NT / 32;
+  const uint32_t warp = tid >> 5;
+  const uint32_t wspan = (my + NW - 1) / NW;
+  const uint32_t wb = min(my, warp * wspan), we = min(my, wb + wspan);
+  const unsigned lanes_below = (1u << lane) - 1u;
 
   auto hist_level = [&](int level, int mshift, uint32_t mval, int dshift, uint32_t dmask) {
     if (staged) {
-      for (uint32_t i = cb; i < ce; ++i) {
+      for (uint32_t i = tid; i < my; i += NT) {
         const uint32_t key = mag_key(stage_val[i]);
         if (mshift >= 32 || (key >> mshift) == mval)
           atomicAdd(&sh.hist[(key >> dshift) & dmask], 1u);
@@ -311,18 +332,30 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   const uint32_t need = rem;
 
   // ---- count strict picks and ties of this CTA, exchange prefixes ----
-  uint32_t na = 0, nb = 0, my_ex = 0;
+  uint32_t na = 0, nb = 0, warp_ex = 0;
   if (staged) {
     uint32_t ca = 0, ct = 0;
-    for (uint32_t i = cb; i < ce; ++i) {
+    for (uint32_t i = wb + lane; i < we; i += 32) {
       const uint32_t s = mag_key(stage_val[i]) >> fshift;
       ca += s > fpfx;
       ct += s == fpfx;
     }
-    uint32_t tot;  // per-CTA counts <= stage_cap < 2^16: pack strict | ties
-    my_ex = block_excl_scan<NT>((ca << 16) | ct, sh.tmp, &tot);
+    // per-CTA counts <= stage_cap < 2^16: pack strict | ties
+    const uint32_t wsum = __reduce_add_sync(kFull, (ca << 16) | ct);
+    if (lane == 0) sh.tmp[warp] = wsum;
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t x = lane < NW ? sh.tmp[lane] : 0u;
+      const uint32_t incl = warp_incl_scan(x);
+      if (lane < NW) sh.tmp[NW + lane] = incl - x;
+      if (lane == NW - 1) sh.tmp[2 * NW] = incl;
+    }
+    __syncthreads();
+    warp_ex = sh.tmp[NW + warp];
+    const uint32_t tot = sh.tmp[2 * NW];
     na = tot >> 16;
     nb = tot & 0xFFFFu;
+    __syncthreads();
   } else {
     traverse([&](bool valid, uint32_t, float val) {
       const uint32_t s = mag_key(val) >> fshift;
@@ -346,37 +379,52 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
 
   // ---- ordered emission: pos = strict_before + min(need, ties_before) ----
   const uint64_t ob = (uint64_t)p * dp.K + ld.koff;
-  auto emit = [&](uint32_t pos, uint32_t idx, float val) {
+  auto emit = [&](uint32_t pos, uint32_t idx, float val, bool zero_residual) {
     if (pos < ld.k) {
       out_idx[ob + pos] = idx;
       out_val[ob + pos] = val;
-      r[idx] = 0.0f;
+      if (zero_residual) r[idx] = 0.0f;
     } else {
       atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
     }
   };
   if (staged) {
-    uint32_t at = a_run + (my_ex >> 16), bt = b_run + (my_ex & 0xFFFFu);
-    uint32_t tl = 0;  // tile (relative to ta) holding staged position cb
-    {
+    // warp rounds of 32 consecutive positions: ballots give each lane its
+    // strict and tie ranks, so the pick-list stores are coalesced and no
+    // block barrier is needed; the emitted index replaces the staged value
+    // (0xFFFFFFFF marks "not emitted") for the residual zeroing below
+    uint32_t at = a_run + (warp_ex >> 16), bt = b_run + (warp_ex & 0xFFFFu);
+    uint32_t tl = 0;  // tile (relative to ta) of this lane's current position
+    if (wb < we) {    // start from the tile holding the warp's first position
       uint32_t hi = tb - ta - 1;
       while (tl < hi) {
         const uint32_t mid = (tl + hi + 1) >> 1;
-        if (sh.tpre[mid] <= cb) tl = mid; else hi = mid - 1;
+        if (sh.tpre[mid] <= wb) tl = mid; else hi = mid - 1;
       }
     }
-    for (uint32_t i = cb; i < ce; ++i) {
-      while (sh.tpre[tl + 1] <= i) ++tl;
-      const float val = stage_val[i];
+    for (uint32_t b0 = wb; b0 < we; b0 += 32) {
+      const uint32_t i = b0 + lane;
+      const bool valid = i < we;
+      const float val = valid ? stage_val[i] : 0.f;
       const uint32_t s = mag_key(val) >> fshift;
-      const bool st = s > fpfx, ti = s == fpfx && bt < need;
-      if (st || ti) {
-        const uint32_t idx =
-            dp.cand_idx[cbase + (uint64_t)(ta + tl - ld.tile_begin) * cap + (i - sh.tpre[tl])];
-        emit(st ? at + min(need, bt) : at + bt, idx, val);
+      const bool st = valid && s > fpfx, ti = valid && s == fpfx;
+      const unsigned mst = __ballot_sync(kFull, st), mti = __ballot_sync(kFull, ti);
+      const uint32_t sb = at + __popc(mst & lanes_below), tb_ = bt + __popc(mti & lanes_below);
+      uint32_t mark = 0xFFFFFFFFu;
+      if (st || (ti && tb_ < need)) {
+        while (sh.tpre[tl + 1] <= i) ++tl;
+        const uint32_t idx = tile_start(ld, ta + tl) + stage_off[i];
+        emit(st ? sb + min(need, tb_) : sb + tb_, idx, val, false);
+        mark = idx;
       }
-      at += st;
-      bt += s == fpfx;
+      if (valid) stage_val[i] = __uint_as_float(mark);
+      at += __popc(mst);
+      bt += __popc(mti);
+    }
+    __syncwarp();
+    for (uint32_t i = wb + lane; i < we; i += 32) {
+      const uint32_t x = __float_as_uint(stage_val[i]);
+      if (x != 0xFFFFFFFFu) r[x] = 0.0f;
     }
   } else {
     traverse([&](bool valid, uint32_t idx, float val) {
@@ -386,8 +434,8 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
       uint32_t tot;
       const uint32_t ex = block_excl_scan<NT>(((uint32_t)st << 16) | (uint32_t)ti, sh.tmp, &tot);
       const uint32_t at = a_run + (ex >> 16), bt = b_run + (ex & 0xFFFFu);
-      if (st) emit(at + min(need, bt), idx, val);
-      else if (ti && bt < need) emit(at + bt, idx, val);
+      if (st) emit(at + min(need, bt), idx, val, true);
+      else if (ti && bt < need) emit(at + bt, idx, val, true);
       a_run += tot >> 16;
       b_run += tot & 0xFFFFu;
     });
@@ -395,12 +443,15 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   C::sync();  // no CTA leaves while another may still read its shared memory
 }
 
+// Dynamic shared memory of a select launch staging `cap` candidates.
+inline size_t stage_smem_bytes(uint32_t cap) { return ((size_t)cap * 6 + 15) / 16 * 16; }
+
 cudaError_t configure_select() {
-  const int most = (int)(kSelectStageMax * sizeof(float));
-  cudaError_t e = cudaFuncSetAttribute(k_select<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       most);
+  const int most = (int)stage_smem_bytes(kSelectStageMax);
+  cudaError_t e = cudaFuncSetAttribute(k_select<1, kSelectThreadsSmall>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, most);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_select<kSelectCluster>,
+  return cudaFuncSetAttribute(k_select<kSelectCluster, kSelectThreads>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, most);
 }
 
@@ -408,16 +459,17 @@ cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out
                           float* out_val, cudaStream_t s) {
   if (dp.n_small) {
     dim3 grid(dp.n_small, dp.P);
-    const size_t smem = dp.stage_small * sizeof(float);
-    k_select<1><<<grid, NT, smem, s>>>(dp, wp, dp.sel_small, dp.stage_small, out_idx, out_val);
+    const size_t smem = stage_smem_bytes(dp.stage_small);
+    k_select<1, kSelectThreadsSmall><<<grid, kSelectThreadsSmall, smem, s>>>(
+        dp, wp, dp.sel_small, dp.stage_small, out_idx, out_val);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (dp.n_large) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(dp.n_large * kSelectCluster, dp.P);
-    cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = dp.stage_large * sizeof(float);
+    cfg.blockDim = dim3(kSelectThreads);
+    cfg.dynamicSmemBytes = stage_smem_bytes(dp.stage_large);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -426,8 +478,8 @@ cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, k_select<kSelectCluster>, dp, wp, dp.sel_large,
-                                       dp.stage_large, out_idx, out_val);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_select<kSelectCluster, kSelectThreads>, dp, wp,
+                                       dp.sel_large, dp.stage_large, out_idx, out_val);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }

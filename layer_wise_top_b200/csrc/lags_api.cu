@@ -134,6 +134,7 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
       ld.sample = (uint32_t)((uint64_t)d < kSampleMax ? d : kSampleMax);
       ld.rank = sample_rank(ld.sample, d, k);
       plan->sparse.push_back((uint32_t)l);
+      for (uint64_t j0 = 0; j0 < k; j0 += 256) plan->pick_chunks.push_back(make_uint2(l, j0));
       // one CTA when its shared memory can stage the expected candidates with
       // a third to spare, else an 8-CTA cluster
       const double expect = expected_candidates(ld);
@@ -191,6 +192,7 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
   plan->o_cval = section(cur, P * (plan->C + 1) * 4);
   plan->o_cidx = section(cur, P * (plan->C + 1) * 4);
   plan->o_first = section(cur, P * T * 4);
+  plan->o_chunks = section(cur, (plan->pick_chunks.size() + 1) * sizeof(uint2));
   plan->o_status = section(cur, kStatusWords * 4);
   plan->ws_bytes = (cur + kAlign - 1) / kAlign * kAlign;
   *out_plan = plan;
@@ -247,6 +249,8 @@ lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t byt
   if (e == cudaSuccess) e = up(plan->o_large, plan->sel_large.data(), plan->sel_large.size() * 4);
   if (e == cudaSuccess) e = up(plan->o_small, plan->sel_small.data(), plan->sel_small.size() * 4);
   if (e == cudaSuccess) e = up(plan->o_sparse, plan->sparse.data(), plan->sparse.size() * 4);
+  if (e == cudaSuccess)
+    e = up(plan->o_chunks, plan->pick_chunks.data(), plan->pick_chunks.size() * sizeof(uint2));
   if (e == cudaSuccess) e = cudaMemsetAsync(base + plan->o_status, 0, kStatusWords * 4, s);
   // pageable sources: make sure the copies are done before returning
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);

@@ -24,7 +24,8 @@ constexpr uint32_t kEstThreads = 512;
 // Cluster size used to select layers whose expected candidates exceed what one
 // CTA stages in shared memory; the other layers use one CTA.
 constexpr int kSelectCluster = 8;
-constexpr uint32_t kSelectThreads = 512;
+constexpr uint32_t kSelectThreads = 512;       // clustered select
+constexpr uint32_t kSelectThreadsSmall = 512;  // single-CTA select (256 measured slower)
 constexpr uint32_t kSelectWindow = 2048;  // tiles whose prefix sits in smem at once
 // Candidates one selection CTA copies to shared memory (sized per launch from
 // the expected candidate counts, at most kSelectStageMax); a CTA with more
@@ -83,9 +84,10 @@ struct DevPlan {
   float* cand_val;            // [P][C]
   uint32_t* cand_idx;         // [P][C]
   uint32_t* pick_first;       // [P][T] first pick slot of each tile (aggregate)
+  const uint2* pick_chunks;   // (sparse layer, first slot) per 256 pick slots
   uint32_t* status;           // kStatusWords
   uint32_t L, T, P;
-  uint32_t n_large, n_small, n_sparse;
+  uint32_t n_large, n_small, n_sparse, n_chunks;
   uint32_t N;
   uint64_t K;
   uint64_t C;  // candidate slots per worker

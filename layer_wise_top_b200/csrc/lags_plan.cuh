@@ -15,10 +15,11 @@ struct lags_plan {
   std::vector<lags::LayerDesc> layers;
   std::vector<lags::TileDesc> tiles;
   std::vector<uint32_t> sel_large, sel_small, sparse;
+  std::vector<uint2> pick_chunks;  // (sparse layer, first slot) per 256 pick slots
   std::vector<int64_t> off, k, koff;
   // workspace sections (byte offsets)
   size_t o_layers = 0, o_tiles = 0, o_large = 0, o_small = 0, o_sparse = 0, o_lo = 0, o_cnt = 0,
-         o_cval = 0, o_cidx = 0, o_first = 0, o_status = 0, ws_bytes = 0;
+         o_cval = 0, o_cidx = 0, o_first = 0, o_chunks = 0, o_status = 0, ws_bytes = 0;
   void* ws = nullptr;
   int device = -1;
   cudaEvent_t ev_before = nullptr, ev_after = nullptr;
@@ -43,6 +44,7 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.cand_val = (float*)(base + plan->o_cval);
   dp.cand_idx = (uint32_t*)(base + plan->o_cidx);
   dp.pick_first = (uint32_t*)(base + plan->o_first);
+  dp.pick_chunks = (const uint2*)(base + plan->o_chunks);
   dp.status = (uint32_t*)(base + plan->o_status);
   dp.L = (uint32_t)plan->L;
   dp.T = (uint32_t)plan->tiles.size();
@@ -50,6 +52,7 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.n_large = (uint32_t)plan->sel_large.size();
   dp.n_small = (uint32_t)plan->sel_small.size();
   dp.n_sparse = (uint32_t)plan->sparse.size();
+  dp.n_chunks = (uint32_t)plan->pick_chunks.size();
   dp.N = (uint32_t)plan->N;
   dp.K = plan->K;
   dp.C = plan->C;

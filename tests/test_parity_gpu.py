@@ -218,3 +218,33 @@ def test_full_lstm():
 @pytest.mark.slow
 def test_full_gpt_1_3b():
     _full_size("gpt_1_3b", 2, [0, 5])
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_negative_zero_weights_and_underflowing_update(fused):
+    """Updates of -tiny / P round to -0; w - (-0) turns a -0 weight into +0,
+    so skipping such an update would be visible.  Weights start at -0."""
+    torch = _torch()
+    from gpu_harness import GpuRun, u32
+    rng = np.random.default_rng(9)
+    sizes, dens, P = [64, 10000, 8193], [1.0, 0.01, 0.001], 16
+    N = sum(sizes)
+    grads = []
+    for p in range(P):
+        g = np.zeros(N, dtype=F32)
+        hot = rng.choice(N, 300, replace=False)
+        g[hot] = (rng.integers(1, 4, hot.size) * np.float32(-1e-45)).astype(F32)
+        g[hot[:50]] = F32(1e-45)
+        grads.append(g)
+    run = GpuRun(sizes, dens, P, 1.0)
+    run.weights.fill_(-0.0)
+    for p in range(P):
+        run.grads[p].copy_(torch.from_numpy(grads[p]))
+    run.step(fused=fused)
+    res0 = [np.zeros(N, dtype=F32) for _ in range(P)]
+    e_idx, e_val, e_res = lo.sparsify(sizes, dens, grads, res0, 1.0)
+    e_dense = lo.aggregate(N, e_idx, e_val)
+    e_w = lo.apply_update(np.full(N, -0.0, dtype=F32), e_dense)
+    assert np.signbit(e_dense).any() and not np.signbit(e_w).all()  # the case occurs
+    assert np.array_equal(u32(run.dense), e_dense.view(np.uint32))
+    assert np.array_equal(u32(run.weights), e_w.view(np.uint32))
