@@ -29,10 +29,12 @@ __device__ __forceinline__ uint32_t tile_of(const LayerDesc& ld, uint32_t x) {
 
 __global__ void __launch_bounds__(256) k_pick_bounds(DevPlan dp, const uint32_t* __restrict__ idx) {
   // one block per (chunk of 256 pick slots of a sparse layer, worker)
+  pdl_trigger();
   const uint2 ch = dp.pick_chunks[blockIdx.x];  // (layer, first slot within the layer)
   const uint32_t p = blockIdx.y;
   const LayerDesc ld = dp.layers[ch.x];
   const uint32_t j = ch.y + threadIdx.x;
+  pdl_wait();
   if (j >= ld.k) return;
   const uint64_t i = (uint64_t)ld.koff + j;
   const uint32_t* pi = idx + (uint64_t)p * dp.K;
@@ -93,6 +95,7 @@ __global__ void __launch_bounds__(kAggThreads)
   extern __shared__ __align__(16) unsigned char agg_smem[];
   AggShared& sh = *reinterpret_cast<AggShared*>(agg_smem);
   AggTileAcc& ta = *reinterpret_cast<AggTileAcc*>(agg_smem + kAggAccOffset);
+  pdl_trigger();
   const uint32_t t = blockIdx.x;
   const TileDesc td = dp.tiles[t];
   const LayerDesc ld = dp.layers[td.layer];
@@ -100,6 +103,7 @@ __global__ void __launch_bounds__(kAggThreads)
   const float fP = (float)P;
   const uint64_t K = dp.K;
   const int tid = threadIdx.x;
+  pdl_wait();
 
   if (ld.k == ld.d) {
     // dense layer: every worker sent every entry; slot = koff + (e - off)
@@ -281,6 +285,8 @@ __global__ void __launch_bounds__(kAggThreads)
 
 __global__ void __launch_bounds__(256) k_apply(uint32_t N, float* __restrict__ w,
                                                const float* __restrict__ dense) {
+  pdl_trigger();
+  pdl_wait();
   const uint32_t n4 = N / 4;
   const uint32_t stride = gridDim.x * blockDim.x;
   float4* w4 = reinterpret_cast<float4*>(w);
@@ -301,8 +307,7 @@ __global__ void __launch_bounds__(256) k_apply(uint32_t N, float* __restrict__ w
 cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStream_t s) {
   if (dp.n_chunks == 0) return cudaSuccess;
   dim3 grid(dp.n_chunks, dp.P);
-  k_pick_bounds<<<grid, 256, 0, s>>>(dp, idx);
-  return cudaGetLastError();
+  return launch_pdl(k_pick_bounds, grid, dim3(256), 0, s, 1, dp, idx);
 }
 
 cudaError_t configure_aggregate() {
@@ -313,16 +318,15 @@ cudaError_t configure_aggregate() {
 cudaError_t launch_aggregate(const DevPlan& dp, const uint32_t* idx, const float* val,
                              float* dense, float* weights, cudaStream_t s) {
   const size_t smem = dp.agg_tile_acc ? kAggAccOffset + sizeof(AggTileAcc) : sizeof(AggShared);
-  k_aggregate<<<dp.T, kAggThreads, smem, s>>>(dp, idx, val, dense, weights, dp.agg_tile_acc != 0);
-  return cudaGetLastError();
+  return launch_pdl(k_aggregate, dim3(dp.T), dim3(kAggThreads), smem, s, 1, dp, idx, val, dense,
+                    weights, dp.agg_tile_acc != 0);
 }
 
 cudaError_t launch_apply(uint32_t N, float* w, const float* dense, cudaStream_t s) {
   uint32_t blocks = (N / 4 + 255) / 256;
   if (blocks > 148u * 16u) blocks = 148u * 16u;
   if (blocks == 0) blocks = 1;
-  k_apply<<<blocks, 256, 0, s>>>(N, w, dense);
-  return cudaGetLastError();
+  return launch_pdl(k_apply, dim3(blocks), dim3(256), 0, s, 1, N, w, dense);
 }
 
 }  // namespace lags

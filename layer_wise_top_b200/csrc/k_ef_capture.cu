@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, Worker
   __shared__ uint32_t s_base[V * NWARP];
   __shared__ uint32_t s_total;
 
+  pdl_trigger();
   const uint32_t t = blockIdx.x, p = blockIdx.y;
   const TileDesc td = dp.tiles[t];
   const LayerDesc ld = dp.layers[td.layer];
@@ -55,6 +56,7 @@ __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, Worker
   const uint32_t base = start & ~3u;
   const uint32_t N = dp.N;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();
 
   float4 a[V];
   float4 gv[V];
@@ -397,8 +399,7 @@ cudaError_t launch_ef_stream(const DevPlan& dp, const WorkerPtrs& wp, float lr,
 cudaError_t launch_ef_capture(const DevPlan& dp, const WorkerPtrs& wp, float lr,
                               uint32_t* out_idx, float* out_val, cudaStream_t s) {
   dim3 grid(dp.T, dp.P);
-  k_ef_capture<<<grid, kEfThreads, 0, s>>>(dp, wp, lr, out_idx, out_val);
-  return cudaGetLastError();
+  return launch_pdl(k_ef_capture, grid, dim3(kEfThreads), 0, s, 1, dp, wp, lr, out_idx, out_val);
 }
 
 }  // namespace lags

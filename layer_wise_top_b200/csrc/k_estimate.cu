@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs
   __shared__ uint32_t s_chunk[kSampleMax / kSampleChunk];  // first element of each run
   __shared__ uint32_t s_tmp[kEstThreads + kEstThreads / 32 + 4];
 
+  pdl_trigger();
   const uint32_t layer = dp.sparse[blockIdx.x];
   const uint32_t p = blockIdx.y;
   const LayerDesc ld = dp.layers[layer];
@@ -29,6 +30,7 @@ __global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs
   const float* __restrict__ r = wp.r[p];
   const uint32_t m = ld.sample;
   const uint32_t nchunk = m / kSampleChunk;
+  pdl_wait();
 
   for (uint32_t i = threadIdx.x; i < kBins; i += kEstThreads) s_hist[i] = 0;
   // sample positions: the whole layer, or nchunk runs of kSampleChunk spread
@@ -84,8 +86,8 @@ cudaError_t configure_estimate() {
 cudaError_t launch_estimate(const DevPlan& dp, const WorkerPtrs& wp, float lr, cudaStream_t s) {
   if (dp.n_sparse == 0) return cudaSuccess;
   dim3 grid(dp.n_sparse, dp.P);
-  k_estimate<<<grid, kEstThreads, kSampleMax * sizeof(uint32_t), s>>>(dp, wp, lr);
-  return cudaGetLastError();
+  return launch_pdl(k_estimate, grid, dim3(kEstThreads), kSampleMax * sizeof(uint32_t), s, 1, dp,
+                    wp, lr);
 }
 
 }  // namespace lags

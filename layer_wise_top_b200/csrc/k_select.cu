@@ -87,12 +87,14 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   // their tile (the index is tile_start + offset)
   extern __shared__ __align__(16) float stage_val[];
   uint16_t* stage_off = reinterpret_cast<uint16_t*>(stage_val + stage_cap);
+  pdl_trigger();
   const uint32_t rank = C::rank();
   const uint32_t layer = list[blockIdx.x / CL];
   const uint32_t p = blockIdx.y;
   const LayerDesc ld = dp.layers[layer];
   const int tid = threadIdx.x, lane = tid & 31;
   float* __restrict__ r = wp.r[p];
+  pdl_wait();
 
   for (int i = tid; i < (int)kBins; i += NT) {
     sh.hist[i] = 0;
@@ -458,30 +460,16 @@ cudaError_t configure_select() {
 cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out_idx,
                           float* out_val, cudaStream_t s) {
   if (dp.n_small) {
-    dim3 grid(dp.n_small, dp.P);
-    const size_t smem = stage_smem_bytes(dp.stage_small);
-    k_select<1, kSelectThreadsSmall><<<grid, kSelectThreadsSmall, smem, s>>>(
-        dp, wp, dp.sel_small, dp.stage_small, out_idx, out_val);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(k_select<1, kSelectThreadsSmall>, dim3(dp.n_small, dp.P),
+                               dim3(kSelectThreadsSmall), stage_smem_bytes(dp.stage_small), s, 1,
+                               dp, wp, dp.sel_small, dp.stage_small, out_idx, out_val);
     if (e != cudaSuccess) return e;
   }
   if (dp.n_large) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(dp.n_large * kSelectCluster, dp.P);
-    cfg.blockDim = dim3(kSelectThreads);
-    cfg.dynamicSmemBytes = stage_smem_bytes(dp.stage_large);
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kSelectCluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, k_select<kSelectCluster, kSelectThreads>, dp, wp,
-                                       dp.sel_large, dp.stage_large, out_idx, out_val);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    return launch_pdl(k_select<kSelectCluster, kSelectThreads>,
+                      dim3(dp.n_large * kSelectCluster, dp.P), dim3(kSelectThreads),
+                      stage_smem_bytes(dp.stage_large), s, kSelectCluster, dp, wp, dp.sel_large,
+                      dp.stage_large, out_idx, out_val);
   }
   return cudaSuccess;
 }

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "lags.h"
 
 namespace lags {
@@ -116,6 +118,46 @@ inline cudaError_t launch_ef(const DevPlan& dp, const WorkerPtrs& wp, float lr, 
 #else
   return launch_ef_capture(dp, wp, lr, out_idx, out_val, s);
 #endif
+}
+
+// ------------------------------------------------------------------ launches
+// Programmatic dependent launch: each kernel of a step is launched so that it
+// may be scheduled while its predecessor's last CTAs still run.  Every kernel
+// lets its dependents launch as soon as it starts (pdl_trigger) and waits for
+// its predecessor to complete, with memory visible, before touching anything
+// the predecessor may have written (pdl_wait).  Plan tables are written only
+// by lags_plan_set_workspace and may be read before the wait.  Launched
+// without the attribute, both are no-ops.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, int cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ helpers
