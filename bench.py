@@ -2,9 +2,8 @@
 """Throughput of the LAGS sparsify + aggregate step on B200.
 
 One step = error feedback + layer-wise exact top-k for all P simulated workers
-(lags_sparsify), the deterministic sparse aggregation (lags_aggregate) and the
-weight update (lags_apply), over one batch of synthetic gradients already in
-HBM.  value = P*N elements per step / step time, in Gelem/s; under torchrun
+(lags_sparsify) and the deterministic sparse aggregation with the weight update
+(lags_aggregate_apply), over one batch of synthetic gradients already in HBM.  value = P*N elements per step / step time, in Gelem/s; under torchrun
 each rank runs its own replica (no collective on the data path) and value sums
 the elements of all ranks over the slowest rank's time.
 
@@ -30,6 +29,12 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "LAGS sparsify+aggregate Gelem/s per step; achieved HBM GB/s vs peak"
+# DRAM bytes (read + write) of one k_ef_capture launch from the ncu capture in
+# profiles/k_ef_capture_vgg16.md (VGG-16 workload, 235,517,088 elements).
+# Other workloads scale it by their element count (the pass is a stream over
+# the elements, so its traffic grows in proportion).
+EF_TRAFFIC_BYTES = 1_885_774_000 + 895_709_696
+EF_TRAFFIC_ELEMENTS = 235_517_088
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 POOL_BUDGET_BYTES = 48 * 1024 ** 3
@@ -329,7 +334,12 @@ def run_ours(args):
             step="lags_sparsify + lags_aggregate_apply (aggregate and apply fused)"),
         "roofline": {"kernel": "k_ef_capture", "bound": "hbm", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak,
+                     "traffic": EF_TRAFFIC_BYTES * (P * N) / EF_TRAFFIC_ELEMENTS,
+                     "traffic_source": ("ncu capture of this workload" if P * N ==
+                                        EF_TRAFFIC_ELEMENTS else
+                                        "ncu capture of the VGG-16 workload, scaled by "
+                                        "elements"),
                      "algorithmic_bytes_per_launch": k1_bytes, "avg_launch_ms": k1_avg,
                      "share_of_step": k1_avg / (ms_max / K)},
         "cpu_baseline": cpu,
