@@ -4,9 +4,12 @@
 // abstract) sums the workers' sparse sets into one averaged dense update:
 // dense_j = ((+0 + v_0j) + v_1j + ... + v_(P-1)j) / P, workers in order, one
 // rounding per add, a correctly rounded division; positions no worker picked
-// are +0.  One CTA per tile of the flattened buffer: it stages all workers'
-// picks of the tile in shared memory, then each thread sums its own span of
-// positions worker by worker.  No atomics and no cross-thread reduction, so the
+// are +0.  One CTA per group of consecutive tiles of one layer (the plan sizes
+// groups to about a thousand expected picks): it stages all workers' picks of
+// the group in shared memory; the thread holding the lowest worker's pick of a
+// position finds the other workers' picks of it by binary search and adds them
+// in worker order.  Tiles expected to hold many picks form groups of one and
+// accumulate worker by worker in a shared tile instead.  No atomics, so the
 // result is bit-identical however the grid is scheduled.  With a weights
 // pointer the same kernel also applies the SGD update (weights -= dense).
 //
@@ -72,7 +75,7 @@ constexpr uint32_t kAggPickCap = 2048;
 constexpr uint32_t kAggOwnerMax = 512;
 
 struct AggShared {
-  uint16_t loc[kAggPickCap];             // pick position inside the tile, per worker ascending
+  uint32_t loc[kAggPickCap];             // pick position inside the group, per worker ascending
   float val[kAggPickCap];
   uint32_t base[LAGS_MAX_WORKERS + 1];   // first staged pick of each worker
   uint32_t rng[2 * LAGS_MAX_WORKERS];
@@ -89,16 +92,20 @@ struct AggTileAcc {
 constexpr size_t kAggAccOffset = (sizeof(AggShared) + 127) / 128 * 128;
 static_assert(kAggAccOffset % 16 == 0, "tile accumulator alignment");
 
-__global__ void __launch_bounds__(kAggThreads)
+__global__ void __launch_bounds__(kAggThreads, 4)
     k_aggregate(DevPlan dp, const uint32_t* __restrict__ idx, const float* __restrict__ val,
                 float* __restrict__ dense, float* __restrict__ weights, bool have_acc) {
   extern __shared__ __align__(16) unsigned char agg_smem[];
   AggShared& sh = *reinterpret_cast<AggShared*>(agg_smem);
   AggTileAcc& ta = *reinterpret_cast<AggTileAcc*>(agg_smem + kAggAccOffset);
   pdl_trigger();
-  const uint32_t t = blockIdx.x;
-  const TileDesc td = dp.tiles[t];
-  const LayerDesc ld = dp.layers[td.layer];
+  // a group of consecutive tiles of one layer: elements [gs, gs + glen)
+  const uint2 grp = dp.agg_groups[blockIdx.x];
+  const uint32_t t = grp.x, nt = grp.y;
+  const TileDesc td0 = dp.tiles[t];
+  const TileDesc tdl = dp.tiles[t + nt - 1];
+  const LayerDesc ld = dp.layers[td0.layer];
+  const TileDesc td{td0.start, tdl.start + tdl.len - td0.start, td0.layer, 0};
   const uint32_t P = dp.P;
   const float fP = (float)P;
   const uint64_t K = dp.K;
@@ -123,7 +130,7 @@ __global__ void __launch_bounds__(kAggThreads)
   if (tid < (int)P) {
     const uint32_t* first = dp.pick_first + (size_t)tid * dp.T;
     uint32_t a = __ldg(first + t);
-    uint32_t b = (t + 1 < ld.tile_end) ? __ldg(first + t + 1) : kend;
+    uint32_t b = (t + nt < ld.tile_end) ? __ldg(first + t + nt) : kend;
     a = min(max(a, ld.koff), kend);  // keeps a bad pick list inside the layer
     b = min(max(b, a), kend);
     sh.rng[2 * tid] = a;
@@ -149,21 +156,31 @@ __global__ void __launch_bounds__(kAggThreads)
       const uint32_t p = worker_of(i);
       const uint64_t slot = p * K + sh.rng[2 * p] + (i - sh.base[p]);
       const uint32_t x = __ldg(idx + slot) - td.start;
-      sh.loc[i] = (uint16_t)(x < td.len ? x : 0xFFFFu);
+      sh.loc[i] = x < td.len ? x : 0xFFFFFFFFu;
       sh.val[i] = __ldg(val + slot);
     }
   }
   const uint32_t head = min(td.len, (4u - (td.start & 3u)) & 3u);
   const uint32_t nvec = (td.len - head) / 4;
 
-  if (staged && (total <= kAggOwnerMax || !have_acc)) {
+  // the tile accumulator covers one tile: groups of several tiles use the
+  // owner search (the plan groups only tiles expected to hold few picks)
+  if (staged && (total <= kAggOwnerMax || !have_acc || nt > 1)) {
     // ---- few picks: zeros everywhere, then each position's first owner ----
-    for (uint32_t i = tid; i < head; i += kAggThreads) dense[td.start + i] = 0.0f;
-    float4* d4 = reinterpret_cast<float4*>(dense + td.start + head);
-    for (uint32_t v = tid; v < nvec; v += kAggThreads) __stcs(d4 + v, make_float4(0.f, 0.f, 0.f, 0.f));
-    for (uint32_t i = head + 4 * nvec + tid; i < td.len; i += kAggThreads) dense[td.start + i] = 0.0f;
-    __syncthreads();  // orders the zeros before the sums written below
-    for (uint32_t i = tid; i < total; i += kAggThreads) {
+    // Owned positions, their sums and their old weights are all gathered
+    // before this thread's first store: a load issued after stores waits for
+    // them to drain.
+    __syncthreads();  // staged picks visible to all threads
+    constexpr uint32_t OI = kAggPickCap / kAggThreads;  // staged picks per thread
+    uint32_t own_x[OI];
+    float own_v[OI], own_w[OI];
+#pragma unroll
+    for (uint32_t j = 0; j < OI; ++j) {
+      own_x[j] = 0xFFFFFFFFu;
+      own_v[j] = 0.0f;
+      own_w[j] = 0.0f;
+      const uint32_t i = tid + j * kAggThreads;
+      if (i >= total) continue;
       const uint32_t x = sh.loc[i];
       if (x >= td.len) continue;
       const uint32_t p = worker_of(i);
@@ -185,15 +202,40 @@ __global__ void __launch_bounds__(kAggThreads)
         }
       }
       if (first_owner) {
-        const float dv = __fdiv_rn(s, fP);
-        dense[td.start + x] = dv;
-        if (weights) weights[td.start + x] = __fsub_rn(weights[td.start + x], dv);
+        own_x[j] = x;
+        own_v[j] = __fdiv_rn(s, fP);
       }
+    }
+    if (weights) {
+#pragma unroll
+      for (uint32_t j = 0; j < OI; ++j)
+        if (own_x[j] != 0xFFFFFFFFu) own_w[j] = weights[td.start + own_x[j]];
+    }
+    for (uint32_t i = tid; i < head; i += kAggThreads) dense[td.start + i] = 0.0f;
+    {
+      // 8 independent 16-byte stores per trip: the loop overhead, not DRAM,
+      // limited a one-store loop
+      float4* d4 = reinterpret_cast<float4*>(dense + td.start + head);
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      uint32_t v = tid;
+      for (; v + 7 * kAggThreads < nvec; v += 8 * kAggThreads) {
+#pragma unroll
+        for (uint32_t u = 0; u < 8; ++u) __stcs(d4 + v + u * kAggThreads, z);
+      }
+      for (; v < nvec; v += kAggThreads) __stcs(d4 + v, z);
+    }
+    for (uint32_t i = head + 4 * nvec + tid; i < td.len; i += kAggThreads) dense[td.start + i] = 0.0f;
+    __syncthreads();  // orders the zeros before the sums written below
+#pragma unroll
+    for (uint32_t j = 0; j < OI; ++j) {
+      if (own_x[j] == 0xFFFFFFFFu) continue;
+      dense[td.start + own_x[j]] = own_v[j];
+      if (weights) weights[td.start + own_x[j]] = __fsub_rn(own_w[j], own_v[j]);
     }
     return;
   }
 
-  if (have_acc) {
+  if (have_acc && nt == 1) {
     // ---- many picks: worker-ordered accumulation in a shared tile ----
     float4* acc4 = reinterpret_cast<float4*>(ta.acc);
     for (uint32_t i = tid; i < kTile / 4; i += kAggThreads) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -318,8 +360,8 @@ cudaError_t configure_aggregate() {
 cudaError_t launch_aggregate(const DevPlan& dp, const uint32_t* idx, const float* val,
                              float* dense, float* weights, cudaStream_t s) {
   const size_t smem = dp.agg_tile_acc ? kAggAccOffset + sizeof(AggTileAcc) : sizeof(AggShared);
-  return launch_pdl(k_aggregate, dim3(dp.T), dim3(kAggThreads), smem, s, 1, dp, idx, val, dense,
-                    weights, dp.agg_tile_acc != 0);
+  return launch_pdl(k_aggregate, dim3(dp.n_groups), dim3(kAggThreads), smem, s, 1, dp, idx, val,
+                    dense, weights, dp.agg_tile_acc != 0);
 }
 
 cudaError_t launch_apply(uint32_t N, float* w, const float* dense, cudaStream_t s) {

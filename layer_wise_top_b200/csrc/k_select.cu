@@ -452,10 +452,49 @@ cudaError_t configure_select() {
   const int most = (int)stage_smem_bytes(kSelectStageMax);
   cudaError_t e = cudaFuncSetAttribute(k_select<1, kSelectThreadsSmall>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, most);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_select<kSelectCluster, kSelectThreads>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_select<kSelectCluster, kSelectThreads>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_select<kSelectClusterHuge, kSelectThreads>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_select<kSelectClusterHuge, kSelectThreads>,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
 }
+
+namespace {
+// Whether the current device can run one 16-CTA select cluster with `smem`
+// bytes of dynamic shared memory per CTA (cached per device and size).
+bool huge_clusters_fit(size_t smem) {
+  static int cached_dev = -1;
+  static size_t cached_smem = 0;
+  static bool cached_fit = false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev == cached_dev && smem == cached_smem) return cached_fit;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kSelectClusterHuge);
+  cfg.blockDim = dim3(kSelectThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kSelectClusterHuge;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  const cudaError_t e = cudaOccupancyMaxActiveClusters(
+      &clusters, k_select<kSelectClusterHuge, kSelectThreads>, &cfg);
+  if (e != cudaSuccess) cudaGetLastError();  // clear; use 8-CTA clusters instead
+  cached_dev = dev;
+  cached_smem = smem;
+  cached_fit = e == cudaSuccess && clusters > 0;
+  return cached_fit;
+}
+}  // namespace
 
 cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out_idx,
                           float* out_val, cudaStream_t s) {
@@ -466,10 +505,23 @@ cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out
     if (e != cudaSuccess) return e;
   }
   if (dp.n_large) {
+    cudaError_t e = launch_pdl(k_select<kSelectCluster, kSelectThreads>,
+                               dim3(dp.n_large * kSelectCluster, dp.P), dim3(kSelectThreads),
+                               stage_smem_bytes(dp.stage_large), s, kSelectCluster, dp, wp,
+                               dp.sel_large, dp.stage_large, out_idx, out_val);
+    if (e != cudaSuccess) return e;
+  }
+  if (dp.n_huge) {
+    const size_t smem = stage_smem_bytes(dp.stage_huge);
+    if (huge_clusters_fit(smem))
+      return launch_pdl(k_select<kSelectClusterHuge, kSelectThreads>,
+                        dim3(dp.n_huge * kSelectClusterHuge, dp.P), dim3(kSelectThreads), smem, s,
+                        kSelectClusterHuge, dp, wp, dp.sel_huge, dp.stage_huge, out_idx, out_val);
+    // 8-CTA clusters with the same staging: shares that do not fit are read
+    // from global memory on every pass (slower, same result)
     return launch_pdl(k_select<kSelectCluster, kSelectThreads>,
-                      dim3(dp.n_large * kSelectCluster, dp.P), dim3(kSelectThreads),
-                      stage_smem_bytes(dp.stage_large), s, kSelectCluster, dp, wp, dp.sel_large,
-                      dp.stage_large, out_idx, out_val);
+                      dim3(dp.n_huge * kSelectCluster, dp.P), dim3(kSelectThreads), smem, s,
+                      kSelectCluster, dp, wp, dp.sel_huge, dp.stage_huge, out_idx, out_val);
   }
   return cudaSuccess;
 }

@@ -136,9 +136,10 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
       plan->sparse.push_back((uint32_t)l);
       for (uint64_t j0 = 0; j0 < k; j0 += 256) plan->pick_chunks.push_back(make_uint2(l, j0));
       // one CTA when its shared memory can stage the expected candidates with
-      // a third to spare, else an 8-CTA cluster
+      // a third to spare, else an 8-CTA cluster, else a 16-CTA cluster
       const double expect = expected_candidates(ld);
-      (1.33 * expect + 512.0 <= (double)kSelectStageMax ? plan->sel_small : plan->sel_large)
+      auto fits = [&](int ctas) { return 1.33 * expect / ctas + 512.0 <= (double)kSelectStageMax; };
+      (fits(1) ? plan->sel_small : fits(kSelectCluster) ? plan->sel_large : plan->sel_huge)
           .push_back((uint32_t)l);
     }
     if (slots >= (1ull << 32) || koff + k >= (1ull << 32)) {
@@ -170,11 +171,31 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
   }
   plan->stage_small = stage_for(plan->sel_small, 1);
   plan->stage_large = stage_for(plan->sel_large, kSelectCluster);
+  plan->stage_huge = stage_for(plan->sel_huge, kSelectClusterHuge);
+  // aggregation groups: consecutive tiles of one layer, about a thousand
+  // expected picks (P k / d per element) per group and at most 16 tiles, but
+  // never so few groups that the GPU has fewer than 4 per SM; tiles expected
+  // to need the shared tile accumulator stay alone
+  {
+    const double cap_by_count =
+        std::max(1.0, std::floor((double)plan->tiles.size() / (4.0 * 148.0)));
+    for (const LayerDesc& ld : plan->layers) {
+      const bool dense_l = ld.k == ld.d;
+      const double per_tile =
+          dense_l ? 0.0 : (double)num_workers * ld.k * std::min<double>(kTile, ld.d) / ld.d;
+      double g = dense_l ? 4.0 : per_tile > 256.0 ? 1.0 : 1024.0 / std::max(per_tile, 1.0);
+      g = std::max(1.0, std::min({g, 16.0, cap_by_count}));
+      const uint32_t gi = (uint32_t)g;
+      for (uint32_t t0 = ld.tile_begin; t0 < ld.tile_end; t0 += gi)
+        plan->agg_groups.push_back(make_uint2(t0, std::min(gi, ld.tile_end - t0)));
+    }
+  }
   // select the layers with the most picks first, so the longest CTAs start early
   auto by_k_desc = [plan](uint32_t a, uint32_t b) {
     return plan->layers[a].k != plan->layers[b].k ? plan->layers[a].k > plan->layers[b].k : a < b;
   };
   std::sort(plan->sel_large.begin(), plan->sel_large.end(), by_k_desc);
+  std::sort(plan->sel_huge.begin(), plan->sel_huge.end(), by_k_desc);
   std::sort(plan->sel_small.begin(), plan->sel_small.end(), by_k_desc);
   std::sort(plan->sparse.begin(), plan->sparse.end(), by_k_desc);
   plan->N = off;
@@ -186,6 +207,7 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
   plan->o_tiles = section(cur, T * sizeof(TileDesc));
   plan->o_large = section(cur, (plan->sel_large.size() + 1) * 4);
   plan->o_small = section(cur, (plan->sel_small.size() + 1) * 4);
+  plan->o_huge = section(cur, (plan->sel_huge.size() + 1) * 4);
   plan->o_sparse = section(cur, (plan->sparse.size() + 1) * 4);
   plan->o_lo = section(cur, P * (uint64_t)num_layers * 4);
   plan->o_cnt = section(cur, P * T * 4);
@@ -193,6 +215,7 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
   plan->o_cidx = section(cur, P * (plan->C + 1) * 4);
   plan->o_first = section(cur, P * T * 4);
   plan->o_chunks = section(cur, (plan->pick_chunks.size() + 1) * sizeof(uint2));
+  plan->o_groups = section(cur, (plan->agg_groups.size() + 1) * sizeof(uint2));
   plan->o_status = section(cur, kStatusWords * 4);
   plan->ws_bytes = (cur + kAlign - 1) / kAlign * kAlign;
   *out_plan = plan;
@@ -248,9 +271,12 @@ lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t byt
   if (e == cudaSuccess) e = up(plan->o_tiles, plan->tiles.data(), plan->tiles.size() * sizeof(TileDesc));
   if (e == cudaSuccess) e = up(plan->o_large, plan->sel_large.data(), plan->sel_large.size() * 4);
   if (e == cudaSuccess) e = up(plan->o_small, plan->sel_small.data(), plan->sel_small.size() * 4);
+  if (e == cudaSuccess) e = up(plan->o_huge, plan->sel_huge.data(), plan->sel_huge.size() * 4);
   if (e == cudaSuccess) e = up(plan->o_sparse, plan->sparse.data(), plan->sparse.size() * 4);
   if (e == cudaSuccess)
     e = up(plan->o_chunks, plan->pick_chunks.data(), plan->pick_chunks.size() * sizeof(uint2));
+  if (e == cudaSuccess)
+    e = up(plan->o_groups, plan->agg_groups.data(), plan->agg_groups.size() * sizeof(uint2));
   if (e == cudaSuccess) e = cudaMemsetAsync(base + plan->o_status, 0, kStatusWords * 4, s);
   // pageable sources: make sure the copies are done before returning
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -308,7 +334,7 @@ lags_status lags_plan_kernel_launches(const lags_plan* plan, int32_t* sparsify,
   const bool any_sparse = !plan->sparse.empty();
   if (sparsify)
     *sparsify = (any_sparse ? 1 : 0) + 1 + (plan->sel_small.empty() ? 0 : 1) +
-                (plan->sel_large.empty() ? 0 : 1);
+                (plan->sel_large.empty() ? 0 : 1) + (plan->sel_huge.empty() ? 0 : 1);
   if (aggregate) *aggregate = 2;
   if (apply) *apply = 1;
   return LAGS_OK;

@@ -26,6 +26,9 @@ constexpr uint32_t kEstThreads = 512;
 // Cluster size used to select layers whose expected candidates exceed what one
 // CTA stages in shared memory; the other layers use one CTA.
 constexpr int kSelectCluster = 8;
+// Layers whose expected candidates exceed what 8 CTAs stage use a 16-CTA
+// cluster (a non-portable size; checked on the device before use).
+constexpr int kSelectClusterHuge = 16;
 constexpr uint32_t kSelectThreads = 512;       // clustered select
 constexpr uint32_t kSelectThreadsSmall = 512;  // single-CTA select (256 measured slower)
 constexpr uint32_t kSelectWindow = 2048;  // tiles whose prefix sits in smem at once
@@ -78,7 +81,8 @@ enum StatusWord : uint32_t { kStatusFlags = 0, kStatusFallbacks = 1, kStatusWord
 struct DevPlan {
   const LayerDesc* layers;
   const TileDesc* tiles;
-  const uint32_t* sel_large;  // sparse layers selected by a cluster
+  const uint32_t* sel_large;  // sparse layers selected by an 8-CTA cluster
+  const uint32_t* sel_huge;   // sparse layers selected by a 16-CTA cluster
   const uint32_t* sel_small;  // sparse layers selected by one CTA
   const uint32_t* sparse;     // all sparse layers (estimate pass)
   uint32_t* lo_key;           // [P][L] candidate threshold key
@@ -87,13 +91,14 @@ struct DevPlan {
   uint32_t* cand_idx;         // [P][C]
   uint32_t* pick_first;       // [P][T] first pick slot of each tile (aggregate)
   const uint2* pick_chunks;   // (sparse layer, first slot) per 256 pick slots
+  const uint2* agg_groups;    // (first tile, tiles) per aggregation CTA
   uint32_t* status;           // kStatusWords
   uint32_t L, T, P;
-  uint32_t n_large, n_small, n_sparse, n_chunks;
+  uint32_t n_large, n_small, n_huge, n_sparse, n_chunks, n_groups;
   uint32_t N;
   uint64_t K;
   uint64_t C;  // candidate slots per worker
-  uint32_t stage_small, stage_large;  // shared-memory staging capacity per select launch
+  uint32_t stage_small, stage_large, stage_huge;  // select staging capacity per launch
   uint32_t agg_tile_acc;  // aggregation launches carry a shared tile accumulator
 };
 

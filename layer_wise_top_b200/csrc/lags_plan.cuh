@@ -14,16 +14,19 @@ struct lags_plan {
   uint64_t N = 0, K = 0, C = 0;
   std::vector<lags::LayerDesc> layers;
   std::vector<lags::TileDesc> tiles;
-  std::vector<uint32_t> sel_large, sel_small, sparse;
+  std::vector<uint32_t> sel_large, sel_small, sel_huge, sparse;
   std::vector<uint2> pick_chunks;  // (sparse layer, first slot) per 256 pick slots
+  std::vector<uint2> agg_groups;   // (first tile, tiles) per aggregation CTA
   std::vector<int64_t> off, k, koff;
   // workspace sections (byte offsets)
-  size_t o_layers = 0, o_tiles = 0, o_large = 0, o_small = 0, o_sparse = 0, o_lo = 0, o_cnt = 0,
-         o_cval = 0, o_cidx = 0, o_first = 0, o_chunks = 0, o_status = 0, ws_bytes = 0;
+  size_t o_layers = 0, o_tiles = 0, o_large = 0, o_small = 0, o_huge = 0, o_sparse = 0, o_lo = 0,
+         o_cnt = 0,
+         o_cval = 0, o_cidx = 0, o_first = 0, o_chunks = 0, o_groups = 0, o_status = 0,
+         ws_bytes = 0;
   void* ws = nullptr;
   int device = -1;
   cudaEvent_t ev_before = nullptr, ev_after = nullptr;
-  uint32_t stage_small = 0, stage_large = 0;  // select staging capacity per launch
+  uint32_t stage_small = 0, stage_large = 0, stage_huge = 0;  // select staging per launch
   uint32_t agg_tile_acc = 0;  // some tile expects more picks than the owner search handles
   lags::DevPlan dp{};  // device view once a workspace is bound
 };
@@ -38,6 +41,7 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.tiles = (const TileDesc*)(base + plan->o_tiles);
   dp.sel_large = (const uint32_t*)(base + plan->o_large);
   dp.sel_small = (const uint32_t*)(base + plan->o_small);
+  dp.sel_huge = (const uint32_t*)(base + plan->o_huge);
   dp.sparse = (const uint32_t*)(base + plan->o_sparse);
   dp.lo_key = (uint32_t*)(base + plan->o_lo);
   dp.tile_cnt = (uint32_t*)(base + plan->o_cnt);
@@ -45,18 +49,22 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.cand_idx = (uint32_t*)(base + plan->o_cidx);
   dp.pick_first = (uint32_t*)(base + plan->o_first);
   dp.pick_chunks = (const uint2*)(base + plan->o_chunks);
+  dp.agg_groups = (const uint2*)(base + plan->o_groups);
   dp.status = (uint32_t*)(base + plan->o_status);
   dp.L = (uint32_t)plan->L;
   dp.T = (uint32_t)plan->tiles.size();
   dp.P = (uint32_t)plan->P;
   dp.n_large = (uint32_t)plan->sel_large.size();
   dp.n_small = (uint32_t)plan->sel_small.size();
+  dp.n_huge = (uint32_t)plan->sel_huge.size();
   dp.n_sparse = (uint32_t)plan->sparse.size();
   dp.n_chunks = (uint32_t)plan->pick_chunks.size();
+  dp.n_groups = (uint32_t)plan->agg_groups.size();
   dp.N = (uint32_t)plan->N;
   dp.K = plan->K;
   dp.C = plan->C;
   dp.stage_small = plan->stage_small;
   dp.stage_large = plan->stage_large;
+  dp.stage_huge = plan->stage_huge;
   dp.agg_tile_acc = plan->agg_tile_acc;
 }

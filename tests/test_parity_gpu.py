@@ -99,6 +99,18 @@ def test_large_layers_cluster_select():
                      expect_fallbacks=lambda fb: fb == 0)
 
 
+def test_sixteen_cta_cluster_select():
+    # ~149k expected candidates: more than eight CTAs stage, so the layer is
+    # selected by a 16-CTA cluster (or 8 CTAs reading from global memory if
+    # the device cannot host the larger cluster)
+    sizes = [2_600_000, 7]
+    dens = [0.05, 1.0]
+    w = WORKLOADS["resnet50"].scaled("huge", P=2, steps=2,
+                                     tensors=[Tensor(f"t{i}", (d,)) for i, d in enumerate(sizes)])
+    run_full_compare(sizes, dens, 2, w.lr, 2, synth_grad_fn(w),
+                     expect_fallbacks=lambda fb: fb == 0)
+
+
 # ----------------------------------------------------------------- ties / degenerate
 def _np_grads(gen, sizes, P, steps):
     N = sum(sizes)
