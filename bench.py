@@ -48,6 +48,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="vgg16",
                     choices=["resnet20", "vgg16", "resnet50", "lstm_ptb", "gpt_1_3b"])
+    ap.add_argument("--dp", action="store_true",
+                    help="data-parallel LAGS: split the job's P workers over the ranks and "
+                         "all-gather their pick lists (strong scaling) instead of replicas")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -219,7 +222,23 @@ def run_ours(args):
 
     w = WORKLOADS[args.config]
     P, N = w.P, w.N
-    plan = Plan(w.sizes, w.densities, P, device=dev)
+    dp = None
+    if args.dp:
+        # the job's P workers split over the ranks; every step all-gathers the
+        # pick lists and aggregates all P workers on every rank
+        if world == 1:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", "29531")
+            dist.init_process_group("nccl", rank=0, world_size=1, device_id=dev,
+                                    timeout=datetime.timedelta(seconds=300))
+        if P % world:
+            raise SystemExit(f"--dp needs the {P} workers to divide over {world} ranks")
+        from layer_wise_top_b200.dist import DataParallelLags
+        dp = DataParallelLags.create(w.sizes, w.densities, P // world, dev)
+        P = P // world  # workers held by this rank
+        plan = dp.local
+    else:
+        plan = Plan(w.sizes, w.densities, P, device=dev)
     step_bytes = P * N * 4
     pool = max(1, min(args.warmup + args.steps, POOL_BUDGET_BYTES // step_bytes))
     grads = []
@@ -235,9 +254,12 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     n_sparsify, n_aggregate, _ = plan.kernel_launches()
-    launches_per_step = n_sparsify + n_aggregate
+    launches_per_step = n_sparsify + n_aggregate  # (the all-gather in --dp is NCCL's)
 
     def step(i):
+        if dp is not None:
+            dp.step(grads[i % pool], res, w.lr, dense, weights)
+            return
         plan.sparsify(grads[i % pool], res, w.lr, idx, val)
         plan.aggregate_apply(idx, val, dense, weights)
 
@@ -276,7 +298,7 @@ def run_ours(args):
     # end to end through the same calls: inputs from pinned host memory each
     # step, the updated weights read back each step
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and dp is None:
         host = [torch.empty(N, dtype=torch.float32, pin_memory=True) for _ in range(P)]
         for p in range(P):
             host[p].copy_(grads[0][p])
@@ -308,7 +330,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
 
-    if world > 1:
+    if world > 1 or dp is not None:
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
     if rank != 0:
@@ -318,17 +340,21 @@ def run_ours(args):
     k1_avg = sum(k1_ms) / len(k1_ms)
     k1_bytes = 12 * P * N
     achieved = k1_bytes / (k1_avg / 1e3) / 1e9
+    job_elems = (P * world if dp is not None else world * P) * N  # all ranks' elements
     line = {
         "metric": METRIC,
-        "value": world * P * N * K / (ms_max / 1e3) / 1e9,
+        "value": job_elems * K / (ms_max / 1e3) / 1e9,
         "unit": "Gelem/s",
         "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_max / K,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": "strong" if dp is not None else "weak",
+        "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic: Philox4x32-10 gradients with the workload's tensor shapes",
         "config": workload_config(
-            w, parallelism=f"replicas x{world}", grad_pool_steps=pool,
+            w, parallelism=(f"data-parallel: {P} workers per rank x {world} ranks, NCCL "
+                            f"all-gather of pick lists" if dp is not None else
+                            f"replicas x{world}"), grad_pool_steps=pool,
             l2=f"inputs larger than L2: {12 * P * N / 1e9:.2f} GB streamed per step vs "
                f"{L2_BYTES / 1e6:.0f} MB L2",
             step="lags_sparsify + lags_aggregate_apply (aggregate and apply fused)"),

@@ -216,6 +216,29 @@ LAGS_API lags_status lags_sparsify_static(lags_plan* plan, const float* const* g
 LAGS_API lags_status lags_plan_set_events(lags_plan* plan, void* before, void* after);
 
 /*
+ * lags_adaptive_densities - per-layer densities from each layer's
+ * communication-to-computation ratio ("Layer-wise Adaptive Gradient
+ * Sparsification ..." review, "proposed method": each layer's sparsification
+ * ratio is set by its communication-to-computation ratio so that its
+ * communication hides behind computation).  Host only, no device.
+ *   layer_sizes       host, [num_layers] d_l > 0, in forward order.
+ *   backward_seconds  host, [num_layers] t_l >= 0: backward time of each layer.
+ *   alpha, beta       message model: a layer sending k picks takes
+ *                     alpha + beta * 8 * k seconds (alpha, beta >= 0).
+ *   rho_min           smallest density, in (0, 1].
+ *   out_densities     host, [num_layers] rho_l in [rho_min, 1].
+ * Rule: backward produces layers L-1 .. 0; layer l's gradient exists at
+ * R_l = sum_{j >= l} t_j, its message starts at max(R_l, end of the previous
+ * message) and must end by R_0 (the end of the backward pass).  Layer l gets
+ * the largest rho in [rho_min, 1] with k_l = ceil(rho d_l) meeting that
+ * deadline (rho_min when none does); messages go out in production order.
+ */
+LAGS_API lags_status lags_adaptive_densities(const int64_t* layer_sizes,
+                                             const double* backward_seconds, int32_t num_layers,
+                                             double alpha, double beta, double rho_min,
+                                             double* out_densities);
+
+/*
  * lags_plan_kernel_launches - how many kernels one lags_sparsify, one
  * lags_aggregate (or lags_aggregate_apply) and one lags_apply call enqueue for
  * this plan (any output pointer may be NULL).

@@ -25,7 +25,8 @@ LAGS_FLAG_TIMEOUT = 0x4
 EXPORTED = ("lags_plan_create", "lags_plan_destroy", "lags_plan_info", "lags_plan_layer",
             "lags_plan_set_workspace", "lags_sparsify", "lags_aggregate", "lags_apply",
             "lags_status_poll", "lags_plan_set_events", "lags_sparsify_static",
-            "lags_aggregate_apply", "lags_plan_kernel_launches", "lags_error_string")
+            "lags_aggregate_apply", "lags_plan_kernel_launches", "lags_adaptive_densities",
+            "lags_error_string")
 
 
 class LagsError(RuntimeError):
@@ -55,6 +56,9 @@ def _load() -> ctypes.CDLL:
     lib.lags_aggregate_apply.argtypes = [vp, vp, vp, vp, vp, vp]
     i32p = ctypes.POINTER(ctypes.c_int32)
     lib.lags_plan_kernel_launches.argtypes = [vp, i32p, i32p, i32p]
+    dp_ = ctypes.POINTER(ctypes.c_double)
+    lib.lags_adaptive_densities.argtypes = [i64p, dp_, i32, ctypes.c_double, ctypes.c_double,
+                                            ctypes.c_double, dp_]
     lib.lags_status_poll.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32),
                                      ctypes.POINTER(ctypes.c_uint32), vp]
     lib.lags_plan_set_events.argtypes = [vp, vp, vp]
@@ -159,6 +163,21 @@ def lags_plan_kernel_launches(plan) -> Tuple[int, int, int]:
     _check(_LIB.lags_plan_kernel_launches(plan, ctypes.byref(a), ctypes.byref(b),
                                           ctypes.byref(c)), "lags_plan_kernel_launches")
     return a.value, b.value, c.value
+
+
+def lags_adaptive_densities(layer_sizes: Sequence[int], backward_seconds: Sequence[float],
+                            alpha: float, beta: float, rho_min: float) -> list:
+    """Per-layer densities from each layer's communication-to-computation
+    ratio (see include/lags.h for the rule)."""
+    L = len(layer_sizes)
+    if len(backward_seconds) != L:
+        raise ValueError("layer_sizes and backward_seconds differ in length")
+    sizes = (ctypes.c_int64 * max(L, 1))(*[int(x) for x in layer_sizes])
+    t = (ctypes.c_double * max(L, 1))(*[float(x) for x in backward_seconds])
+    out = (ctypes.c_double * max(L, 1))()
+    _check(_LIB.lags_adaptive_densities(sizes, t, L, float(alpha), float(beta), float(rho_min),
+                                        out), "lags_adaptive_densities")
+    return [out[i] for i in range(L)]
 
 
 def lags_apply(plan, weights: int, dense_out: int, stream: int = 0) -> None:

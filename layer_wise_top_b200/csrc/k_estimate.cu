@@ -2,8 +2,8 @@
 //
 // Before the fused pass streams a layer, one CTA per sparse (worker, layer)
 // draws a sample of m_l entries of acc = residual + lr*grad (the whole layer
-// when it is at most kSampleMax long, otherwise 256 evenly spaced runs of 64
-// contiguous entries) and finds the magnitude key of the sample's r*-th
+// when it is at most kSampleMax long, otherwise 256 runs of 64 contiguous
+// entries, one at a hashed offset inside each of 256 equal strata) and finds the magnitude key of the sample's r*-th
 // largest entry, rounded down to a level-1 radix bin edge.  The fused pass
 // then keeps every entry at or above that key as a candidate.  r* is chosen on
 // the host so that, for a sample drawn from the layer, the candidates hold the
@@ -15,6 +15,16 @@
 #include "lags_internal.cuh"
 
 namespace lags {
+
+// Integer finaliser (xor-shift-multiply) to place the sample runs.
+__device__ __forceinline__ uint32_t mix32(uint32_t x) {
+  x ^= x >> 16;
+  x *= 0x7FEB352Du;
+  x ^= x >> 15;
+  x *= 0x846CA68Bu;
+  x ^= x >> 16;
+  return x;
+}
 
 __global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs wp, float lr) {
   extern __shared__ uint32_t s_keys[];  // kSampleMax
@@ -36,8 +46,13 @@ __global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs
   // sample positions: the whole layer, or nchunk runs of kSampleChunk spread
   // evenly over it
   if (m != ld.d)
-    for (uint32_t c = threadIdx.x; c < nchunk; c += kEstThreads)
-      s_chunk[c] = ld.off + (uint32_t)((uint64_t)c * (ld.d - kSampleChunk) / (nchunk - 1));
+    for (uint32_t c = threadIdx.x; c < nchunk; c += kEstThreads) {
+      // stratified: run c lies at a hashed offset inside the c-th of nchunk
+      // equal strata, so every region of the layer is sampled in proportion
+      const uint32_t a = (uint32_t)((uint64_t)c * ld.d / nchunk);
+      const uint32_t b = (uint32_t)((uint64_t)(c + 1) * ld.d / nchunk);
+      s_chunk[c] = ld.off + a + mix32(c * 0x9E3779B9u + layer) % (b - a - kSampleChunk + 1);
+    }
   __syncthreads();
   constexpr uint32_t U = 8;  // loads per array in flight per thread
   for (uint32_t i0 = 0; i0 < m; i0 += kEstThreads * U) {

@@ -34,11 +34,16 @@ size_t section(size_t& cursor, size_t bytes) {
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
-// Candidate slots per tile for a layer picking k of d entries: about six times
-// the expected number of candidates per tile plus a floor, in warp multiples.
-uint32_t slot_capacity(uint64_t d, uint64_t k) {
-  double expect = (double)kTile * 6.0 * (double)k / (double)d;
-  double cap = std::ceil(expect) + 64.0;
+// Candidate slots per tile for a layer of d entries split in `ntiles` tiles,
+// expecting `cand` candidates: six times a tile's share (candidates spread
+// evenly), or up to 24 times it (and at most 1.5x the layer's expected total)
+// when the large values crowd into a few tiles, e.g. a segment spanning
+// tensors of different gradient scales; plus 64, in warp multiples.
+uint32_t slot_capacity(uint64_t d, uint64_t ntiles, double cand) {
+  const double share = cand * std::min<double>(kTile, (double)d) / (double)d;
+  const double spread = 6.0 * share;
+  const double crowded = std::min(1.5 * cand, 24.0 * cand / (double)ntiles);
+  const double cap = std::ceil(std::max(spread, crowded)) + 64.0;
   uint64_t c = ((uint64_t)cap + 31) / 32 * 32;
   return (uint32_t)(c < kTile ? c : kTile);
 }
@@ -128,11 +133,11 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
     ld.tile_end = (uint32_t)plan->tiles.size();
     const bool dense = k == (uint64_t)d;
     if (!dense) {
-      ld.slot_cap = slot_capacity(d, k);
-      ld.slot_base = (uint32_t)slots;
-      slots += (uint64_t)(ld.tile_end - ld.tile_begin) * ld.slot_cap;
       ld.sample = (uint32_t)((uint64_t)d < kSampleMax ? d : kSampleMax);
       ld.rank = sample_rank(ld.sample, d, k);
+      ld.slot_cap = slot_capacity(d, ld.tile_end - ld.tile_begin, expected_candidates(ld));
+      ld.slot_base = (uint32_t)slots;
+      slots += (uint64_t)(ld.tile_end - ld.tile_begin) * ld.slot_cap;
       plan->sparse.push_back((uint32_t)l);
       for (uint64_t j0 = 0; j0 < k; j0 += 256) plan->pick_chunks.push_back(make_uint2(l, j0));
       // one CTA when its shared memory can stage the expected candidates with
@@ -326,6 +331,37 @@ lags_status lags_aggregate_apply(lags_plan* plan, const uint32_t* idx, const flo
   cudaError_t e = launch_pick_bounds(plan->dp, idx, s);
   if (e == cudaSuccess) e = launch_aggregate(plan->dp, idx, val, dense_out, weights, s);
   return cuda_status(e);
+}
+
+lags_status lags_adaptive_densities(const int64_t* layer_sizes, const double* backward_seconds,
+                                    int32_t num_layers, double alpha, double beta,
+                                    double rho_min, double* out_densities) {
+  if (!layer_sizes || !backward_seconds || !out_densities || num_layers < 1) return LAGS_ERR_INVALID_ARG;
+  if (!(alpha >= 0.0) || !(beta >= 0.0) || !(rho_min > 0.0) || !(rho_min <= 1.0))
+    return LAGS_ERR_INVALID_ARG;
+  double end = 0.0;  // R_0: the backward pass ends after every layer
+  for (int32_t l = 0; l < num_layers; ++l) {
+    if (layer_sizes[l] <= 0 || !(backward_seconds[l] >= 0.0)) return LAGS_ERR_INVALID_ARG;
+    end += backward_seconds[l];
+  }
+  double produced = 0.0, link_free = 0.0;
+  for (int32_t l = num_layers - 1; l >= 0; --l) {
+    produced += backward_seconds[l];  // R_l = sum_{j >= l} t_j
+    const double start = std::max(produced, link_free);
+    const double d = (double)layer_sizes[l];
+    const double budget = end - start - alpha;  // seconds left for 8 k beta
+    double rho = rho_min;
+    if (budget >= 0.0) {
+      const double kmax = beta > 0.0 ? std::floor(budget / (8.0 * beta)) : d;
+      rho = std::min(1.0, std::max(rho_min, kmax / d));
+    }
+    // the k this density yields (the rule of lags_plan_create), for the link
+    const double kd = std::ceil(rho * d);
+    const double k = kd < 1.0 ? 1.0 : std::min(kd, d);
+    out_densities[l] = rho;
+    link_free = start + alpha + beta * 8.0 * k;
+  }
+  return LAGS_OK;
 }
 
 lags_status lags_plan_kernel_launches(const lags_plan* plan, int32_t* sparsify,

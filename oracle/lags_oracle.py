@@ -28,6 +28,13 @@ and in the design notes:
       in order 0..P-1, a worker that did not pick j contributing nothing, and
       a true IEEE division by P.
   R7  weights <- fl32(weights - dense)  (plain S-SGD, lr already inside acc).
+  R8  adaptive densities ("proposed method": each layer's ratio follows its
+      communication-to-computation ratio so that communication hides behind
+      computation): layers come out of backprop in reverse order; layer l's
+      message starts when its gradient exists (sum of the backward times of
+      layers >= l) and the previous message has ended, takes alpha + 8 beta k
+      seconds, and gets the largest density whose message ends by the end of
+      the backward pass (rho_min if none does).
 """
 from __future__ import annotations
 
@@ -149,6 +156,29 @@ def aggregate(N: int, out_idx: np.ndarray, out_val: np.ndarray) -> np.ndarray:
 def apply_update(weights: np.ndarray, dense: np.ndarray) -> np.ndarray:
     """weights - dense, one fp32 rounding (R7)."""
     return np.subtract(weights, dense, dtype=F32)
+
+
+def adaptive_densities(sizes: Sequence[int], backward_seconds: Sequence[float], alpha: float,
+                       beta: float, rho_min: float) -> List[float]:
+    """Per-layer densities by reading R8, in the order of operations written
+    there (double precision)."""
+    end = 0.0
+    for t in backward_seconds:
+        end += float(t)
+    out = [0.0] * len(sizes)
+    produced, link_free = 0.0, 0.0
+    for l in range(len(sizes) - 1, -1, -1):
+        produced += float(backward_seconds[l])
+        start = max(produced, link_free)
+        d = float(sizes[l])
+        budget = end - start - alpha
+        rho = rho_min
+        if budget >= 0.0:
+            kmax = math.floor(budget / (8.0 * beta)) if beta > 0.0 else d
+            rho = min(1.0, max(rho_min, kmax / d))
+        out[l] = rho
+        link_free = start + alpha + beta * 8.0 * k_of(int(sizes[l]), rho)
+    return out
 
 
 def run_workload(sizes: Sequence[int], densities: Sequence[float], P: int, lr: float,
