@@ -179,11 +179,12 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
   plan->stage_huge = stage_for(plan->sel_huge, kSelectClusterHuge);
   // aggregation groups: consecutive tiles of one layer, about a thousand
   // expected picks (P k / d per element) per group and at most 16 tiles, but
-  // never so few groups that the GPU has fewer than 4 per SM; tiles expected
+  // never so few groups that the GPU has fewer than 8 per SM (grouping only
+  // pays when tiles far outnumber the CTAs that run at once); tiles expected
   // to need the shared tile accumulator stay alone
   {
     const double cap_by_count =
-        std::max(1.0, std::floor((double)plan->tiles.size() / (4.0 * 148.0)));
+        std::max(1.0, std::floor((double)plan->tiles.size() / (8.0 * 148.0)));
     for (const LayerDesc& ld : plan->layers) {
       const bool dense_l = ld.k == ld.d;
       const double per_tile =
