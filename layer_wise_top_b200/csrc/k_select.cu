@@ -25,6 +25,7 @@
 
 #include "block_ops.cuh"
 #include "lags_internal.cuh"
+#include "tma.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -58,12 +59,6 @@ struct Cluster {
   }
 };
 
-// First element of tile t of layer ld: tiles start on multiples of kTile in
-// the flattened buffer, except a layer's first tile, which starts at the layer.
-__device__ __forceinline__ uint32_t tile_start(const LayerDesc& ld, uint32_t t) {
-  return t == ld.tile_begin ? ld.off : (ld.off / kTile + (t - ld.tile_begin)) * kTile;
-}
-
 template <int NT>
 struct SelectShared {
   uint32_t hist[kBins];          // this CTA's histogram (then the merged copy)
@@ -83,10 +78,10 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   __shared__ SelectShared<NT> sh;
   // CTA 0 of a cluster: cluster-wide histograms, one per level
   __shared__ uint32_t merged[CL > 1 ? 3 : 1][kBins];
-  // staged candidates: stage_cap values, then stage_cap 16-bit offsets inside
-  // their tile (the index is tile_start + offset)
+  // staged candidates: stage_cap values, then their stage_cap global indices
   extern __shared__ __align__(16) float stage_val[];
-  uint16_t* stage_off = reinterpret_cast<uint16_t*>(stage_val + stage_cap);
+  uint32_t* stage_idx = reinterpret_cast<uint32_t*>(stage_val + stage_cap);
+  __shared__ __align__(8) uint64_t stage_bar;  // completion of the bulk copies
   pdl_trigger();
   const uint32_t rank = C::rank();
   const uint32_t layer = list[blockIdx.x / CL];
@@ -184,60 +179,66 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
       __syncthreads();
     }
   };
-  // Staged share: the values of this CTA's candidates, in index order, copied
-  // once to shared memory (the tile prefix sums stay in sh.tpre, so a staged
-  // position maps back to its candidate slot for the index at emission).
-  const bool staged = fast && my <= stage_cap && tb - ta <= kSelectWindow;
-  if (staged) {
+  // Staged share: this CTA's candidate runs (one per tile, in index order) are
+  // copied to shared memory by the bulk-copy engine, one cp.async.bulk per
+  // tile and array, completing on one mbarrier.  Each run is padded to a
+  // 16-byte multiple with entries of magnitude key 0; the share is staged only
+  // when the candidate threshold is at least 2^20 (level-0 bin >= 1), so every
+  // real candidate outranks the padding and the padding is never counted into
+  // a pick, a tie or the bin holding the k-th largest key.
+  bool staged = false, stage_timeout = false;
+  uint32_t my_pad = 0;  // staged entries, padding included
+  const uint32_t lo_key = dp.lo_key[(size_t)p * dp.L + layer];
+  if (fast && tb - ta <= kSelectWindow && lo_key >= (1u << 20)) {
     const uint32_t nw = tb - ta;
     constexpr int PER = kSelectWindow / NT;
     uint32_t c[PER], sum = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const uint32_t q = tid * PER + i;
-      c[i] = q < nw ? __ldg(cnt + ta + q) : 0u;
+      c[i] = q < nw ? (__ldg(cnt + ta + q) + 3u) & ~3u : 0u;
       sum += c[i];
     }
-    uint32_t wtotal;
-    uint32_t ex = block_excl_scan<NT>(sum, sh.tmp, &wtotal);
+    uint32_t ex = block_excl_scan<NT>(sum, sh.tmp, &my_pad);
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const uint32_t q = tid * PER + i;
       if (q < nw) sh.tpre[q] = ex;
       ex += c[i];
     }
-    if (tid == 0) sh.tpre[nw] = wtotal;
-    __syncthreads();
-    constexpr uint32_t U = 8;  // candidates per thread with loads in flight
-    for (uint32_t b = 0; b < wtotal; b += NT * U) {
-      float fv[U];
-      uint32_t iv[U];
-#pragma unroll
-      for (uint32_t u = 0; u < U; ++u) {
-        const uint32_t v = b + u * NT + tid;
-        fv[u] = 0.f;
-        iv[u] = 0;
-        if (v < wtotal) {
-          uint32_t lo = 0, hi = nw - 1;
-          while (lo < hi) {
-            const uint32_t mid = (lo + hi + 1) >> 1;
-            if (sh.tpre[mid] <= v) lo = mid; else hi = mid - 1;
-          }
-          const uint64_t slot = cbase + (uint64_t)(ta + lo - ld.tile_begin) * cap + (v - sh.tpre[lo]);
-          fv[u] = __ldg(dp.cand_val + slot);
-          iv[u] = __ldg(dp.cand_idx + slot) - tile_start(ld, ta + lo);
-        }
-      }
-#pragma unroll
-      for (uint32_t u = 0; u < U; ++u) {
-        const uint32_t v = b + u * NT + tid;
-        if (v < wtotal) {
-          stage_val[v] = fv[u];
-          stage_off[v] = (uint16_t)iv[u];
-        }
-      }
+    staged = my_pad <= stage_cap;  // block-uniform
+    if (tid == 0) {
+      sh.tpre[nw] = my_pad;
+      mbar_init(&stage_bar, 1);
+      mbar_init_fence();
+      if (staged) mbar_arrive_expect_tx(&stage_bar, my_pad * 8u);  // before any copy
     }
     __syncthreads();
+    if (staged) {
+      for (uint32_t q = tid; q < nw; q += NT) {
+        const uint32_t n = sh.tpre[q + 1] - sh.tpre[q];
+        if (n == 0) continue;
+        const uint64_t slot = cbase + (uint64_t)(ta + q - ld.tile_begin) * cap;
+        bulk_load(stage_val + sh.tpre[q], dp.cand_val + slot, n * 4u, &stage_bar);
+        bulk_load(stage_idx + sh.tpre[q], dp.cand_idx + slot, n * 4u, &stage_bar);
+      }
+      const bool ok = mbar_wait_bounded(&stage_bar, 0, kSelectSpinLimit);
+      if (__syncthreads_or(!ok)) {
+        // the copies did not complete: report, and select from global memory
+        if (tid == 0) atomicOr(dp.status + kStatusFlags, LAGS_FLAG_TIMEOUT);
+        staged = false;
+        stage_timeout = true;
+      } else {
+        for (uint32_t q = tid; q < nw; q += NT) {  // padding: key 0, no index
+          const uint32_t real = __ldg(cnt + ta + q);
+          for (uint32_t j = sh.tpre[q] + real; j < sh.tpre[q + 1]; ++j) {
+            stage_val[j] = 0.0f;
+            stage_idx[j] = 0xFFFFFFFFu;
+          }
+        }
+        __syncthreads();
+      }
+    }
   }
   // (Candidate lists and counts are read through the read-only path: nothing
   // writes them during this kernel, and plain loads would be ordered behind the
@@ -264,13 +265,13 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   // positions [wb, we) and walks them 32 at a time
   constexpr uint32_t NW = NT / 32;
   const uint32_t warp = tid >> 5;
-  const uint32_t wspan = (my + NW - 1) / NW;
-  const uint32_t wb = min(my, warp * wspan), we = min(my, wb + wspan);
+  const uint32_t wspan = (my_pad + NW - 1) / NW;
+  const uint32_t wb = min(my_pad, warp * wspan), we = min(my_pad, wb + wspan);
   const unsigned lanes_below = (1u << lane) - 1u;
 
   auto hist_level = [&](int level, int mshift, uint32_t mval, int dshift, uint32_t dmask) {
     if (staged) {
-      for (uint32_t i = tid; i < my; i += NT) {
+      for (uint32_t i = tid; i < my_pad; i += NT) {
         const uint32_t key = mag_key(stage_val[i]);
         if (mshift >= 32 || (key >> mshift) == mval)
           atomicAdd(&sh.hist[(key >> dshift) & dmask], 1u);
@@ -342,7 +343,7 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
       ca += s > fpfx;
       ct += s == fpfx;
     }
-    // per-CTA counts <= stage_cap < 2^16: pack strict | ties
+    // per-CTA counts <= my_pad <= stage_cap < 2^16: pack strict | ties
     const uint32_t wsum = __reduce_add_sync(kFull, (ca << 16) | ct);
     if (lane == 0) sh.tmp[warp] = wsum;
     __syncthreads();
@@ -396,14 +397,6 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
     // block barrier is needed; the emitted index replaces the staged value
     // (0xFFFFFFFF marks "not emitted") for the residual zeroing below
     uint32_t at = a_run + (warp_ex >> 16), bt = b_run + (warp_ex & 0xFFFFu);
-    uint32_t tl = 0;  // tile (relative to ta) of this lane's current position
-    if (wb < we) {    // start from the tile holding the warp's first position
-      uint32_t hi = tb - ta - 1;
-      while (tl < hi) {
-        const uint32_t mid = (tl + hi + 1) >> 1;
-        if (sh.tpre[mid] <= wb) tl = mid; else hi = mid - 1;
-      }
-    }
     for (uint32_t b0 = wb; b0 < we; b0 += 32) {
       const uint32_t i = b0 + lane;
       const bool valid = i < we;
@@ -414,8 +407,7 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
       const uint32_t sb = at + __popc(mst & lanes_below), tb_ = bt + __popc(mti & lanes_below);
       uint32_t mark = 0xFFFFFFFFu;
       if (st || (ti && tb_ < need)) {
-        while (sh.tpre[tl + 1] <= i) ++tl;
-        const uint32_t idx = tile_start(ld, ta + tl) + stage_off[i];
+        const uint32_t idx = stage_idx[i];
         emit(st ? sb + min(need, tb_) : sb + tb_, idx, val, false);
         mark = idx;
       }
@@ -442,11 +434,13 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
       b_run += tot & 0xFFFFu;
     });
   }
+  if (stage_timeout && tid == 0)  // give copies still in flight a bounded chance to land
+    mbar_wait_bounded(&stage_bar, 0, kSelectSpinLimit);
   C::sync();  // no CTA leaves while another may still read its shared memory
 }
 
 // Dynamic shared memory of a select launch staging `cap` candidates.
-inline size_t stage_smem_bytes(uint32_t cap) { return ((size_t)cap * 6 + 15) / 16 * 16; }
+inline size_t stage_smem_bytes(uint32_t cap) { return (size_t)cap * 8; }
 
 cudaError_t configure_select() {
   const int most = (int)stage_smem_bytes(kSelectStageMax);

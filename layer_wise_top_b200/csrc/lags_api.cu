@@ -162,8 +162,13 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
   // candidate count of one CTA (the sample rank scaled to the layer) plus 512
   auto stage_for = [plan](const std::vector<uint32_t>& list, uint32_t ctas) {
     double most = 0.0;
-    for (uint32_t l : list) most = std::max(most, expected_candidates(plan->layers[l]) / ctas);
-    uint64_t cap = ((uint64_t)std::ceil(1.5 * most + 512.0) + 255) / 256 * 256;
+    for (uint32_t l : list) {
+      const LayerDesc& ld = plan->layers[l];
+      const double tiles = std::ceil((double)(ld.tile_end - ld.tile_begin) / ctas);
+      // staged runs are padded to multiples of 4 entries: up to 3 per tile
+      most = std::max(most, 1.5 * expected_candidates(ld) / ctas + 3.0 * tiles);
+    }
+    uint64_t cap = ((uint64_t)std::ceil(most + 512.0) + 255) / 256 * 256;
     return (uint32_t)std::min<uint64_t>(std::max<uint64_t>(cap, kSelectStageMin), kSelectStageMax);
   };
   // aggregation: a tile of a sparse layer is expected to hold P * k * kTile / d

@@ -36,7 +36,8 @@ constexpr uint32_t kSelectWindow = 2048;  // tiles whose prefix sits in smem at 
 // the expected candidate counts, at most kSelectStageMax); a CTA with more
 // reads them from global memory on every pass instead.
 constexpr uint32_t kSelectStageMin = 1024;
-constexpr uint32_t kSelectStageMax = 22528;
+constexpr uint32_t kSelectStageMax = 20480;  // multiple of 4 (16-byte staged runs)
+constexpr uint32_t kSelectSpinLimit = 1u << 22;  // polls of the staging mbarrier
 
 
 // Radix digits of the magnitude key (bits 30..0 of the fp32 pattern).
