@@ -5,7 +5,12 @@
 // candidates; if the sampled threshold held (at least k_l candidates and no
 // tile overflowed its slots) they work on the candidate lists, otherwise on
 // the full acc of the layer (held in the residual buffer after the fused
-// pass).  Either way the result is the exact top-k of the layer:
+// pass).  Either way the result is the exact top-k of the layer.  CL is 1, 8
+// or (for layers whose candidates need more shared memory than 8 CTAs hold)
+// 16, a non-portable cluster size used only where the occupancy query says it
+// fits.  A CTA whose candidates fit in shared memory stages them there with
+// plain bulk copies (cp.async.bulk, one per tile and array, completing on one
+// mbarrier); every pass below then reads shared memory only.
 //
 //  1. radix select on the magnitude key (bits 30..20, 19..9, 8..0): every CTA
 //     builds a shared-memory histogram of its share (warp-aggregated with
