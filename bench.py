@@ -51,6 +51,12 @@ def parse_args():
     ap.add_argument("--dp", action="store_true",
                     help="data-parallel LAGS: split the job's P workers over the ranks and "
                          "all-gather their pick lists (strong scaling) instead of replicas")
+    ap.add_argument("--layerwise", action="store_true",
+                    help="--dp with layer-wise pipelining: buckets of layers from the merge "
+                         "planner, each sparsified, all-gathered and aggregated on its own")
+    ap.add_argument("--bwd-ps-per-elem", type=float, default=10.0,
+                    help="--layerwise: backward time per gradient element (picoseconds) "
+                         "the merge planner assumes")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -223,6 +229,10 @@ def run_ours(args):
     w = WORKLOADS[args.config]
     P, N = w.P, w.N
     dp = None
+    lw = None
+    buckets = None
+    if args.layerwise:
+        args.dp = True
     if args.dp:
         # the job's P workers split over the ranks; every step all-gathers the
         # pick lists and aggregates all P workers on every rank
@@ -233,12 +243,28 @@ def run_ours(args):
                                     timeout=datetime.timedelta(seconds=300))
         if P % world:
             raise SystemExit(f"--dp needs the {P} workers to divide over {world} ranks")
-        from layer_wise_top_b200.dist import DataParallelLags
-        dp = DataParallelLags.create(w.sizes, w.densities, P // world, dev)
+        from layer_wise_top_b200.dist import DataParallelLags, LayerwiseLags
+        if args.layerwise:
+            # message model: NVLink all-gather of 8 B per pick per worker,
+            # 20 us start-up, the measured 770 GB/s peer bandwidth
+            import layer_wise_top_b200 as lags
+            h = lags.lags_plan_create(w.sizes, w.densities, 1)
+            ks = [lags.lags_plan_layer(h, l)[1] for l in range(w.L)]
+            lags.lags_plan_destroy(h)
+            buckets, _ = lags.lags_merge_layers(
+                [8 * P * k for k in ks], [d * args.bwd_ps_per_elem * 1e-12 for d in w.sizes],
+                2e-5, 1.0 / 770e9)
+            lw = LayerwiseLags.create(w.sizes, w.densities, P // world, buckets, dev)
+            dp = lw
+        else:
+            dp = DataParallelLags.create(w.sizes, w.densities, P // world, dev)
         P = P // world  # workers held by this rank
-        plan = dp.local
+        plan = dp.local[0] if lw is not None else dp.local
     else:
         plan = Plan(w.sizes, w.densities, P, device=dev)
+    # plans whose fused pass is timed and whose status words are read
+    local_plans = lw.local if lw is not None else [plan]
+    status_plans = local_plans + (lw.total if lw is not None else [])
     step_bytes = P * N * 4
     pool = max(1, min(args.warmup + args.steps, POOL_BUDGET_BYTES // step_bytes))
     grads = []
@@ -248,13 +274,16 @@ def run_ours(args):
             synth.worker_grads_device(w, p, s + 1000 * rank, bufs[p])
         grads.append(bufs)
     res = [torch.zeros(N, dtype=torch.float32, device=dev) for _ in range(P)]
-    idx, val = plan.empty_picks()
+    idx, val = plan.empty_picks() if lw is None else (None, None)
     dense = torch.empty(N, dtype=torch.float32, device=dev)
     weights = torch.zeros(N, dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
 
-    n_sparsify, n_aggregate, _ = plan.kernel_launches()
-    launches_per_step = n_sparsify + n_aggregate  # (the all-gather in --dp is NCCL's)
+    launches_per_step = 0  # (the all-gather in --dp is NCCL's)
+    for pl in local_plans:
+        launches_per_step += pl.kernel_launches()[0]
+    for pl in (lw.total if lw is not None else [plan]):
+        launches_per_step += pl.kernel_launches()[1]
 
     def step(i):
         if dp is not None:
@@ -263,14 +292,21 @@ def run_ours(args):
         plan.sparsify(grads[i % pool], res, w.lr, idx, val)
         plan.aggregate_apply(idx, val, dense, weights)
 
+    def poll_all():
+        f, fb = 0, 0
+        for pl in status_plans:
+            a, b = pl.poll()
+            f, fb = f | a, fb + b
+        return f, fb
+
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
-    flags, fallbacks = plan.poll()
+    flags, fallbacks = poll_all()
 
     K = args.steps
-    ev_k1 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(K)]
+    ev_k1 = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in local_plans] for _ in range(K)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
@@ -280,16 +316,19 @@ def run_ours(args):
     time.sleep(0.3)
     t0.record()
     for i in range(K):
-        plan.set_events(*ev_k1[i])
+        for pl, evs in zip(local_plans, ev_k1[i]):
+            pl.set_events(*evs)
         step(args.warmup + i)
     t1.record()
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    plan.set_events(None, None)
+    for pl in local_plans:
+        pl.set_events(None, None)
     ms = t0.elapsed_time(t1)
-    k1_ms = [a.elapsed_time(b) for a, b in ev_k1]
-    flags2, fallbacks2 = plan.poll()
+    # fused-pass time per step, summed over the buckets of a layer-wise step
+    k1_ms = [sum(a.elapsed_time(b) for a, b in evs) for evs in ev_k1]
+    flags2, fallbacks2 = poll_all()
     ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
@@ -330,8 +369,10 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
 
-    if world > 1 or dp is not None:
+    is_dp = dp is not None
+    if world > 1 or is_dp:
         dist.barrier(device_ids=[local])
+        del dp, lw  # their streams and NCCL work go before the process group
         dist.destroy_process_group()
     if rank != 0:
         return 0
@@ -340,21 +381,23 @@ def run_ours(args):
     k1_avg = sum(k1_ms) / len(k1_ms)
     k1_bytes = 12 * P * N
     achieved = k1_bytes / (k1_avg / 1e3) / 1e9
-    job_elems = (P * world if dp is not None else world * P) * N  # all ranks' elements
+    job_elems = world * P * N  # all ranks' elements
     line = {
         "metric": METRIC,
         "value": job_elems * K / (ms_max / 1e3) / 1e9,
         "unit": "Gelem/s",
         "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_max / K,
-        "higher_is_better": True, "scaling": "strong" if dp is not None else "weak",
+        "higher_is_better": True, "scaling": "strong" if is_dp else "weak",
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic: Philox4x32-10 gradients with the workload's tensor shapes",
         "config": workload_config(
             w, parallelism=(f"data-parallel: {P} workers per rank x {world} ranks, NCCL "
-                            f"all-gather of pick lists" if dp is not None else
-                            f"replicas x{world}"), grad_pool_steps=pool,
+                            f"all-gather of pick lists" if is_dp else f"replicas x{world}")
+            + (f", layer-wise: {len(buckets)} buckets of layers (merge planner, backward "
+               f"{args.bwd_ps_per_elem} ps/element, 20 us + 8 B/pick at 770 GB/s per message)"
+               if buckets else ""), grad_pool_steps=pool,
             l2=f"inputs larger than L2: {12 * P * N / 1e9:.2f} GB streamed per step vs "
                f"{L2_BYTES / 1e6:.0f} MB L2",
             step="lags_sparsify + lags_aggregate_apply (aggregate and apply fused)"),

@@ -89,6 +89,31 @@ typedef enum {
 LAGS_API lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities,
                              int32_t num_layers, int32_t num_workers, lags_plan** out_plan);
 
+/*
+ * lags_plan_create_range - a plan for layers [layer_begin, layer_end) of the
+ * model that layer_sizes/densities describe (all num_layers of them), for
+ * layer-wise pipelining: LAGS ("Layer-wise Adaptive Gradient Sparsification
+ * ..." review, "proposed method") sparsifies and sends each layer as soon as
+ * the backward pass has produced it, instead of after the whole pass.
+ *   - Element indices stay those of the whole model: grads, residuals,
+ *     dense_out and weights are the whole model's buffers and the emitted
+ *     indices are global.  Calls on the plan read and write only the range's
+ *     elements [offset of layer_begin, N) and its own pick lists.
+ *   - The plan's layers are numbered from 0 (= model layer layer_begin) in
+ *     lags_plan_layer; its pick lists are [P][K] with K the range's picks.
+ *   - lags_plan_info reports N = one past the range's last element (buffers
+ *     must hold at least N elements) and that K.
+ *   - Each layer is selected, aggregated and applied exactly as by a plan of
+ *     the whole model, so the plans of a partition of the layers together
+ *     give bit for bit the results of one whole-model plan.
+ * Other arguments and errors as lags_plan_create; also LAGS_ERR_INVALID_ARG
+ * unless 0 <= layer_begin < layer_end <= num_layers.
+ */
+LAGS_API lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* densities,
+                                            int32_t num_layers, int32_t num_workers,
+                                            int32_t layer_begin, int32_t layer_end,
+                                            lags_plan** out_plan);
+
 /* Frees the host tables.  The workspace stays the caller's. */
 LAGS_API lags_status lags_plan_destroy(lags_plan* plan);
 
@@ -162,7 +187,8 @@ LAGS_API lags_status lags_aggregate_apply(lags_plan* plan, const uint32_t* idx, 
                                           float* dense_out, float* weights, void* stream);
 
 /*
- * lags_apply - weights <- weights - dense_out over the plan's N elements.
+ * lags_apply - weights <- weights - dense_out over the plan's elements
+ * (0 .. N-1, or the range of a lags_plan_create_range plan).
  *   weights    device float[N], 16-byte aligned, updated in place.
  *   dense_out  device float[N], 16-byte aligned.
  */
@@ -237,6 +263,35 @@ LAGS_API lags_status lags_adaptive_densities(const int64_t* layer_sizes,
                                              const double* backward_seconds, int32_t num_layers,
                                              double alpha, double beta, double rho_min,
                                              double* out_densities);
+
+/*
+ * lags_merge_layers - cut the layers into buckets of consecutive layers, one
+ * message per bucket, so that the last message ends as early as possible
+ * (merged-gradient wait-free backpropagation, "MG-WFBP: Efficient Data
+ * Communication for Distributed Synchronous SGD Algorithms" review, "proposed
+ * method": small per-layer messages are merged to save start-up costs, the
+ * merge is optimal for the iteration time, found by dynamic programming in
+ * O(L^2) once before training).  Host only, no device.
+ *   message_bytes     host, [num_layers] bytes >= 0 each layer sends (for
+ *                     LAGS: 8 * k_l * workers per rank).
+ *   backward_seconds  host, [num_layers] t_l >= 0: backward time of each layer.
+ *   alpha, beta       message model: B bytes in one message take
+ *                     alpha + beta * B seconds (alpha, beta >= 0).
+ *   out_bucket_first  host, [num_layers]: receives the first layer of every
+ *                     bucket, ascending; bucket b is layers
+ *                     [first[b], first[b+1]) (the last ends at num_layers).
+ *   out_num_buckets   host, receives the bucket count.
+ *   out_end_seconds   host, receives the end of the last message (may be NULL).
+ * Model: backward produces layers L-1 .. 0; layer l exists at
+ * R_l = sum_{j >= l} t_j; a bucket's message starts once its first layer is
+ * produced and the previous message has ended; messages go out in production
+ * order.  Among cuts with the same end time the planner prefers longer
+ * buckets, starting from the last layers.
+ */
+LAGS_API lags_status lags_merge_layers(const int64_t* message_bytes,
+                                       const double* backward_seconds, int32_t num_layers,
+                                       double alpha, double beta, int32_t* out_bucket_first,
+                                       int32_t* out_num_buckets, double* out_end_seconds);
 
 /*
  * lags_plan_kernel_launches - how many kernels one lags_sparsify, one

@@ -10,8 +10,9 @@ from ._binding import (  # noqa: F401
     LAGS_ERR_UNSUPPORTED_DEVICE, LAGS_ERR_WORKSPACE, LAGS_FLAG_BAD_PICKS, LAGS_MAX_WORKERS,
     LAGS_OK, LIB_PATH, LagsError, lags_aggregate, lags_aggregate_apply, lags_apply,
     lags_adaptive_densities, lags_error_string, lags_plan_kernel_launches,
-    lags_plan_create, lags_plan_destroy, lags_plan_info, lags_plan_layer,
-    lags_plan_set_events, lags_plan_set_workspace, lags_sparsify, lags_sparsify_static, lags_status_poll, library,
+    lags_merge_layers, lags_plan_create, lags_plan_create_range, lags_plan_destroy,
+    lags_plan_info, lags_plan_layer, lags_plan_set_events, lags_plan_set_workspace,
+    lags_sparsify, lags_sparsify_static, lags_status_poll, library,
 )
 
 

@@ -26,7 +26,7 @@ EXPORTED = ("lags_plan_create", "lags_plan_destroy", "lags_plan_info", "lags_pla
             "lags_plan_set_workspace", "lags_sparsify", "lags_aggregate", "lags_apply",
             "lags_status_poll", "lags_plan_set_events", "lags_sparsify_static",
             "lags_aggregate_apply", "lags_plan_kernel_launches", "lags_adaptive_densities",
-            "lags_error_string")
+            "lags_plan_create_range", "lags_merge_layers", "lags_error_string")
 
 
 class LagsError(RuntimeError):
@@ -45,6 +45,8 @@ def _load() -> ctypes.CDLL:
     st = ctypes.c_int
     lib.lags_plan_create.argtypes = [i64p, ctypes.POINTER(ctypes.c_double), i32, i32,
                                      ctypes.POINTER(vp)]
+    lib.lags_plan_create_range.argtypes = [i64p, ctypes.POINTER(ctypes.c_double), i32, i32,
+                                           i32, i32, ctypes.POINTER(vp)]
     lib.lags_plan_destroy.argtypes = [vp]
     lib.lags_plan_info.argtypes = [vp, i64p, i64p, ctypes.POINTER(ctypes.c_size_t)]
     lib.lags_plan_layer.argtypes = [vp, i32, i64p, i64p, i64p]
@@ -59,6 +61,8 @@ def _load() -> ctypes.CDLL:
     dp_ = ctypes.POINTER(ctypes.c_double)
     lib.lags_adaptive_densities.argtypes = [i64p, dp_, i32, ctypes.c_double, ctypes.c_double,
                                             ctypes.c_double, dp_]
+    lib.lags_merge_layers.argtypes = [i64p, dp_, i32, ctypes.c_double, ctypes.c_double, i32p,
+                                      i32p, dp_]
     lib.lags_status_poll.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32),
                                      ctypes.POINTER(ctypes.c_uint32), vp]
     lib.lags_plan_set_events.argtypes = [vp, vp, vp]
@@ -97,6 +101,20 @@ def lags_plan_create(layer_sizes: Sequence[int], densities: Sequence[float],
     out = ctypes.c_void_p()
     _check(_LIB.lags_plan_create(sizes, dens, L, int(num_workers), ctypes.byref(out)),
            "lags_plan_create")
+    return out
+
+
+def lags_plan_create_range(layer_sizes: Sequence[int], densities: Sequence[float],
+                           num_workers: int, layer_begin: int, layer_end: int) -> ctypes.c_void_p:
+    L = len(layer_sizes)
+    if len(densities) != L:
+        raise ValueError("layer_sizes and densities differ in length")
+    sizes = (ctypes.c_int64 * max(L, 1))(*[int(x) for x in layer_sizes])
+    dens = (ctypes.c_double * max(L, 1))(*[float(x) for x in densities])
+    out = ctypes.c_void_p()
+    _check(_LIB.lags_plan_create_range(sizes, dens, L, int(num_workers), int(layer_begin),
+                                       int(layer_end), ctypes.byref(out)),
+           "lags_plan_create_range")
     return out
 
 
@@ -178,6 +196,24 @@ def lags_adaptive_densities(layer_sizes: Sequence[int], backward_seconds: Sequen
     _check(_LIB.lags_adaptive_densities(sizes, t, L, float(alpha), float(beta), float(rho_min),
                                         out), "lags_adaptive_densities")
     return [out[i] for i in range(L)]
+
+
+def lags_merge_layers(message_bytes: Sequence[int], backward_seconds: Sequence[float],
+                      alpha: float, beta: float) -> Tuple[list, float]:
+    """Buckets of consecutive layers, one message each, whose last message
+    ends earliest (see include/lags.h for the model).  Returns the list of
+    (first layer, end layer) pairs in forward order and that end time."""
+    L = len(message_bytes)
+    if len(backward_seconds) != L:
+        raise ValueError("message_bytes and backward_seconds differ in length")
+    b = (ctypes.c_int64 * max(L, 1))(*[int(x) for x in message_bytes])
+    t = (ctypes.c_double * max(L, 1))(*[float(x) for x in backward_seconds])
+    first = (ctypes.c_int32 * max(L, 1))()
+    nb, end = ctypes.c_int32(), ctypes.c_double()
+    _check(_LIB.lags_merge_layers(b, t, L, float(alpha), float(beta), first, ctypes.byref(nb),
+                                  ctypes.byref(end)), "lags_merge_layers")
+    f = [first[i] for i in range(nb.value)] + [L]
+    return [(f[i], f[i + 1]) for i in range(nb.value)], end.value
 
 
 def lags_apply(plan, weights: int, dense_out: int, stream: int = 0) -> None:

@@ -325,15 +325,20 @@ __global__ void __launch_bounds__(kAggThreads, 4)
   }
 }
 
-__global__ void __launch_bounds__(256) k_apply(uint32_t N, float* __restrict__ w,
+__global__ void __launch_bounds__(256) k_apply(uint32_t first, uint32_t end,
+                                               float* __restrict__ w,
                                                const float* __restrict__ dense) {
+  // elements [first, end): a scalar head up to the first 16-byte boundary,
+  // float4 over the aligned middle, a scalar tail
   pdl_trigger();
   pdl_wait();
-  const uint32_t n4 = N / 4;
+  const uint32_t a0 = min(end, (first + 3u) & ~3u);
+  const uint32_t n4 = (end - a0) / 4;
+  const uint32_t gid = blockIdx.x * blockDim.x + threadIdx.x;
   const uint32_t stride = gridDim.x * blockDim.x;
-  float4* w4 = reinterpret_cast<float4*>(w);
-  const float4* d4 = reinterpret_cast<const float4*>(dense);
-  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+  float4* w4 = reinterpret_cast<float4*>(w + a0);
+  const float4* d4 = reinterpret_cast<const float4*>(dense + a0);
+  for (uint32_t i = gid; i < n4; i += stride) {
     float4 a = w4[i];
     const float4 b = __ldcs(d4 + i);
     a.x = __fsub_rn(a.x, b.x);
@@ -342,8 +347,9 @@ __global__ void __launch_bounds__(256) k_apply(uint32_t N, float* __restrict__ w
     a.w = __fsub_rn(a.w, b.w);
     w4[i] = a;
   }
-  const uint32_t tail = n4 * 4 + blockIdx.x * blockDim.x + threadIdx.x;
-  if (tail < N) w[tail] = __fsub_rn(w[tail], dense[tail]);
+  if (gid < a0 - first) w[first + gid] = __fsub_rn(w[first + gid], dense[first + gid]);
+  const uint32_t tail = a0 + n4 * 4 + gid;
+  if (tail < end) w[tail] = __fsub_rn(w[tail], dense[tail]);
 }
 
 cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStream_t s) {
@@ -364,11 +370,12 @@ cudaError_t launch_aggregate(const DevPlan& dp, const uint32_t* idx, const float
                     dense, weights, dp.agg_tile_acc != 0);
 }
 
-cudaError_t launch_apply(uint32_t N, float* w, const float* dense, cudaStream_t s) {
-  uint32_t blocks = (N / 4 + 255) / 256;
+cudaError_t launch_apply(uint32_t first, uint32_t end, float* w, const float* dense,
+                         cudaStream_t s) {
+  uint32_t blocks = ((end - first) / 4 + 255) / 256;
   if (blocks > 148u * 16u) blocks = 148u * 16u;
   if (blocks == 0) blocks = 1;
-  return launch_pdl(k_apply, dim3(blocks), dim3(256), 0, s, 1, N, w, dense);
+  return launch_pdl(k_apply, dim3(blocks), dim3(256), 0, s, 1, first, end, w, dense);
 }
 
 }  // namespace lags

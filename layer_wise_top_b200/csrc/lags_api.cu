@@ -94,19 +94,35 @@ extern "C" {
 
 lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities,
                              int32_t num_layers, int32_t num_workers, lags_plan** out_plan) {
+  return lags_plan_create_range(layer_sizes, densities, num_layers, num_workers, 0, num_layers,
+                                out_plan);
+}
+
+lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* densities,
+                                   int32_t num_layers, int32_t num_workers, int32_t layer_begin,
+                                   int32_t layer_end, lags_plan** out_plan) {
   if (!out_plan) return LAGS_ERR_INVALID_ARG;
   *out_plan = nullptr;
   if (!layer_sizes || !densities || num_layers < 1 || num_layers > (1 << 24) ||
-      num_workers < 1 || num_workers > LAGS_MAX_WORKERS)
+      num_workers < 1 || num_workers > LAGS_MAX_WORKERS || layer_begin < 0 ||
+      layer_end <= layer_begin || layer_end > num_layers)
     return LAGS_ERR_INVALID_ARG;
+  // element offsets are those of the whole model: skip the layers before the range
+  uint64_t off = 0;
+  for (int32_t l = 0; l < layer_begin; ++l) {
+    if (layer_sizes[l] <= 0) return LAGS_ERR_INVALID_ARG;
+    off += (uint64_t)layer_sizes[l];
+    if (off >= (1ull << 32)) return LAGS_ERR_INVALID_ARG;
+  }
   lags_plan* plan = new (std::nothrow) lags_plan();
   if (!plan) return LAGS_ERR_INVALID_ARG;
-  plan->L = num_layers;
+  plan->L = layer_end - layer_begin;
   plan->P = num_workers;
-  uint64_t off = 0, koff = 0, slots = 0;
-  for (int32_t l = 0; l < num_layers; ++l) {
-    const int64_t d = layer_sizes[l];
-    const double rho = densities[l];
+  plan->N0 = off;
+  uint64_t koff = 0, slots = 0;
+  for (int32_t l = 0; l < plan->L; ++l) {
+    const int64_t d = layer_sizes[layer_begin + l];
+    const double rho = densities[layer_begin + l];
     if (d <= 0 || !(rho > 0.0) || !(rho <= 1.0)) {
       delete plan;
       return LAGS_ERR_INVALID_ARG;
@@ -220,7 +236,7 @@ lags_status lags_plan_create(const int64_t* layer_sizes, const double* densities
   plan->o_small = section(cur, (plan->sel_small.size() + 1) * 4);
   plan->o_huge = section(cur, (plan->sel_huge.size() + 1) * 4);
   plan->o_sparse = section(cur, (plan->sparse.size() + 1) * 4);
-  plan->o_lo = section(cur, P * (uint64_t)num_layers * 4);
+  plan->o_lo = section(cur, P * (uint64_t)plan->L * 4);
   plan->o_cnt = section(cur, P * T * 4);
   plan->o_cval = section(cur, P * (plan->C + 1) * 4);
   plan->o_cidx = section(cur, P * (plan->C + 1) * 4);
@@ -370,6 +386,47 @@ lags_status lags_adaptive_densities(const int64_t* layer_sizes, const double* ba
   return LAGS_OK;
 }
 
+lags_status lags_merge_layers(const int64_t* message_bytes, const double* backward_seconds,
+                              int32_t num_layers, double alpha, double beta,
+                              int32_t* out_bucket_first, int32_t* out_num_buckets,
+                              double* out_end_seconds) {
+  if (!message_bytes || !backward_seconds || !out_bucket_first || !out_num_buckets ||
+      num_layers < 1 || num_layers > (1 << 20) || !(alpha >= 0.0) || !(beta >= 0.0))
+    return LAGS_ERR_INVALID_ARG;
+  const int32_t L = num_layers;
+  // ready[l]: the backward pass has produced layers L-1 .. l (it runs downwards)
+  std::vector<double> ready(L + 1, 0.0);
+  for (int32_t l = L - 1; l >= 0; --l) {
+    if (message_bytes[l] < 0 || !(backward_seconds[l] >= 0.0)) return LAGS_ERR_INVALID_ARG;
+    ready[l] = ready[l + 1] + backward_seconds[l];
+  }
+  // best[i]: earliest time at which messages covering layers [i, L) can have
+  // been sent, over all ways of cutting them into buckets of consecutive
+  // layers; a bucket [i, j) is one message of alpha + beta * bytes that starts
+  // once layer i is produced and the previous message (layers [j, L)) is done.
+  // Since that start time only grows with the previous end time, the best cut
+  // of [i, L) extends a best cut of some [j, L): best[i] = min over j, O(L^2)
+  // in all.  Equal end times go to the longer bucket.
+  std::vector<double> best(L + 1, 0.0);
+  std::vector<int32_t> next(L + 1, L);
+  for (int32_t i = L - 1; i >= 0; --i) {
+    double bytes = 0.0;
+    for (int32_t j = i + 1; j <= L; ++j) {
+      bytes += (double)message_bytes[j - 1];
+      const double end = std::max(ready[i], best[j]) + alpha + beta * bytes;
+      if (j == i + 1 || end <= best[i]) {
+        best[i] = end;
+        next[i] = j;
+      }
+    }
+  }
+  int32_t nb = 0;
+  for (int32_t i = 0; i < L; i = next[i]) out_bucket_first[nb++] = i;
+  *out_num_buckets = nb;
+  if (out_end_seconds) *out_end_seconds = best[0];
+  return LAGS_OK;
+}
+
 lags_status lags_plan_kernel_launches(const lags_plan* plan, int32_t* sparsify,
                                       int32_t* aggregate, int32_t* apply) {
   if (!plan) return LAGS_ERR_INVALID_ARG;
@@ -386,7 +443,8 @@ lags_status lags_apply(const lags_plan* plan, float* weights, const float* dense
                        void* stream) {
   if (!plan || !weights || !dense_out) return LAGS_ERR_INVALID_ARG;
   if (!aligned(weights, 16) || !aligned(dense_out, 16)) return LAGS_ERR_ALIGNMENT;
-  return cuda_status(launch_apply((uint32_t)plan->N, weights, dense_out, (cudaStream_t)stream));
+  return cuda_status(launch_apply((uint32_t)plan->N0, (uint32_t)plan->N, weights, dense_out,
+                                  (cudaStream_t)stream));
 }
 
 lags_status lags_plan_set_events(lags_plan* plan, void* before, void* after) {

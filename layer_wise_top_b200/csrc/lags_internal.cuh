@@ -114,7 +114,7 @@ cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out
 cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStream_t s);
 cudaError_t launch_aggregate(const DevPlan& dp, const uint32_t* idx, const float* val,
                              float* dense, float* weights, cudaStream_t s);
-cudaError_t launch_apply(uint32_t N, float* w, const float* dense, cudaStream_t s);
+cudaError_t launch_apply(uint32_t first, uint32_t end, float* w, const float* dense, cudaStream_t s);
 
 // The fused error-feedback pass used by lags_sparsify.
 inline cudaError_t launch_ef(const DevPlan& dp, const WorkerPtrs& wp, float lr, uint32_t* out_idx,

@@ -11,7 +11,7 @@
 
 struct lags_plan {
   int32_t L = 0, P = 0;
-  uint64_t N = 0, K = 0, C = 0;
+  uint64_t N0 = 0, N = 0, K = 0, C = 0;  // elements [N0, N) of the model; K picks per worker
   std::vector<lags::LayerDesc> layers;
   std::vector<lags::TileDesc> tiles;
   std::vector<uint32_t> sel_large, sel_small, sel_huge, sparse;

@@ -23,7 +23,7 @@ on CPU ranks.
 """
 from __future__ import annotations
 
-from typing import List, Optional, Sequence
+from typing import List, Optional, Sequence, Tuple
 
 import torch
 import torch.distributed as dist
@@ -73,3 +73,109 @@ class DataParallelLags:
         self.local.sparsify(grads, residuals, lr, self.idx_local, self.val_local)
         self.exchange()
         self.total.aggregate_apply(self.idx_all, self.val_all, dense_out, weights)
+
+
+class LayerwiseLags:
+    """LAGS-SGD step with layer-wise pipelining.
+
+    The layers are cut into buckets of consecutive layers (for instance by
+    ``lags_merge_layers``).  The backward pass produces the last layers first,
+    so the buckets are processed from the last to the first, each as soon as
+    its gradients exist (``ready[b]``, an event the caller records after
+    producing bucket b): sparsify the bucket on the current stream, start the
+    all-gather of its pick lists without waiting, and aggregate + apply it on
+    a second stream once the gather has landed.  The next bucket's
+    sparsification therefore overlaps the previous bucket's exchange, and all
+    of it overlaps the rest of the backward pass ("Layer-wise Adaptive
+    Gradient Sparsification ..." review, "proposed method": layer-wise
+    selection lets communication start before back-propagation ends).
+
+    Every layer is selected and aggregated exactly as by one whole-model plan,
+    so the results equal ``DataParallelLags.step`` bit for bit, whatever the
+    buckets.
+    """
+
+    def __init__(self, local_plans, total_plans, buckets, workers_per_rank: int,
+                 device: torch.device, group: Optional[dist.ProcessGroup] = None):
+        if len(local_plans) != len(buckets) or len(total_plans) != len(buckets):
+            raise ValueError("one local and one total plan per bucket")
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.device = torch.device(device)
+        self.buckets = [(int(a), int(b)) for a, b in buckets]
+        self.local = list(local_plans)
+        self.total = list(total_plans)
+        self.P_local = int(workers_per_rank)
+        self.P_total = self.P_local * self.world
+        self.idx_local, self.val_local, self.idx_all, self.val_all = [], [], [], []
+        for plan in self.local:
+            n = self.P_local * plan.K
+            self.idx_local.append(torch.empty(n, dtype=torch.int32, device=device))
+            self.val_local.append(torch.empty(n, dtype=torch.float32, device=device))
+            self.idx_all.append(torch.empty(n * self.world, dtype=torch.int32, device=device))
+            self.val_all.append(torch.empty(n * self.world, dtype=torch.float32, device=device))
+        self.agg_stream = (torch.cuda.Stream(device=self.device)
+                           if self.device.type == "cuda" else None)
+
+    @classmethod
+    def create(cls, layer_sizes: Sequence[int], densities: Sequence[float],
+               workers_per_rank: int, buckets: Sequence[Tuple[int, int]],
+               device: torch.device,
+               group: Optional[dist.ProcessGroup] = None) -> "LayerwiseLags":
+        """Range plans on `device`, one pair per bucket of layers."""
+        from .plan import Plan
+        world = dist.get_world_size(group)
+        check_buckets(buckets, len(layer_sizes))
+        local = [Plan(layer_sizes, densities, workers_per_rank, device=device, layer_range=b)
+                 for b in buckets]
+        total = [Plan(layer_sizes, densities, workers_per_rank * world, device=device,
+                      layer_range=b) for b in buckets]
+        return cls(local, total, buckets, workers_per_rank, device, group)
+
+    def step(self, grads: List[torch.Tensor], residuals: List[torch.Tensor], lr: float,
+             dense_out: torch.Tensor, weights: torch.Tensor, ready=None) -> None:
+        """grads/residuals: this rank's `workers_per_rank` whole-model buffers.
+        ready: None, or one CUDA event per bucket (forward order) after which
+        that bucket's gradients are complete."""
+        if len(grads) != self.P_local or len(residuals) != self.P_local:
+            raise ValueError(f"need {self.P_local} gradient and residual buffers per rank")
+        if ready is not None and len(ready) != len(self.buckets):
+            raise ValueError("one ready event per bucket")
+        cuda = self.agg_stream is not None
+        main = torch.cuda.current_stream(self.device) if cuda else None
+        if cuda:
+            self.agg_stream.wait_stream(main)  # dense/weights written before this step
+        for b in reversed(range(len(self.buckets))):
+            if ready is not None and ready[b] is not None:
+                main.wait_event(ready[b])
+            self.local[b].sparsify(grads, residuals, lr, self.idx_local[b], self.val_local[b])
+            works = [dist.all_gather_into_tensor(self.idx_all[b], self.idx_local[b],
+                                                 group=self.group, async_op=True),
+                     dist.all_gather_into_tensor(self.val_all[b], self.val_local[b],
+                                                 group=self.group, async_op=True)]
+            if cuda:
+                with torch.cuda.stream(self.agg_stream):
+                    for w in works:
+                        w.wait()  # the aggregation stream waits; the host does not
+                    self.total[b].aggregate_apply(self.idx_all[b], self.val_all[b],
+                                                  dense_out, weights)
+            else:
+                for w in works:
+                    w.wait()
+                self.total[b].aggregate_apply(self.idx_all[b], self.val_all[b], dense_out,
+                                              weights)
+        if cuda:
+            # the next step reuses the pick buffers and reads dense/weights
+            main.wait_stream(self.agg_stream)
+
+
+def check_buckets(buckets: Sequence[Tuple[int, int]], num_layers: int) -> None:
+    """Buckets must cover layers 0..num_layers-1 in order, without gaps."""
+    at = 0
+    for a, b in buckets:
+        if a != at or b <= a:
+            raise ValueError(f"buckets must partition the layers in order, got {list(buckets)}")
+        at = b
+    if at != num_layers:
+        raise ValueError(f"buckets cover {at} of {num_layers} layers")

@@ -3,7 +3,7 @@ and the benchmark use.  It only checks tensors and passes their pointers and
 the current CUDA stream to the C entry points."""
 from __future__ import annotations
 
-from typing import List, Optional, Sequence
+from typing import List, Optional, Sequence, Tuple
 
 import torch
 
@@ -25,17 +25,30 @@ def _need(t: torch.Tensor, dtype, numel: int, what: str) -> None:
 
 
 class Plan:
-    """Layer table of one flattened gradient buffer shared by P workers."""
+    """Layer table of one flattened gradient buffer shared by P workers.
+
+    With `layer_range=(begin, end)` the plan covers only model layers
+    [begin, end): buffers stay the whole model's (N is one past the range's
+    last element), indices stay global, and the pick lists hold only the
+    range's K picks per worker."""
 
     def __init__(self, layer_sizes: Sequence[int], densities: Sequence[float], P: int,
-                 device: Optional[torch.device] = None):
+                 device: Optional[torch.device] = None,
+                 layer_range: Optional[Tuple[int, int]] = None):
         self.device = torch.device(device if device is not None else "cuda")
-        self.handle = B.lags_plan_create(layer_sizes, densities, P)
+        if layer_range is None:
+            lb, le = 0, len(layer_sizes)
+            self.handle = B.lags_plan_create(layer_sizes, densities, P)
+        else:
+            lb, le = int(layer_range[0]), int(layer_range[1])
+            self.handle = B.lags_plan_create_range(layer_sizes, densities, P, lb, le)
+        self.layer_range = (lb, le)
         self.P = int(P)
-        self.L = len(layer_sizes)
+        self.L = le - lb
         self.N, self.K, self.workspace_bytes = B.lags_plan_info(self.handle)
         self.layers = [B.lags_plan_layer(self.handle, l) for l in range(self.L)]
-        self.sizes = [int(x) for x in layer_sizes]
+        self.sizes = [int(x) for x in layer_sizes[lb:le]]
+        self.first = self.layers[0][0]  # first element of the plan's layers
         with torch.cuda.device(self.device):
             self.workspace = torch.empty(max(self.workspace_bytes, 256), dtype=torch.uint8,
                                          device=self.device)

@@ -7,5 +7,6 @@ fallback.
 """
 from .lags_oracle import (  # noqa: F401
     adaptive_densities, aggregate, aggregate_layer, apply_update, error_feedback, k_of, layer_plan,
-    magnitude_order, run_workload, select_layer, sparsify, sparsify_layer,
+    magnitude_order, merge_layers, message_schedule_end, run_workload, select_layer, sparsify,
+    sparsify_layer,
 )

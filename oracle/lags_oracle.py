@@ -35,6 +35,16 @@ and in the design notes:
       layers >= l) and the previous message has ended, takes alpha + 8 beta k
       seconds, and gets the largest density whose message ends by the end of
       the backward pass (rho_min if none does).
+  R9  merged messages ("MG-WFBP: Efficient Data Communication for Distributed
+      Synchronous SGD Algorithms" review, "proposed method": merge small
+      per-layer messages to save start-up costs, choosing the merge that
+      minimises the iteration time, by dynamic programming in O(L^2), once
+      before training): the layers are cut into buckets of consecutive layers,
+      one message per bucket; with the timing of R8 (a message of B bytes
+      takes alpha + beta B and starts once its bucket's first layer, the last
+      one backprop produces, exists and the previous message has ended) the
+      cut minimises the end of the last message.  Equal end times go to the
+      longer bucket, deciding from the last layers towards the first.
 """
 from __future__ import annotations
 
@@ -179,6 +189,50 @@ def adaptive_densities(sizes: Sequence[int], backward_seconds: Sequence[float], 
         out[l] = rho
         link_free = start + alpha + beta * 8.0 * k_of(int(sizes[l]), rho)
     return out
+
+
+def message_schedule_end(buckets: Sequence[Tuple[int, int]], message_bytes: Sequence[int],
+                         backward_seconds: Sequence[float], alpha: float,
+                         beta: float) -> float:
+    """End of the last message when the layers are sent as `buckets` (reading
+    R9's timing): buckets go out from the last layers to the first."""
+    L = len(message_bytes)
+    ready = [0.0] * (L + 1)  # ready[l]: layers L-1 .. l have been produced
+    for l in range(L - 1, -1, -1):
+        ready[l] = ready[l + 1] + float(backward_seconds[l])
+    link_free = 0.0
+    for first, end in sorted(buckets, reverse=True):
+        nbytes = 0.0
+        for l in range(first, end):
+            nbytes += float(message_bytes[l])
+        link_free = max(ready[first], link_free) + alpha + beta * nbytes
+    return link_free
+
+
+def merge_layers(message_bytes: Sequence[int], backward_seconds: Sequence[float], alpha: float,
+                 beta: float) -> Tuple[List[Tuple[int, int]], float]:
+    """Bucket cut of reading R9 by dynamic programming over suffixes: the best
+    cut of layers [i, L) is a first bucket [i, j) after a best cut of [j, L),
+    because a bucket's end only grows with the end of the messages before it.
+    Returns the buckets in forward order and the end of the last message."""
+    L = len(message_bytes)
+    ready = [0.0] * (L + 1)
+    for l in range(L - 1, -1, -1):
+        ready[l] = ready[l + 1] + float(backward_seconds[l])
+    best = [0.0] * (L + 1)  # best[L]: nothing to send
+    cut = [L] * (L + 1)
+    for i in range(L - 1, -1, -1):
+        nbytes = 0.0
+        for j in range(i + 1, L + 1):
+            nbytes += float(message_bytes[j - 1])
+            end = max(ready[i], best[j]) + alpha + beta * nbytes
+            if j == i + 1 or end <= best[i]:  # ties: the longer bucket
+                best[i], cut[i] = end, j
+    buckets, i = [], 0
+    while i < L:
+        buckets.append((i, cut[i]))
+        i = cut[i]
+    return buckets, best[0]
 
 
 def run_workload(sizes: Sequence[int], densities: Sequence[float], P: int, lr: float,

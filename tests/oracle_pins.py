@@ -225,3 +225,33 @@ def check_k_rule(lo, workloads):
         for d, rho in zip(w.sizes, w.densities):
             exact = math.ceil(Fraction(repr(rho)) * d)
             assert lo.k_of(d, rho) == max(1, min(d, exact)), (w.name, d, rho)
+
+
+def check_merge_hand(lo):
+    """Merged-message planner on the hand-worked four-layer fixture (R9)."""
+    from conftest import read_golden
+    g = read_golden("merge_four_layers.txt")
+    b = [int(x) for x in g["bytes"]]
+    t = [float(x) for x in g["backward"]]
+    a, beta = float(g["alpha"][0]), float(g["beta"][0])
+    f = [int(x) for x in g["first"]] + [len(b)]
+    want = [(f[i], f[i + 1]) for i in range(len(f) - 1)]
+    assert lo.message_schedule_end([(l, l + 1) for l in range(len(b))], b, t, a, beta) == \
+        float(g["singles_end"][0])
+    assert lo.merge_layers(b, t, a, beta) == (want, float(g["end"][0]))
+
+
+def check_merge_bruteforce(lo, seed=7):
+    """The planner's cut ends no later than any cut of a small model."""
+    rng = np.random.default_rng(seed)
+    for _ in range(20):
+        n = int(rng.integers(2, 8))
+        b = [int(x) for x in rng.integers(0, 1_000_000, n)]
+        t = [float(x) for x in rng.exponential(1e-3, n)]
+        alpha, beta = float(rng.uniform(0, 1e-3)), float(rng.uniform(0, 1e-9))
+        buckets, end = lo.merge_layers(b, t, alpha, beta)
+        assert end == lo.message_schedule_end(buckets, b, t, alpha, beta)
+        for mask in range(1 << (n - 1)):
+            f = [0] + [i + 1 for i in range(n - 1) if mask >> i & 1] + [n]
+            cut = [(f[i], f[i + 1]) for i in range(len(f) - 1)]
+            assert end <= lo.message_schedule_end(cut, b, t, alpha, beta) * (1 + 1e-12)

@@ -125,3 +125,108 @@ def test_two_rank_exchange_matches_single_process():
     assert np.array_equal(idx, e_idx)  # rank-major global worker order
     assert np.array_equal(dense.view(np.uint32), e_dense.view(np.uint32))
     assert np.array_equal(weights.view(np.uint32), e_w.view(np.uint32))
+
+
+# ----------------------------------------------------------- layer-wise pipeline
+BUCKETS = [(0, 1), (1, 3), (3, 4)]
+
+
+class _OracleRangeLocal:
+    """Stand-in for a rank's sparsify plan over layers [lb, le)."""
+
+    def __init__(self, lb, le):
+        import oracle.lags_oracle as lo
+        self.lb, self.le = lb, le
+        self.off = sum(SIZES[:lb])
+        self.end = sum(SIZES[:le])
+        self.K = lo.layer_plan(SIZES[lb:le], DENS[lb:le])[4]
+
+    def sparsify(self, grads, residuals, lr, idx, val):
+        import torch
+        import oracle.lags_oracle as lo
+        a, b = self.off, self.end
+        gi = [g.numpy()[a:b] for g in grads]
+        ri = [r.numpy()[a:b] for r in residuals]
+        out_idx, out_val, new = lo.sparsify(SIZES[self.lb:self.le], DENS[self.lb:self.le], gi,
+                                            ri, lr)
+        idx.copy_(torch.from_numpy((out_idx + a).reshape(-1).view(np.int32)))
+        val.copy_(torch.from_numpy(out_val.reshape(-1)))
+        for r, n in zip(residuals, new):
+            r[a:b].copy_(torch.from_numpy(n))
+
+
+class _OracleRangeTotal(_OracleRangeLocal):
+    """Stand-in for the all-workers aggregation plan over layers [lb, le)."""
+
+    def __init__(self, lb, le, P_total):
+        super().__init__(lb, le)
+        self.P = P_total
+
+    def aggregate_apply(self, idx_all, val_all, dense, weights):
+        import torch
+        import oracle.lags_oracle as lo
+        a, b = self.off, self.end
+        idx = idx_all.numpy().view(np.uint32).reshape(self.P, self.K) - np.uint32(a)
+        val = val_all.numpy().reshape(self.P, self.K)
+        d = lo.aggregate(b - a, idx, val)
+        dense[a:b].copy_(torch.from_numpy(d))
+        weights[a:b].copy_(torch.from_numpy(lo.apply_update(weights.numpy()[a:b], d)))
+
+
+def _layerwise_rank_main(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+    from layer_wise_top_b200.dist import LayerwiseLags
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        local = [_OracleRangeLocal(a, b) for a, b in BUCKETS]
+        total = [_OracleRangeTotal(a, b, P_LOCAL * world) for a, b in BUCKETS]
+        lw = LayerwiseLags(local, total, BUCKETS, P_LOCAL, torch.device("cpu"))
+        N = sum(SIZES)
+        res = [torch.zeros(N) for _ in range(P_LOCAL)]
+        dense = torch.full((N,), float("nan"))
+        weights = torch.zeros(N)
+        for s in range(STEPS):
+            grads = [torch.from_numpy(_grad(rank * P_LOCAL + p, s)) for p in range(P_LOCAL)]
+            lw.step(grads, res, LR, dense, weights)
+        q.put((rank, dense.numpy().tobytes(), weights.numpy().tobytes(),
+               [t.numpy().tobytes() for t in lw.idx_all]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_layerwise_pipeline_matches_single_process():
+    import oracle.lags_oracle as lo
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_layerwise_rank_main, args=(r, world, port, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    try:
+        out = dict((r, (d, w, i)) for r, d, w, i in (q.get(timeout=120) for _ in range(world)))
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    assert out[0] == out[1]
+    P = P_LOCAL * world
+    hist = lo.run_workload(SIZES, DENS, P, LR, STEPS, lambda p, s: _grad(p, s))
+    e_idx, _, _, e_dense, e_w = hist[-1]
+    dense = np.frombuffer(out[0][0], dtype=np.float32)
+    weights = np.frombuffer(out[0][1], dtype=np.float32)
+    assert np.array_equal(dense.view(np.uint32), e_dense.view(np.uint32))
+    assert np.array_equal(weights.view(np.uint32), e_w.view(np.uint32))
+    # each bucket's gathered lists are the whole-model lists' columns of its layers
+    _, ks, koffs, _, _ = lo.layer_plan(SIZES, DENS)
+    for (a, b), raw in zip(BUCKETS, out[0][2]):
+        got = np.frombuffer(raw, dtype=np.uint32).reshape(P, -1)
+        assert np.array_equal(got, e_idx[:, koffs[a]:koffs[b - 1] + ks[b - 1]])

@@ -76,3 +76,11 @@ def test_run_workload_carries_residual():
     vals = [float(h[1][0, 0]) for h in hist]
     assert picks == [0, 1, 2, 3, 0]
     assert vals == [1.0, 2.0, 3.0, 4.0, 4.0]
+
+
+def test_merge_hand_example():
+    pins.check_merge_hand(lo)
+
+
+def test_merge_against_every_cut():
+    pins.check_merge_bruteforce(lo)

@@ -99,7 +99,45 @@ def _sparsify_layer_emit_grad(off, k, grads, residuals, lr):
     return idx, val, new
 
 
+def _merge_variant(start_when_first_produced=False, no_start_up=False):
+    def merge(message_bytes, backward_seconds, alpha, beta):
+        L = len(message_bytes)
+        ready = [0.0] * (L + 1)
+        for l in range(L - 1, -1, -1):
+            ready[l] = ready[l + 1] + float(backward_seconds[l])
+        best, cut = [0.0] * (L + 1), [L] * (L + 1)
+        for i in range(L - 1, -1, -1):
+            nbytes = 0.0
+            for j in range(i + 1, L + 1):
+                nbytes += float(message_bytes[j - 1])
+                start = ready[j - 1] if start_when_first_produced else ready[i]
+                end = max(start, best[j]) + (0.0 if no_start_up else alpha) + beta * nbytes
+                if j == i + 1 or end <= best[i]:
+                    best[i], cut[i] = end, j
+        buckets, i = [], 0
+        while i < L:
+            buckets.append((i, cut[i]))
+            i = cut[i]
+        return buckets, best[0]
+    return merge
+
+
+def _schedule_forward_order(buckets, message_bytes, backward_seconds, alpha, beta):
+    L = len(message_bytes)
+    ready = [0.0] * (L + 1)
+    for l in range(L - 1, -1, -1):
+        ready[l] = ready[l + 1] + float(backward_seconds[l])
+    link_free = 0.0
+    for first, end in sorted(buckets):  # sends the first layers first
+        nbytes = sum(float(message_bytes[l]) for l in range(first, end))
+        link_free = max(ready[first], link_free) + alpha + beta * nbytes
+    return link_free
+
+
 MUTANTS = {
+    "merge_starts_too_early": ("merge_layers", _merge_variant(start_when_first_produced=True)),
+    "merge_without_start_up": ("merge_layers", _merge_variant(no_start_up=True)),
+    "schedule_forward_order": ("message_schedule_end", _schedule_forward_order),
     "fma_error_feedback": ("error_feedback", _ef_fma),
     "no_residual_term": ("error_feedback", _ef_grad_only),
     "tie_to_higher_index": ("magnitude_order", _order_high_index),
@@ -119,6 +157,7 @@ ALL_PINS = [
     pins.check_error_feedback_fp64, pins.check_aggregate_fp64, pins.check_apply_fp64,
     pins.check_invariants, pins.check_dense_rho1, pins.check_single_worker,
     lambda m: pins.check_k_rule(m, WORKLOADS.values()),
+    pins.check_merge_hand, pins.check_merge_bruteforce,
 ]
 
 
