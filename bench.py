@@ -57,6 +57,9 @@ def parse_args():
     ap.add_argument("--bwd-ps-per-elem", type=float, default=10.0,
                     help="--layerwise: backward time per gradient element (picoseconds) "
                          "the merge planner assumes")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture each step (one graph per gradient buffer of the pool) in a "
+                         "CUDA graph and time graph replays")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -299,14 +302,38 @@ def run_ours(args):
             f, fb = f | a, fb + b
         return f, fb
 
+    K = args.steps
+
+    def k1_events():
+        return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in local_plans]
+
+    graphs = None
+    if args.graph:
+        # one eager step creates the NCCL communicators; then one graph per
+        # gradient buffer, with the fused-pass timing events captured inside
+        step(0)
+        torch.cuda.synchronize()
+        from layer_wise_top_b200.dist import capture_step
+        g_events = [k1_events() for _ in range(pool)]
+        graphs = []
+        for j in range(pool):
+            for pl, evs in zip(local_plans, g_events[j]):
+                pl.set_events(*evs)
+            graphs.append(capture_step(step, j))
+        for pl in local_plans:
+            pl.set_events(None, None)
+        eager_step = step
+
+        def step(i):  # noqa: F811
+            graphs[i % pool].replay()
+
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
     flags, fallbacks = poll_all()
 
-    K = args.steps
-    ev_k1 = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in local_plans] for _ in range(K)]
+    ev_k1 = [k1_events() for _ in range(K)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
@@ -316,8 +343,9 @@ def run_ours(args):
     time.sleep(0.3)
     t0.record()
     for i in range(K):
-        for pl, evs in zip(local_plans, ev_k1[i]):
-            pl.set_events(*evs)
+        if graphs is None:
+            for pl, evs in zip(local_plans, ev_k1[i]):
+                pl.set_events(*evs)
         step(args.warmup + i)
     t1.record()
     torch.cuda.synchronize()
@@ -326,6 +354,9 @@ def run_ours(args):
     for pl in local_plans:
         pl.set_events(None, None)
     ms = t0.elapsed_time(t1)
+    if graphs is not None:
+        # each graph's events hold its last replay, all inside the timed region
+        ev_k1 = [g_events[j] for j in sorted({(args.warmup + i) % pool for i in range(K)})]
     # fused-pass time per step, summed over the buckets of a layer-wise step
     k1_ms = [sum(a.elapsed_time(b) for a, b in evs) for evs in ev_k1]
     flags2, fallbacks2 = poll_all()
@@ -337,6 +368,8 @@ def run_ours(args):
     # end to end through the same calls: inputs from pinned host memory each
     # step, the updated weights read back each step
     e2e = None
+    if graphs is not None:
+        step = eager_step  # the e2e leg below times the eager calls
     if not args.no_e2e and dp is None:
         host = [torch.empty(N, dtype=torch.float32, pin_memory=True) for _ in range(P)]
         for p in range(P):
@@ -372,7 +405,7 @@ def run_ours(args):
     is_dp = dp is not None
     if world > 1 or is_dp:
         dist.barrier(device_ids=[local])
-        del dp, lw  # their streams and NCCL work go before the process group
+        del dp, lw, graphs  # graphs holding NCCL calls go before the process group
         dist.destroy_process_group()
     if rank != 0:
         return 0
@@ -400,7 +433,8 @@ def run_ours(args):
                if buckets else ""), grad_pool_steps=pool,
             l2=f"inputs larger than L2: {12 * P * N / 1e9:.2f} GB streamed per step vs "
                f"{L2_BYTES / 1e6:.0f} MB L2",
-            step="lags_sparsify + lags_aggregate_apply (aggregate and apply fused)"),
+            step="lags_sparsify + lags_aggregate_apply (aggregate and apply fused)"
+                 + (", replayed from CUDA graphs" if args.graph else "")),
         "roofline": {"kernel": "k_ef_capture", "bound": "hbm", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak,

@@ -237,7 +237,9 @@ LAGS_API lags_status lags_sparsify_static(lags_plan* plan, const float* const* g
  * later lags_sparsify on this plan records `before` on its stream just before
  * it launches the fused error-feedback pass and `after` just after it, so
  * cudaEventElapsedTime(before, after) is that kernel's device time.  Pass
- * NULL, NULL to stop.  The events stay the caller's.
+ * NULL, NULL to stop.  The events stay the caller's.  Inside stream capture
+ * the records are captured as external event nodes, so every replay of the
+ * graph records them again.
  */
 LAGS_API lags_status lags_plan_set_events(lags_plan* plan, void* before, void* after);
 

@@ -324,10 +324,18 @@ lags_status lags_sparsify(lags_plan* plan, const float* const* grads, float* con
   if (!fill_workers(plan, grads, residuals, &wp, &err)) return err;
   cudaStream_t s = (cudaStream_t)stream;
   const bool timed = plan->ev_before && plan->ev_after;
+  // under stream capture the timing events become event-record nodes of the
+  // graph (recorded at every replay) instead of capture-internal markers
+  unsigned rec_flags = cudaEventRecordDefault;
+  if (timed) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return LAGS_ERR_CUDA;
+    if (cs == cudaStreamCaptureStatusActive) rec_flags = cudaEventRecordExternal;
+  }
   cudaError_t e = launch_estimate(plan->dp, wp, lr, s);
-  if (e == cudaSuccess && timed) e = cudaEventRecord(plan->ev_before, s);
+  if (e == cudaSuccess && timed) e = cudaEventRecordWithFlags(plan->ev_before, s, rec_flags);
   if (e == cudaSuccess) e = launch_ef(plan->dp, wp, lr, out_idx, out_val, s);
-  if (e == cudaSuccess && timed) e = cudaEventRecord(plan->ev_after, s);
+  if (e == cudaSuccess && timed) e = cudaEventRecordWithFlags(plan->ev_after, s, rec_flags);
   if (e == cudaSuccess) e = launch_select(plan->dp, wp, out_idx, out_val, s);
   return cuda_status(e);
 }

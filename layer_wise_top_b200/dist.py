@@ -82,11 +82,12 @@ class LayerwiseLags:
     ``lags_merge_layers``).  The backward pass produces the last layers first,
     so the buckets are processed from the last to the first, each as soon as
     its gradients exist (``ready[b]``, an event the caller records after
-    producing bucket b): sparsify the bucket on the current stream, start the
-    all-gather of its pick lists without waiting, and aggregate + apply it on
-    a second stream once the gather has landed.  The next bucket's
-    sparsification therefore overlaps the previous bucket's exchange, and all
-    of it overlaps the rest of the backward pass ("Layer-wise Adaptive
+    producing bucket b): sparsify the bucket (consecutive buckets on two
+    alternating streams), start the all-gather of its pick lists without
+    waiting, and aggregate + apply it on a third stream once the gather has
+    landed.  A bucket's selection overlaps the next bucket's fused pass, its
+    exchange overlaps the next buckets' sparsification, and all of it
+    overlaps the rest of the backward pass ("Layer-wise Adaptive
     Gradient Sparsification ..." review, "proposed method": layer-wise
     selection lets communication start before back-propagation ends).
 
@@ -115,8 +116,12 @@ class LayerwiseLags:
             self.val_local.append(torch.empty(n, dtype=torch.float32, device=device))
             self.idx_all.append(torch.empty(n * self.world, dtype=torch.int32, device=device))
             self.val_all.append(torch.empty(n * self.world, dtype=torch.float32, device=device))
-        self.agg_stream = (torch.cuda.Stream(device=self.device)
-                           if self.device.type == "cuda" else None)
+        cuda = self.device.type == "cuda"
+        self.agg_stream = torch.cuda.Stream(device=self.device) if cuda else None
+        # consecutive buckets sparsify on alternating streams, so one bucket's
+        # (latency-bound) selection overlaps the next bucket's fused pass
+        self.sp_streams = ([torch.cuda.Stream(device=self.device) for _ in range(2)]
+                           if cuda else None)
 
     @classmethod
     def create(cls, layer_sizes: Sequence[int], densities: Sequence[float],
@@ -145,15 +150,21 @@ class LayerwiseLags:
         cuda = self.agg_stream is not None
         main = torch.cuda.current_stream(self.device) if cuda else None
         if cuda:
-            self.agg_stream.wait_stream(main)  # dense/weights written before this step
-        for b in reversed(range(len(self.buckets))):
+            # inputs, dense and weights are written on `main` before this step
+            for st in (self.agg_stream, *self.sp_streams):
+                st.wait_stream(main)
+        for n, b in enumerate(reversed(range(len(self.buckets)))):
+            sp = self.sp_streams[n % 2] if cuda else None
             if ready is not None and ready[b] is not None:
-                main.wait_event(ready[b])
-            self.local[b].sparsify(grads, residuals, lr, self.idx_local[b], self.val_local[b])
-            works = [dist.all_gather_into_tensor(self.idx_all[b], self.idx_local[b],
-                                                 group=self.group, async_op=True),
-                     dist.all_gather_into_tensor(self.val_all[b], self.val_local[b],
-                                                 group=self.group, async_op=True)]
+                sp.wait_event(ready[b])
+            with torch.cuda.stream(sp) if cuda else _nullctx():
+                self.local[b].sparsify(grads, residuals, lr, self.idx_local[b],
+                                       self.val_local[b])
+                # NCCL orders the gathers by issue order and waits for `sp`
+                works = [dist.all_gather_into_tensor(self.idx_all[b], self.idx_local[b],
+                                                     group=self.group, async_op=True),
+                         dist.all_gather_into_tensor(self.val_all[b], self.val_local[b],
+                                                     group=self.group, async_op=True)]
             if cuda:
                 with torch.cuda.stream(self.agg_stream):
                     for w in works:
@@ -167,7 +178,33 @@ class LayerwiseLags:
                                               weights)
         if cuda:
             # the next step reuses the pick buffers and reads dense/weights
-            main.wait_stream(self.agg_stream)
+            for st in (self.agg_stream, *self.sp_streams):
+                main.wait_stream(st)
+
+
+class _nullctx:
+    def __enter__(self):
+        return None
+
+    def __exit__(self, *exc):
+        return False
+
+
+def capture_step(step, *args, **kwargs):
+    """Capture one call of ``step(*args, **kwargs)`` (a LAGS step on fixed
+    buffers: ``DataParallelLags.step`` or ``LayerwiseLags.step``) in a CUDA
+    graph and return it; ``graph.replay()`` then runs the same step without
+    host work per kernel or per bucket.  Run one eager step first, so that the
+    NCCL communicators exist.  Release the graphs before destroying the
+    process group."""
+    dev = torch.cuda.current_device()
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.graph(graph, stream=side):
+        step(*args, **kwargs)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    return graph
 
 
 def check_buckets(buckets: Sequence[Tuple[int, int]], num_layers: int) -> None:

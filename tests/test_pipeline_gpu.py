@@ -201,3 +201,47 @@ def test_layerwise_pipeline_one_rank_equals_plain_step(name, cut):
         assert k0 == plan.K
     finally:
         dist.destroy_process_group()
+
+
+def test_layerwise_step_replayed_from_cuda_graph():
+    import torch
+    import torch.distributed as dist
+    from layer_wise_top_b200 import Plan
+    from layer_wise_top_b200.dist import LayerwiseLags, capture_step
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(_free_port())
+    dev = torch.device("cuda", 0)
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=dev,
+                            timeout=datetime.timedelta(seconds=60))
+    graph = None
+    try:
+        w = WORKLOADS["resnet20"]
+        P, N = w.P, w.N
+        buckets = [(0, 5), (5, 6), (6, 20), (20, 21)]
+        lw = LayerwiseLags.create(w.sizes, w.densities, P, buckets, dev)
+        plan = Plan(w.sizes, w.densities, P, device=dev)
+        grads = [torch.empty(N, device=dev) for _ in range(P)]
+        res_a = [torch.zeros(N, device=dev) for _ in range(P)]
+        res_b = [torch.zeros(N, device=dev) for _ in range(P)]
+        dense_a, dense_b = torch.empty(N, device=dev), torch.empty(N, device=dev)
+        w_a, w_b = torch.zeros(N, device=dev), torch.zeros(N, device=dev)
+        idx, val = plan.empty_picks()
+        steps = 4
+        for s in range(steps):
+            for p in range(P):
+                synth.worker_grads_device(w, p, s, grads[p])
+            if s == 0:
+                lw.step(grads, res_a, w.lr, dense_a, w_a)  # eager: creates the communicator
+                graph = capture_step(lw.step, grads, res_a, w.lr, dense_a, w_a)
+            else:
+                graph.replay()
+            plan.sparsify(grads, res_b, w.lr, idx, val)
+            plan.aggregate_apply(idx, val, dense_b, w_b)
+        torch.cuda.synchronize()
+        assert np.array_equal(_u32(dense_a), _u32(dense_b))
+        assert np.array_equal(_u32(w_a), _u32(w_b))
+        for a, b in zip(res_a, res_b):
+            assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    finally:
+        graph = None
+        dist.destroy_process_group()
