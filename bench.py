@@ -57,6 +57,10 @@ def parse_args():
     ap.add_argument("--bwd-ps-per-elem", type=float, default=10.0,
                     help="--layerwise: backward time per gradient element (picoseconds) "
                          "the merge planner assumes")
+    ap.add_argument("--dense", action="store_true",
+                    help="the dense S-SGD baseline instead of LAGS: worker-ordered sum of "
+                         "lr*g (lags_dense_sum), NCCL all-reduce of the ranks' sums, division "
+                         "and update (lags_dense_finish); the job's P workers split over ranks")
     ap.add_argument("--graph", action="store_true",
                     help="capture each step (one graph per gradient buffer of the pool) in a "
                          "CUDA graph and time graph replays")
@@ -207,6 +211,105 @@ def cpu_baseline(w):
                        f"elements, zero residual), sparsify+aggregate, numpy single thread "
                        f"on {os.cpu_count()} host cores"),
             "seconds": secs}
+
+
+def run_dense(args):
+    """Dense S-SGD baseline: same workload, metric and timing rules as LAGS."""
+    import torch
+    import torch.distributed as dist
+    import synth
+    from layer_wise_top_b200.dist import DenseSgd
+    from synth.configs import WORKLOADS
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world == 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29532")
+        dist.init_process_group("nccl", rank=0, world_size=1, device_id=dev,
+                                timeout=datetime.timedelta(seconds=300))
+    else:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    w = WORKLOADS[args.config]
+    if w.P % world:
+        raise SystemExit(f"--dense needs the {w.P} workers to divide over {world} ranks")
+    P, N = w.P // world, w.N
+    ds = DenseSgd.create(N, P, dev)
+    pool = max(1, min(args.warmup + args.steps, POOL_BUDGET_BYTES // (P * N * 4)))
+    grads = []
+    for s in range(pool):
+        bufs = [torch.empty(N, dtype=torch.float32, device=dev) for _ in range(P)]
+        for p in range(P):
+            synth.worker_grads_device(w, rank * P + p, s, bufs[p])
+        grads.append(bufs)
+    dense = torch.empty(N, dtype=torch.float32, device=dev)
+    weights = torch.zeros(N, dtype=torch.float32, device=dev)
+    K = args.steps
+    ev_sum = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+
+    def step(i, evs=None):
+        if evs is not None:
+            evs[0].record()
+        ds.kernels.sum(grads[i % pool], w.lr, ds.sum)
+        if evs is not None:
+            evs[1].record()
+        if ds.world > 1:
+            dist.all_reduce(ds.sum, op=dist.ReduceOp.SUM)
+        ds.kernels.finish(ds.sum, ds.P_total, dense, weights)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t0.record()
+    for i in range(K):
+        step(args.warmup + i, ev_sum[i])
+    t1.record()
+    torch.cuda.synchronize()
+    dist.barrier(device_ids=[local])
+    clk = clocks.stop()
+    ms_t = torch.tensor([t0.elapsed_time(t1)], dtype=torch.float64, device=dev)
+    dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    sum_ms = sum(a.elapsed_time(b) for a, b in ev_sum) / K
+    dist.barrier(device_ids=[local])
+    del ds
+    dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peak, peak_kind = measured_peak()
+    sum_bytes = 4 * P * N + 4 * N
+    achieved = sum_bytes / (sum_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC + " (dense S-SGD baseline)",
+        "value": world * P * N * K / (ms_max / 1e3) / 1e9, "unit": "Gelem/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_max / K,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic: Philox4x32-10 gradients with the workload's tensor shapes",
+        "config": workload_config(
+            w, parallelism=f"data-parallel: {P} workers per rank x {world} ranks, NCCL "
+                           f"all-reduce of the dense sums", grad_pool_steps=pool,
+            step="dense S-SGD: lags_dense_sum + all-reduce + lags_dense_finish (with update)",
+            l2=f"inputs larger than L2: {4 * P * N / 1e9:.2f} GB read per step"),
+        "roofline": {"kernel": "k_dense_sum", "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes_per_launch": sum_bytes, "avg_launch_ms": sum_ms,
+                     "share_of_step": sum_ms / (ms_max / K)},
+        "cpu_baseline": None, "e2e": None, "gpu_launches": 2 * K, "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
 
 
 def run_ours(args):
@@ -459,6 +562,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.dense:
+        return run_dense(args)
     return run_ours(args)
 
 

@@ -296,6 +296,36 @@ LAGS_API lags_status lags_merge_layers(const int64_t* message_bytes,
                                        int32_t* out_num_buckets, double* out_end_seconds);
 
 /*
+ * lags_dense_sum - first half of one dense S-SGD step, the baseline LAGS-SGD
+ * is compared with ("Layer-wise Adaptive Gradient Sparsification ..." review,
+ * main findings: every worker sends its whole gradient, the averaged gradient
+ * updates the model):
+ *   sum_out_j = fl32( ((+0 + fl32(lr g_0j)) + fl32(lr g_1j)) + ... ),
+ * workers in order 0..num_workers-1.  This is the sum a LAGS step with every
+ * density 1 and zero residuals forms, so lags_dense_sum + lags_dense_finish
+ * give that step's dense update bit for bit.  With several ranks, the caller
+ * all-reduces the ranks' sums between the two calls (the all-reduce adds the
+ * ranks' sums in its own order).
+ *   grads        host array of num_workers device pointers, each a float[N]
+ *                gradient (16-byte aligned); read only.
+ *   num_workers  1 .. LAGS_MAX_WORKERS.
+ *   N            elements per buffer, >= 1.
+ *   sum_out      device float[N], 16-byte aligned; fully overwritten.
+ * No plan or workspace is involved.
+ */
+LAGS_API lags_status lags_dense_sum(const float* const* grads, int32_t num_workers, int64_t N,
+                                    float lr, float* sum_out, void* stream);
+
+/*
+ * lags_dense_finish - second half of the dense S-SGD step:
+ *   dense_out_j = fl32(sum_j / num_workers_total)   (a true IEEE division)
+ *   weights_j   = fl32(weights_j - dense_out_j)     (skipped if weights is NULL)
+ *   sum, dense_out, weights  device float[N], 16-byte aligned.
+ */
+LAGS_API lags_status lags_dense_finish(const float* sum, int64_t N, int32_t num_workers_total,
+                                       float* dense_out, float* weights, void* stream);
+
+/*
  * lags_plan_kernel_launches - how many kernels one lags_sparsify, one
  * lags_aggregate (or lags_aggregate_apply) and one lags_apply call enqueue for
  * this plan (any output pointer may be NULL).

@@ -10,7 +10,7 @@ from ._binding import (  # noqa: F401
     LAGS_ERR_UNSUPPORTED_DEVICE, LAGS_ERR_WORKSPACE, LAGS_FLAG_BAD_PICKS, LAGS_MAX_WORKERS,
     LAGS_OK, LIB_PATH, LagsError, lags_aggregate, lags_aggregate_apply, lags_apply,
     lags_adaptive_densities, lags_error_string, lags_plan_kernel_launches,
-    lags_merge_layers, lags_plan_create, lags_plan_create_range, lags_plan_destroy,
+    lags_dense_finish, lags_dense_sum, lags_merge_layers, lags_plan_create, lags_plan_create_range, lags_plan_destroy,
     lags_plan_info, lags_plan_layer, lags_plan_set_events, lags_plan_set_workspace,
     lags_sparsify, lags_sparsify_static, lags_status_poll, library,
 )
@@ -20,4 +20,7 @@ def __getattr__(name):
     if name == "Plan":
         from .plan import Plan
         return Plan
+    if name == "DenseKernels":
+        from .plan import DenseKernels
+        return DenseKernels
     raise AttributeError(name)

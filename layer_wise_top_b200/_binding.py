@@ -26,7 +26,8 @@ EXPORTED = ("lags_plan_create", "lags_plan_destroy", "lags_plan_info", "lags_pla
             "lags_plan_set_workspace", "lags_sparsify", "lags_aggregate", "lags_apply",
             "lags_status_poll", "lags_plan_set_events", "lags_sparsify_static",
             "lags_aggregate_apply", "lags_plan_kernel_launches", "lags_adaptive_densities",
-            "lags_plan_create_range", "lags_merge_layers", "lags_error_string")
+            "lags_plan_create_range", "lags_merge_layers", "lags_dense_sum",
+            "lags_dense_finish", "lags_error_string")
 
 
 class LagsError(RuntimeError):
@@ -63,6 +64,9 @@ def _load() -> ctypes.CDLL:
                                             ctypes.c_double, dp_]
     lib.lags_merge_layers.argtypes = [i64p, dp_, i32, ctypes.c_double, ctypes.c_double, i32p,
                                       i32p, dp_]
+    lib.lags_dense_sum.argtypes = [ctypes.POINTER(vp), i32, ctypes.c_int64, ctypes.c_float, vp,
+                                   vp]
+    lib.lags_dense_finish.argtypes = [vp, ctypes.c_int64, i32, vp, vp, vp]
     lib.lags_status_poll.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32),
                                      ctypes.POINTER(ctypes.c_uint32), vp]
     lib.lags_plan_set_events.argtypes = [vp, vp, vp]
@@ -214,6 +218,21 @@ def lags_merge_layers(message_bytes: Sequence[int], backward_seconds: Sequence[f
                                   ctypes.byref(end)), "lags_merge_layers")
     f = [first[i] for i in range(nb.value)] + [L]
     return [(f[i], f[i + 1]) for i in range(nb.value)], end.value
+
+
+def lags_dense_sum(grads: Sequence[int], N: int, lr: float, sum_out: int,
+                   stream: int = 0) -> None:
+    P = len(grads)
+    g = (ctypes.c_void_p * max(P, 1))(*[ctypes.c_void_p(x) for x in grads])
+    _check(_LIB.lags_dense_sum(g, P, int(N), ctypes.c_float(lr), ctypes.c_void_p(sum_out),
+                               ctypes.c_void_p(stream)), "lags_dense_sum")
+
+
+def lags_dense_finish(sum_in: int, N: int, num_workers_total: int, dense_out: int,
+                      weights: int = 0, stream: int = 0) -> None:
+    _check(_LIB.lags_dense_finish(ctypes.c_void_p(sum_in), int(N), int(num_workers_total),
+                                  ctypes.c_void_p(dense_out), ctypes.c_void_p(weights),
+                                  ctypes.c_void_p(stream)), "lags_dense_finish")
 
 
 def lags_apply(plan, weights: int, dense_out: int, stream: int = 0) -> None:

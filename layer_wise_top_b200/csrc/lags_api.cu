@@ -435,6 +435,31 @@ lags_status lags_merge_layers(const int64_t* message_bytes, const double* backwa
   return LAGS_OK;
 }
 
+lags_status lags_dense_sum(const float* const* grads, int32_t num_workers, int64_t N, float lr,
+                           float* sum_out, void* stream) {
+  if (!grads || !sum_out || num_workers < 1 || num_workers > LAGS_MAX_WORKERS || N < 1)
+    return LAGS_ERR_INVALID_ARG;
+  if (!aligned(sum_out, 16)) return LAGS_ERR_ALIGNMENT;
+  DenseGrads gp;
+  std::memset(&gp, 0, sizeof(gp));
+  for (int32_t p = 0; p < num_workers; ++p) {
+    if (!grads[p]) return LAGS_ERR_INVALID_ARG;
+    if (!aligned(grads[p], 16)) return LAGS_ERR_ALIGNMENT;
+    gp.g[p] = grads[p];
+  }
+  return cuda_status(launch_dense_sum(gp, (uint32_t)num_workers, (uint64_t)N, lr, sum_out,
+                                      (cudaStream_t)stream));
+}
+
+lags_status lags_dense_finish(const float* sum, int64_t N, int32_t num_workers_total,
+                              float* dense_out, float* weights, void* stream) {
+  if (!sum || !dense_out || N < 1 || num_workers_total < 1) return LAGS_ERR_INVALID_ARG;
+  if (!aligned(sum, 16) || !aligned(dense_out, 16) || (weights && !aligned(weights, 16)))
+    return LAGS_ERR_ALIGNMENT;
+  return cuda_status(launch_dense_finish(sum, (uint64_t)N, (uint32_t)num_workers_total,
+                                         dense_out, weights, (cudaStream_t)stream));
+}
+
 lags_status lags_plan_kernel_launches(const lags_plan* plan, int32_t* sparsify,
                                       int32_t* aggregate, int32_t* apply) {
   if (!plan) return LAGS_ERR_INVALID_ARG;

@@ -75,6 +75,11 @@ struct WorkerPtrs {
   float* r[LAGS_MAX_WORKERS];
 };
 
+// Gradient buffers of the dense S-SGD baseline, one per worker.
+struct DenseGrads {
+  const float* g[LAGS_MAX_WORKERS];
+};
+
 // Device status words (in the workspace).
 enum StatusWord : uint32_t { kStatusFlags = 0, kStatusFallbacks = 1, kStatusWords = 64 };
 
@@ -115,6 +120,10 @@ cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStrea
 cudaError_t launch_aggregate(const DevPlan& dp, const uint32_t* idx, const float* val,
                              float* dense, float* weights, cudaStream_t s);
 cudaError_t launch_apply(uint32_t first, uint32_t end, float* w, const float* dense, cudaStream_t s);
+cudaError_t launch_dense_sum(const DenseGrads& gp, uint32_t P, uint64_t N, float lr, float* sum,
+                             cudaStream_t s);
+cudaError_t launch_dense_finish(const float* sum, uint64_t N, uint32_t P, float* dense,
+                                float* weights, cudaStream_t s);
 
 // The fused error-feedback pass used by lags_sparsify.
 inline cudaError_t launch_ef(const DevPlan& dp, const WorkerPtrs& wp, float lr, uint32_t* out_idx,

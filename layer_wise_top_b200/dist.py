@@ -182,6 +182,42 @@ class LayerwiseLags:
                 main.wait_stream(st)
 
 
+class DenseSgd:
+    """Dense S-SGD over `world` ranks x `workers_per_rank` workers, the
+    baseline of the LAGS review's comparisons: every rank sums its workers'
+    fl(lr g) in worker order (``lags_dense_sum``), the ranks all-reduce the
+    sums (NCCL, over NVLink), and every rank divides by the job's worker count
+    and updates its weights (``lags_dense_finish``).  With one rank the result
+    is the LAGS step at density 1, bit for bit; with more, the all-reduce adds
+    the ranks' sums in its own order.  The message is the whole gradient,
+    4 N bytes per rank, against 8 K bytes per worker for LAGS."""
+
+    def __init__(self, kernels, N: int, workers_per_rank: int, device: torch.device,
+                 group: Optional[dist.ProcessGroup] = None):
+        self.kernels = kernels
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.N = int(N)
+        self.P_local = int(workers_per_rank)
+        self.P_total = self.P_local * self.world
+        self.sum = torch.empty(self.N, dtype=torch.float32, device=device)
+
+    @classmethod
+    def create(cls, N: int, workers_per_rank: int, device: torch.device,
+               group: Optional[dist.ProcessGroup] = None) -> "DenseSgd":
+        from .plan import DenseKernels
+        return cls(DenseKernels(N, device), N, workers_per_rank, device, group)
+
+    def step(self, grads: List[torch.Tensor], lr: float, dense_out: torch.Tensor,
+             weights: torch.Tensor) -> None:
+        if len(grads) != self.P_local:
+            raise ValueError(f"need {self.P_local} gradient buffers per rank")
+        self.kernels.sum(grads, lr, self.sum)
+        if self.world > 1:
+            dist.all_reduce(self.sum, op=dist.ReduceOp.SUM, group=self.group)
+        self.kernels.finish(self.sum, self.P_total, dense_out, weights)
+
+
 class _nullctx:
     def __enter__(self):
         return None

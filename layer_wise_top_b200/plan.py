@@ -124,3 +124,32 @@ class Plan:
     def poll(self, stream: Optional[torch.cuda.Stream] = None):
         """(flags, exact_fallbacks) since the last poll; synchronises the stream."""
         return B.lags_status_poll(self.handle, _stream(stream, self.device))
+
+
+class DenseKernels:
+    """The dense S-SGD baseline's two kernels on torch tensors (no plan)."""
+
+    def __init__(self, N: int, device: Optional[torch.device] = None):
+        self.N = int(N)
+        self.device = torch.device(device if device is not None else "cuda")
+
+    def sum(self, grads: List[torch.Tensor], lr: float, out: torch.Tensor,
+            stream: Optional[torch.cuda.Stream] = None) -> None:
+        """out = worker-ordered sum of fl(lr * g_p)."""
+        for i, g in enumerate(grads):
+            _need(g, torch.float32, self.N, f"grads[{i}]")
+        _need(out, torch.float32, self.N, "sum_out")
+        B.lags_dense_sum([g.data_ptr() for g in grads], self.N, lr, out.data_ptr(),
+                         _stream(stream, self.device))
+
+    def finish(self, sum_in: torch.Tensor, P_total: int, dense_out: torch.Tensor,
+               weights: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None) -> None:
+        """dense_out = sum / P_total; weights -= dense_out when given."""
+        _need(sum_in, torch.float32, self.N, "sum")
+        _need(dense_out, torch.float32, self.N, "dense_out")
+        if weights is not None:
+            _need(weights, torch.float32, self.N, "weights")
+        B.lags_dense_finish(sum_in.data_ptr(), self.N, P_total, dense_out.data_ptr(),
+                            weights.data_ptr() if weights is not None else 0,
+                            _stream(stream, self.device))

@@ -6,7 +6,8 @@ product path (``layer_wise_top_b200``) never imports it and has no CPU
 fallback.
 """
 from .lags_oracle import (  # noqa: F401
-    adaptive_densities, aggregate, aggregate_layer, apply_update, error_feedback, k_of, layer_plan,
+    adaptive_densities, aggregate, aggregate_layer, apply_update, dense_sgd_update, error_feedback,
+    k_of, layer_plan,
     magnitude_order, merge_layers, message_schedule_end, run_workload, select_layer, sparsify,
     sparsify_layer,
 )

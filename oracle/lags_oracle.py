@@ -191,6 +191,17 @@ def adaptive_densities(sizes: Sequence[int], backward_seconds: Sequence[float], 
     return out
 
 
+def dense_sgd_update(grads: Sequence[np.ndarray], lr: float) -> np.ndarray:
+    """Dense S-SGD update, the baseline of the LAGS review's comparisons
+    ("main findings": LAGS-SGD against dense S-SGD, where every worker sends
+    its whole gradient): every worker sends fl32(lr g) at every position (R1
+    with a zero residual), aggregated in worker order as in R6."""
+    P, N = len(grads), grads[0].size
+    vals = np.stack([error_feedback(np.zeros(N, dtype=F32), g, lr) for g in grads])
+    idx = np.tile(np.arange(N, dtype=np.uint32), (P, 1))
+    return aggregate_layer(0, N, idx, vals)
+
+
 def message_schedule_end(buckets: Sequence[Tuple[int, int]], message_bytes: Sequence[int],
                          backward_seconds: Sequence[float], alpha: float,
                          beta: float) -> float:

@@ -230,3 +230,79 @@ def test_two_rank_layerwise_pipeline_matches_single_process():
     for (a, b), raw in zip(BUCKETS, out[0][2]):
         got = np.frombuffer(raw, dtype=np.uint32).reshape(P, -1)
         assert np.array_equal(got, e_idx[:, koffs[a]:koffs[b - 1] + ks[b - 1]])
+
+
+# ------------------------------------------------------------- dense S-SGD
+class _OracleDense:
+    """Stand-in for the dense S-SGD kernels."""
+
+    def sum(self, grads, lr, out):
+        import torch
+        acc = np.zeros(out.numel(), dtype=np.float32)
+        for g in grads:
+            acc = np.add(acc, np.multiply(np.float32(lr), g.numpy(), dtype=np.float32),
+                         dtype=np.float32)
+        out.copy_(torch.from_numpy(acc))
+
+    def finish(self, s, P_total, dense, weights):
+        import torch
+        import oracle.lags_oracle as lo
+        d = np.divide(s.numpy(), np.float32(P_total), dtype=np.float32)
+        dense.copy_(torch.from_numpy(d))
+        weights.copy_(torch.from_numpy(lo.apply_update(weights.numpy(), d)))
+
+
+def _dense_rank_main(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+    from layer_wise_top_b200.dist import DenseSgd
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        N = sum(SIZES)
+        ds = DenseSgd(_OracleDense(), N, P_LOCAL, torch.device("cpu"))
+        dense = torch.empty(N)
+        weights = torch.zeros(N)
+        grads = [torch.from_numpy(_grad(rank * P_LOCAL + p, 0)) for p in range(P_LOCAL)]
+        ds.step(grads, LR, dense, weights)
+        q.put((rank, dense.numpy().tobytes(), weights.numpy().tobytes()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_dense_sgd_all_reduce():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dense_rank_main, args=(r, world, port, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    try:
+        out = dict((r, (d, w)) for r, d, w in (q.get(timeout=120) for _ in range(world)))
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    assert all(p.exitcode == 0 for p in procs)
+    assert out[0] == out[1]
+    # each rank sums its own workers in order; the two ranks' sums are added once
+    f = np.float32
+    partial = []
+    for r in range(world):
+        acc = np.zeros(sum(SIZES), dtype=f)
+        for p in range(P_LOCAL):
+            acc = np.add(acc, np.multiply(f(LR), _grad(r * P_LOCAL + p, 0), dtype=f), dtype=f)
+        partial.append(acc)
+    want = np.divide(np.add(partial[0], partial[1], dtype=f), f(world * P_LOCAL), dtype=f)
+    dense = np.frombuffer(out[0][0], dtype=f)
+    assert np.array_equal(dense.view(np.uint32), want.view(np.uint32))
+    import oracle.lags_oracle as lo
+    w_want = lo.apply_update(np.zeros(sum(SIZES), dtype=f), want)
+    assert np.array_equal(np.frombuffer(out[0][1], dtype=f).view(np.uint32),
+                          w_want.view(np.uint32))

@@ -84,3 +84,22 @@ def test_merge_hand_example():
 
 def test_merge_against_every_cut():
     pins.check_merge_bruteforce(lo)
+
+
+def test_dense_sgd_integer_closed_form():
+    # integer gradients, lr = 1: every partial sum is exact, so P * dense is
+    # the integer sum and dense is its correctly rounded quotient
+    rng = np.random.default_rng(12)
+    P, N = 5, 257
+    g = [rng.integers(-1000, 1000, N).astype(np.float32) for _ in range(P)]
+    tot = np.sum(np.stack(g).astype(np.int64), axis=0)
+    got = lo.dense_sgd_update(g, 1.0)
+    assert np.array_equal(got, (tot.astype(np.float64) / P).astype(np.float32))
+
+
+def test_dense_sgd_is_lags_at_density_one():
+    rng = np.random.default_rng(13)
+    sizes = [7, 300, 33]
+    g = [rng.standard_normal(sum(sizes)).astype(np.float32) for _ in range(3)]
+    hist = lo.run_workload(sizes, [1.0] * 3, 3, 0.25, 1, lambda p, s: g[p])
+    assert np.array_equal(lo.dense_sgd_update(g, 0.25).view(np.uint32), hist[0][3].view(np.uint32))
