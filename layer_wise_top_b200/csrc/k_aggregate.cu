@@ -21,6 +21,7 @@
 // picks.  It also checks that the lists are ascending and inside their layer.
 #include "block_ops.cuh"
 #include "lags_internal.cuh"
+#include "tma.cuh"
 
 namespace lags {
 
@@ -74,7 +75,11 @@ constexpr uint32_t kAggPickCap = 2048;
 // workers' picks into shared memory one worker at a time instead.
 constexpr uint32_t kAggOwnerMax = 512;
 
+// Zeros the owner path sends to the dense output with bulk stores.
+constexpr uint32_t kAggZeroBytes = 4096;  // keeps 4 tile-accumulator CTAs per SM
+
 struct AggShared {
+  float4 zero[kAggZeroBytes / 16];       // first: 16-byte aligned source of the bulk stores
   uint32_t loc[kAggPickCap];             // pick position inside the group, per worker ascending
   float val[kAggPickCap];
   uint32_t base[LAGS_MAX_WORKERS + 1];   // first staged pick of each worker
@@ -110,6 +115,10 @@ __global__ void __launch_bounds__(kAggThreads, 4)
   const float fP = (float)P;
   const uint64_t K = dp.K;
   const int tid = threadIdx.x;
+  // source of the bulk zero stores (this CTA's own shared memory)
+  for (uint32_t i = tid; i < kAggZeroBytes / 16; i += kAggThreads)
+    sh.zero[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  fence_proxy_async_shared();  // visible to the bulk copies after the next barrier
   pdl_wait();
 
   if (ld.k == ld.d) {
@@ -142,6 +151,23 @@ __global__ void __launch_bounds__(kAggThreads, 4)
   if (tid < (int)P) sh.base[tid] = before;
   if (tid == 0) sh.base[P] = total;
   __syncthreads();
+  const bool staged = total <= kAggPickCap;
+  // the tile accumulator covers one tile: groups of several tiles use the
+  // owner search (the plan groups only tiles expected to hold few picks)
+  const bool owner_path = staged && (total <= kAggOwnerMax || !have_acc || nt > 1);
+  const uint32_t head = min(td.len, (4u - (td.start & 3u)) & 3u);
+  const uint32_t nvec = (td.len - head) / 4;
+  if (owner_path && tid == 0 && nvec > 0) {
+    // the group's 16-byte-aligned middle is cleared by the bulk-copy engine
+    // while the CTA stages and sums its picks; waited for before the sums
+    char* dst = reinterpret_cast<char*>(dense + td.start + head);
+    const uint64_t bytes = (uint64_t)nvec * 16;
+    for (uint64_t o = 0; o < bytes; o += kAggZeroBytes) {
+      const uint64_t n = bytes - o < kAggZeroBytes ? bytes - o : kAggZeroBytes;
+      bulk_store(dst + o, sh.zero, (uint32_t)n);
+    }
+    bulk_commit();
+  }
   auto worker_of = [&](uint32_t i) {  // staged pick i: last worker p with base[p] <= i
     uint32_t p = 0, hi = P - 1;
     while (p < hi) {
@@ -150,7 +176,6 @@ __global__ void __launch_bounds__(kAggThreads, 4)
     }
     return p;
   };
-  const bool staged = total <= kAggPickCap;
   if (staged) {
     for (uint32_t i = tid; i < total; i += kAggThreads) {
       const uint32_t p = worker_of(i);
@@ -160,12 +185,7 @@ __global__ void __launch_bounds__(kAggThreads, 4)
       sh.val[i] = __ldg(val + slot);
     }
   }
-  const uint32_t head = min(td.len, (4u - (td.start & 3u)) & 3u);
-  const uint32_t nvec = (td.len - head) / 4;
-
-  // the tile accumulator covers one tile: groups of several tiles use the
-  // owner search (the plan groups only tiles expected to hold few picks)
-  if (staged && (total <= kAggOwnerMax || !have_acc || nt > 1)) {
+  if (owner_path) {
     // ---- few picks: zeros everywhere, then each position's first owner ----
     // Owned positions, their sums and their old weights are all gathered
     // before this thread's first store: a load issued after stores waits for
@@ -211,20 +231,13 @@ __global__ void __launch_bounds__(kAggThreads, 4)
       for (uint32_t j = 0; j < OI; ++j)
         if (own_x[j] != 0xFFFFFFFFu) own_w[j] = weights[td.start + own_x[j]];
     }
+    // the unaligned ends of the group (the middle went to the bulk copies)
     for (uint32_t i = tid; i < head; i += kAggThreads) dense[td.start + i] = 0.0f;
-    {
-      // 8 independent 16-byte stores per trip: the loop overhead, not DRAM,
-      // limited a one-store loop
-      float4* d4 = reinterpret_cast<float4*>(dense + td.start + head);
-      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-      uint32_t v = tid;
-      for (; v + 7 * kAggThreads < nvec; v += 8 * kAggThreads) {
-#pragma unroll
-        for (uint32_t u = 0; u < 8; ++u) __stcs(d4 + v + u * kAggThreads, z);
-      }
-      for (; v < nvec; v += kAggThreads) __stcs(d4 + v, z);
-    }
     for (uint32_t i = head + 4 * nvec + tid; i < td.len; i += kAggThreads) dense[td.start + i] = 0.0f;
+    if (tid == 0 && nvec > 0) {
+      bulk_wait_all();             // the bulk zeros have landed ...
+      fence_proxy_async_global();  // ... and are ordered before generic stores
+    }
     __syncthreads();  // orders the zeros before the sums written below
 #pragma unroll
     for (uint32_t j = 0; j < OI; ++j) {

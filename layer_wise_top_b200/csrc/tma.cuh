@@ -1,6 +1,6 @@
 // Thin wrappers over the sm_90+/sm_100 PTX used to stream tiles with the bulk
 // copy engine: mbarrier phase tracking and cp.async.bulk global -> shared.
-// Only the plain (non-multicast) bulk copy is used.
+// Only the plain (non-multicast) bulk copies are used, in both directions.
 #pragma once
 
 #include <stdint.h>
@@ -59,6 +59,32 @@ __device__ __forceinline__ void bulk_load(void* dst_smem, const void* src_gmem, 
           "r"(smem_addr(dst_smem)),
       "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
+}
+
+// Bulk copy of `bytes` (multiple of 16; both addresses 16-byte aligned) from
+// this CTA's shared memory to global memory, tracked by the executing
+// thread's bulk async-groups (bulk_commit / bulk_wait_all).
+__device__ __forceinline__ void bulk_store(void* dst_gmem, const void* src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst_gmem),
+               "r"(smem_addr(src_smem)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until every bulk store this thread committed has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy (bulk copy) reads of them.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Order completed async-proxy writes to global memory before this thread's
+// later generic-proxy accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 }  // namespace lags
