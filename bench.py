@@ -48,6 +48,12 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="vgg16",
                     choices=["resnet20", "vgg16", "resnet50", "lstm_ptb", "gpt_1_3b"])
+    ap.add_argument("--tensors", default=None, metavar="A:B",
+                    help="only tensors A..B-1 of the workload (a smaller case of the same "
+                         "kernels, for profiling)")
+    ap.add_argument("--pool", type=int, default=None,
+                    help="at most this many pre-generated gradient steps on the device "
+                         "(default: one per step, within 48 GB)")
     ap.add_argument("--dp", action="store_true",
                     help="data-parallel LAGS: split the job's P workers over the ranks and "
                          "all-gather their pick lists (strong scaling) instead of replicas")
@@ -67,6 +73,17 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
+
+
+def workload(args):
+    from synth.configs import WORKLOADS
+    w = WORKLOADS[args.config]
+    if args.tensors:
+        a, b = (int(x) for x in args.tensors.split(":"))
+        if not 0 <= a < b <= w.L:
+            raise SystemExit(f"--tensors {args.tensors}: the workload has {w.L} tensors")
+        w = w.scaled(f"{w.name}[{a}:{b}]", tensors=w.tensors[a:b])
+    return w
 
 
 def workload_config(w, **extra):
@@ -170,7 +187,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     from synth.configs import WORKLOADS
-    w = WORKLOADS[args.config]
+    w = workload(args)
     layers, total = oracle_sample_layers(w, 4_000_000)
     sample = (f"one worker per step (worker = step mod P), layers {layers[0]}..{layers[-1]} "
               f"({total} elements), zero residual; numpy oracle, single thread")
@@ -233,12 +250,13 @@ def run_dense(args):
                                 timeout=datetime.timedelta(seconds=300))
     else:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-    w = WORKLOADS[args.config]
+    w = workload(args)
     if w.P % world:
         raise SystemExit(f"--dense needs the {w.P} workers to divide over {world} ranks")
     P, N = w.P // world, w.N
     ds = DenseSgd.create(N, P, dev)
-    pool = max(1, min(args.warmup + args.steps, POOL_BUDGET_BYTES // (P * N * 4)))
+    pool = max(1, min(args.warmup + args.steps, POOL_BUDGET_BYTES // (P * N * 4),
+                      args.pool or 1 << 30))
     grads = []
     for s in range(pool):
         bufs = [torch.empty(N, dtype=torch.float32, device=dev) for _ in range(P)]
@@ -332,7 +350,7 @@ def run_ours(args):
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    w = WORKLOADS[args.config]
+    w = workload(args)
     P, N = w.P, w.N
     dp = None
     lw = None
@@ -372,7 +390,8 @@ def run_ours(args):
     local_plans = lw.local if lw is not None else [plan]
     status_plans = local_plans + (lw.total if lw is not None else [])
     step_bytes = P * N * 4
-    pool = max(1, min(args.warmup + args.steps, POOL_BUDGET_BYTES // step_bytes))
+    pool = max(1, min(args.warmup + args.steps, POOL_BUDGET_BYTES // step_bytes,
+                      args.pool or 1 << 30))
     grads = []
     for s in range(pool):
         bufs = [torch.empty(N, dtype=torch.float32, device=dev) for _ in range(P)]
