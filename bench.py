@@ -520,6 +520,22 @@ def run_ours(args):
                "unit": "Gelem/s", "steps": ke, "h2d_bytes_per_step": P * N * 4,
                "d2h_bytes_per_step": N * 4}
 
+    # lags_apply alone (outside the step: the step applies the update fused
+    # into the aggregation), 12 bytes per element
+    apply_ms = None
+    if dp is None:
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        ka = max(3, min(K, 10))
+        plan.apply(weights, dense)
+        torch.cuda.synchronize()
+        a0.record()
+        for _ in range(ka):
+            plan.apply(weights, dense)
+        a1.record()
+        torch.cuda.synchronize()
+        apply_ms = a0.elapsed_time(a1) / ka
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
@@ -537,6 +553,8 @@ def run_ours(args):
     k1_bytes = 12 * P * N
     achieved = k1_bytes / (k1_avg / 1e3) / 1e9
     job_elems = world * P * N  # all ranks' elements
+    K_picks = sum(pl.K for pl in local_plans)
+    step_alg_bytes = 12 * P * N + 4 * N + 16 * P * K_picks
     line = {
         "metric": METRIC,
         "value": job_elems * K / (ms_max / 1e3) / 1e9,
@@ -567,6 +585,14 @@ def run_ours(args):
                                         "elements"),
                      "algorithmic_bytes_per_launch": k1_bytes, "avg_launch_ms": k1_avg,
                      "share_of_step": k1_avg / (ms_max / K)},
+        "step_hbm": {
+            "algorithmic_bytes": step_alg_bytes,
+            "formula": "12 P N (grad, residual in, residual out) + 4 N (dense) + 16 P K "
+                       "(picks written, then read back)",
+            "achieved_gbs": step_alg_bytes / (ms_max / K / 1e3) / 1e9,
+            "frac": step_alg_bytes / (ms_max / K / 1e3) / 1e9 / peak},
+        "apply": None if apply_ms is None else {
+            "ms": apply_ms, "bytes": 12 * N, "achieved_gbs": 12 * N / (apply_ms / 1e3) / 1e9},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches_per_step * K,
