@@ -68,6 +68,11 @@ typedef enum {
 /* Largest number of simulated workers one plan accepts. */
 #define LAGS_MAX_WORKERS 256
 
+/* Largest N (elements per worker buffer) a plan accepts: indices are uint32,
+ * and the kernels' index arithmetic (a tile's 16-byte groups, a grid's
+ * threads past the end) stays below 2^32 with this much headroom. */
+#define LAGS_MAX_ELEMENTS 4294901760ull /* 2^32 - 65536 */
+
 /* Bits of the device status word returned by lags_status_poll(). */
 #define LAGS_FLAG_BAD_PICKS 0x1u /* lags_aggregate saw an unsorted or out-of-layer index */
 #define LAGS_FLAG_TIMEOUT 0x4u   /* a kernel's bounded wait on its own bulk copies gave up;
@@ -78,7 +83,7 @@ typedef enum {
 /*
  * lags_plan_create - describe one flattened gradient buffer.
  *   layer_sizes  host, [num_layers] int64: d_l > 0, layers stored back to back
- *                in this order; N = sum d_l must be < 2^32.
+ *                in this order; N = sum d_l must be <= LAGS_MAX_ELEMENTS.
  *   densities    host, [num_layers] double: rho_l in (0, 1]; k_l follows the
  *                rule above (rho_l = 1 or k_l = d_l sends the layer densely).
  *   num_workers  P, 1 <= P <= LAGS_MAX_WORKERS.

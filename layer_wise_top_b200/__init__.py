@@ -7,7 +7,7 @@ CPU fallback.
 """
 from ._binding import (  # noqa: F401
     EXPORTED, LAGS_ERR_ALIGNMENT, LAGS_ERR_BAD_PICKS, LAGS_ERR_CUDA, LAGS_ERR_INVALID_ARG,
-    LAGS_ERR_UNSUPPORTED_DEVICE, LAGS_ERR_WORKSPACE, LAGS_FLAG_BAD_PICKS, LAGS_MAX_WORKERS,
+    LAGS_ERR_UNSUPPORTED_DEVICE, LAGS_ERR_WORKSPACE, LAGS_FLAG_BAD_PICKS, LAGS_MAX_ELEMENTS, LAGS_MAX_WORKERS,
     LAGS_OK, LIB_PATH, LagsError, lags_aggregate, lags_aggregate_apply, lags_apply,
     lags_adaptive_densities, lags_error_string, lags_plan_kernel_launches,
     lags_dense_finish, lags_dense_sum, lags_merge_layers, lags_plan_create, lags_plan_create_range, lags_plan_destroy,

@@ -18,6 +18,7 @@ LAGS_ERR_UNSUPPORTED_DEVICE = 4
 LAGS_ERR_WORKSPACE = 5
 LAGS_ERR_BAD_PICKS = 6
 LAGS_MAX_WORKERS = 256
+LAGS_MAX_ELEMENTS = (1 << 32) - 65536
 LAGS_FLAG_BAD_PICKS = 0x1
 LAGS_FLAG_INTERNAL = 0x2
 LAGS_FLAG_TIMEOUT = 0x4

@@ -361,8 +361,8 @@ __global__ void __launch_bounds__(256) k_apply(uint32_t first, uint32_t end,
     w4[i] = a;
   }
   if (gid < a0 - first) w[first + gid] = __fsub_rn(w[first + gid], dense[first + gid]);
-  const uint32_t tail = a0 + n4 * 4 + gid;
-  if (tail < end) w[tail] = __fsub_rn(w[tail], dense[tail]);
+  const uint32_t tail0 = a0 + n4 * 4;  // (compared as a count: tail0 + gid may pass 2^32)
+  if (gid < end - tail0) w[tail0 + gid] = __fsub_rn(w[tail0 + gid], dense[tail0 + gid]);
 }
 
 cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStream_t s) {

@@ -112,7 +112,7 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
   for (int32_t l = 0; l < layer_begin; ++l) {
     if (layer_sizes[l] <= 0) return LAGS_ERR_INVALID_ARG;
     off += (uint64_t)layer_sizes[l];
-    if (off >= (1ull << 32)) return LAGS_ERR_INVALID_ARG;
+    if (off > LAGS_MAX_ELEMENTS) return LAGS_ERR_INVALID_ARG;
   }
   lags_plan* plan = new (std::nothrow) lags_plan();
   if (!plan) return LAGS_ERR_INVALID_ARG;
@@ -129,7 +129,7 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
     }
     double kd = std::ceil(rho * (double)d);
     uint64_t k = kd < 1.0 ? 1 : (kd >= (double)d ? (uint64_t)d : (uint64_t)kd);
-    if (off + (uint64_t)d >= (1ull << 32)) {  // indices are uint32
+    if (off + (uint64_t)d > LAGS_MAX_ELEMENTS) {  // indices are uint32, with headroom
       delete plan;
       return LAGS_ERR_INVALID_ARG;
     }

@@ -98,3 +98,17 @@ def test_k_rule_uses_double_density():
         assert L.lags_plan_layer(h, 1)[1] == 2048
     finally:
         L.lags_plan_destroy(h)
+
+
+def test_plan_size_limit():
+    # N may reach LAGS_MAX_ELEMENTS (2^32 - 65536) and not one element more
+    top = L.LAGS_MAX_ELEMENTS
+    h = L.lags_plan_create([top - 100_003 - 7, 100_003, 7], [1e-7, 0.001, 0.5], 1)
+    N, K, _ = L.lags_plan_info(h)
+    assert N == top and L.lags_plan_layer(h, 2)[0] == top - 7
+    L.lags_plan_destroy(h)
+    with pytest.raises(L.LagsError):
+        L.lags_plan_create([top - 6, 7], [0.01, 0.5], 1)
+    # a range plan past the limit is rejected too, even if its own layers are small
+    with pytest.raises(L.LagsError):
+        L.lags_plan_create_range([top, 5], [0.01, 0.5], 1, 1, 2)
