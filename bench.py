@@ -218,7 +218,7 @@ def run_reference(args):
 def cpu_baseline(w):
     layers, total = oracle_sample_layers(w, 8_000_000)
     secs, elems, step = 0.0, 0, 0
-    while secs < 10.0 and step < 8:
+    while secs < 12.0 and step < 16:
         t, e = time_oracle(w, step % w.P, step, layers)
         secs += t
         elems += e

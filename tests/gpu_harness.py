@@ -39,6 +39,7 @@ class GpuRun:
         """One step; `fused` uses lags_aggregate_apply instead of
         lags_aggregate + lags_apply (the results must be identical)."""
         if self.keep_prev:
+            self.prev = None  # drop the old copy first: full-size workloads fill the device
             self.prev = [r.clone() for r in self.res]
         self.plan.sparsify(self.grads, self.res, self.lr, self.idx, self.val)
         if fused:

@@ -91,3 +91,5 @@ def test_max_size_plan():
             picked_ties = idx[val.abs() == vmin]
             assert first_tie > int(picked_ties.max())
         torch.cuda.synchronize()
+    del run, g, prev, res, dense
+    torch.cuda.empty_cache()  # about 100 GB: leave the device to the next tests
