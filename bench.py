@@ -54,6 +54,9 @@ def parse_args():
     ap.add_argument("--pool", type=int, default=None,
                     help="at most this many pre-generated gradient steps on the device "
                          "(default: one per step, within 48 GB)")
+    ap.add_argument("--global-topk", type=float, default=None, metavar="RHO",
+                    help="SLGS: one top-k over the whole flattened model at density RHO "
+                         "instead of layer-wise (single-GPU replicas only)")
     ap.add_argument("--dp", action="store_true",
                     help="data-parallel LAGS: split the job's P workers over the ranks and "
                          "all-gather their pick lists (strong scaling) instead of replicas")
@@ -384,6 +387,8 @@ def run_ours(args):
             dp = DataParallelLags.create(w.sizes, w.densities, P // world, dev)
         P = P // world  # workers held by this rank
         plan = dp.local[0] if lw is not None else dp.local
+    elif args.global_topk is not None:
+        plan = Plan([N], [args.global_topk], P, device=dev)
     else:
         plan = Plan(w.sizes, w.densities, P, device=dev)
     # plans whose fused pass is timed and whose status words are read
@@ -573,6 +578,8 @@ def run_ours(args):
                if buckets else ""), grad_pool_steps=pool,
             l2=f"inputs larger than L2: {12 * P * N / 1e9:.2f} GB streamed per step vs "
                f"{L2_BYTES / 1e6:.0f} MB L2",
+            selection=(f"global top-k over all {N} elements at density {args.global_topk}"
+                       if args.global_topk is not None else "layer-wise top-k"),
             step="lags_sparsify + lags_aggregate_apply (aggregate and apply fused)"
                  + (", replayed from CUDA graphs" if args.graph else "")),
         "roofline": {"kernel": "k_ef_capture", "bound": "hbm", "achieved": achieved,

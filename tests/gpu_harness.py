@@ -131,3 +131,63 @@ def check_invariants(run: GpuRun, workers: Iterable[int], check_dense: bool = Tr
             dense[li] = dense[li] + val_all[p]
         dense = dense / torch.tensor(float(run.P), dtype=torch.float32, device="cuda")
         assert torch.equal(dense.view(torch.int32), run.dense.view(torch.int32)), "dense"
+
+
+def check_layer_chunked(run: GpuRun, l: int, lr: float, chunk: int = 1 << 28) -> None:
+    """The properties that fix layer l's top-k, checked on the GPU in chunks
+    (for layers too large for the oracle or for whole-layer temporaries),
+    for every worker: picks ascending and inside the layer, each value equal
+    to acc at its index, picked residuals +0 and all others acc, every picked
+    magnitude at least every unpicked one, ties to the lower index; and the
+    dense update recomputed from the picks in worker order.  Needs
+    keep_prev=True."""
+    assert run.prev is not None, "run with keep_prev=True"
+    off, k, koff = run.plan.layers[l]
+    d = run.plan.sizes[l]
+    K = run.plan.K
+    lr_t = torch.tensor(lr, dtype=torch.float32, device="cuda")
+
+    def bits(t):
+        return t.view(torch.int32)
+
+    for p in range(run.P):
+        idx = run.idx[p * K + koff:p * K + koff + k].to(torch.int64) & 0xFFFFFFFF
+        val = run.val[p * K + koff:p * K + koff + k]
+        assert bool((idx[1:] > idx[:-1]).all()) and int(idx[0]) >= off
+        assert int(idx[-1]) < off + d
+        g, prev, res = run.grads[p], run.prev[p], run.res[p]
+        assert torch.equal(bits(val), bits(prev[idx] + lr_t * g[idx])), f"values p={p}"
+        assert int(bits(res[idx]).abs().max()) == 0, f"picked residuals p={p}"
+        vmin = float(val.abs().min())
+        top_unpicked, first_tie = 0.0, None
+        for a in range(off, off + d, chunk):
+            b = min(a + chunk, off + d)
+            inside = (idx >= a) & (idx < b)
+            sel = idx[inside] - a
+            want = prev[a:b] + lr_t * g[a:b]
+            want[sel] = 0.0
+            assert torch.equal(bits(res[a:b]), bits(want)), f"residual p={p} chunk {a}"
+            mag = want.abs()
+            mag[sel] = -1.0
+            top_unpicked = max(top_unpicked, float(mag.max()))
+            ties = torch.nonzero(mag == vmin)
+            if first_tie is None and ties.numel():
+                first_tie = a + int(ties[0])
+        assert vmin >= top_unpicked, f"p={p}: a picked magnitude is below an unpicked one"
+        if first_tie is not None:
+            assert first_tie > int(idx[val.abs() == vmin].max()), f"p={p}: tie order"
+    # dense update: the workers' picks added in worker order from +0, one
+    # rounding per add, then divided by P (positions nobody picked: +0)
+    picks = []
+    for p in range(run.P):
+        picks.append((run.idx[p * K + koff:p * K + koff + k].to(torch.int64) & 0xFFFFFFFF,
+                      run.val[p * K + koff:p * K + koff + k]))
+    fP = torch.tensor(float(run.P), dtype=torch.float32, device="cuda")
+    for a in range(off, off + d, chunk):
+        b = min(a + chunk, off + d)
+        acc = torch.zeros(b - a, dtype=torch.float32, device="cuda")
+        for idx, val in picks:
+            inside = (idx >= a) & (idx < b)
+            sel = idx[inside] - a
+            acc[sel] = acc[sel] + val[inside]
+        assert torch.equal(bits(run.dense[a:b]), bits(acc / fP)), f"dense chunk {a}"

@@ -46,6 +46,27 @@ def test_global_topk_one_segment(name, P, steps, max_fallbacks):
         assert np.array_equal(_u32(run.weights), e_w.view(np.uint32))
 
 
+def test_global_topk_1_3b_one_segment():
+    """SLGS on the 1.3B transformer: one segment of 1,311,178,752 elements
+    (k = 1,311,179), two workers, two steps, checked in chunks against the
+    properties that fix the selection and the worker-ordered dense update."""
+    import torch
+    from gpu_harness import GpuRun, check_layer_chunked
+    w = WORKLOADS["gpt_1_3b"]
+    P = 2
+    run = GpuRun([w.N], [0.001], P, w.lr, keep_prev=True)
+    assert run.plan.K == 1_311_179
+    for s in range(2):
+        for p in range(P):
+            synth.worker_grads_device(w, p, s, run.grads[p])
+        run.step(fused=s == 1)
+        flags, _ = run.plan.poll()
+        assert flags == 0
+        check_layer_chunked(run, 0, w.lr)
+    del run
+    torch.cuda.empty_cache()
+
+
 def test_step_captured_in_cuda_graph():
     """The calls only enqueue kernels (no allocation, no synchronisation), so a
     step can be captured; replays give the eager results bit for bit."""
