@@ -70,12 +70,13 @@ struct SelectShared {
   uint32_t tpre[kSelectWindow + 1];
   uint32_t tmp[NT + NT / 32 + 4];
   uint32_t xch[4];               // read by the other CTAs of the cluster
+  uint32_t split[2];             // first tiles of this CTA's and the next CTA's share
 };
 
 }  // namespace
 
 template <int CL, int NT>
-__global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const uint32_t* list,
+__global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, WorkerPtrs wp, const uint32_t* list,
                                                uint32_t stage_cap,
                                                uint32_t* __restrict__ out_idx,
                                                float* __restrict__ out_val) {
@@ -104,32 +105,89 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
 
   // ---- mode: candidate lists or exhaustive ----
   const uint32_t nt = ld.tile_end - ld.tile_begin;
-  const uint32_t ta = ld.tile_begin + (uint32_t)((uint64_t)nt * rank / CL);
-  const uint32_t tb = ld.tile_begin + (uint32_t)((uint64_t)nt * (rank + 1) / CL);
+  // this CTA's share of the segment: equal tile ranges (see below for the
+  // candidate-balanced split a crowded segment gets)
+  uint32_t ta = ld.tile_begin + (uint32_t)((uint64_t)nt * rank / CL);
+  uint32_t tb = ld.tile_begin + (uint32_t)((uint64_t)nt * (rank + 1) / CL);
   const uint32_t cap = ld.slot_cap;
   const uint32_t* cnt = dp.tile_cnt + (size_t)p * dp.T;
-  uint32_t my = 0, ovf = 0;
+  uint32_t my = 0, ovf = 0, pad = 0;
   for (uint32_t t = ta + tid; t < tb; t += NT) {
     const uint32_t c = __ldg(cnt + t);
     my += c;
     ovf |= c > cap;
+    pad += (c + 3u) & ~3u;
   }
   my = block_sum<NT>(my, sh.tmp);
   ovf = block_sum<NT>(ovf, sh.tmp);
+  pad = block_sum<NT>(pad, sh.tmp);
+  // A tile whose candidates overflowed its slots is still usable when this
+  // CTA stages its share: the CTA then recompacts that tile's candidates from
+  // its acc (held in the residual buffer) instead of copying the slots.  Only
+  // an overflow in a share that cannot be staged forces the exhaustive path.
+  const uint32_t lo_key = dp.lo_key[(size_t)p * dp.L + layer];
+  const bool stageable = tb - ta <= kSelectWindow && lo_key >= (1u << 20) && pad <= stage_cap;
   if (tid == 0) {
     sh.xch[0] = my;
-    sh.xch[1] = ovf;
+    sh.xch[1] = ovf && !stageable;
   }
   C::sync();  // also publishes the zeroed histograms cluster-wide
   uint64_t total = 0;
-  uint32_t any_ovf = 0;
+  uint32_t any_bad = 0;
 #pragma unroll
   for (int q = 0; q < CL; ++q) {
     const uint32_t* x = C::remote(sh.xch, q);
     total += x[0];
-    any_ovf |= x[1];
+    any_bad |= x[1];
   }
-  const bool fast = !any_ovf && total >= ld.k;
+  bool fast = !any_bad && total >= ld.k;
+  if constexpr (CL > 1) {
+    if (any_bad && total >= ld.k) {  // cluster-uniform: every CTA read the same words
+      // A crowded segment (its large values gather in a few tiles, as in a
+      // global top-k over tensors of different scales) overflows one CTA's
+      // stage under equal tile shares.  Split it again so that every CTA
+      // holds about the same number of (padded) candidates: CTA r takes the
+      // tiles whose candidate prefix lies in [total r / CL, total (r+1) / CL).
+      // The shares stay contiguous and in index order.
+      uint32_t ptot = 0;
+      for (uint32_t t = ld.tile_begin + tid; t < ld.tile_end; t += NT)
+        ptot += (__ldg(cnt + t) + 3u) & ~3u;
+      ptot = block_sum<NT>(ptot, sh.tmp);
+      const uint64_t lo_t = (uint64_t)ptot * rank / CL, hi_t = (uint64_t)ptot * (rank + 1) / CL;
+      if (tid < 2) sh.split[tid] = ld.tile_end;
+      uint64_t run = 0;  // candidates before the window
+      for (uint32_t w0 = ld.tile_begin; w0 < ld.tile_end; w0 += NT) {
+        const uint32_t t = w0 + tid;
+        const uint32_t c = t < ld.tile_end ? (__ldg(cnt + t) + 3u) & ~3u : 0u;
+        uint32_t wtot;
+        const uint64_t pre = run + block_excl_scan<NT>(c, sh.tmp, &wtot);
+        if (t < ld.tile_end && pre >= lo_t) atomicMin(&sh.split[0], t);
+        if (t < ld.tile_end && pre >= hi_t) atomicMin(&sh.split[1], t);
+        run += wtot;
+      }
+      __syncthreads();
+      ta = rank == 0 ? ld.tile_begin : sh.split[0];
+      tb = rank == CL - 1 ? ld.tile_end : sh.split[1];
+      ovf = 0;
+      pad = 0;
+      for (uint32_t t = ta + tid; t < tb; t += NT) {
+        const uint32_t c = __ldg(cnt + t);
+        ovf |= c > cap;
+        pad += (c + 3u) & ~3u;
+      }
+      ovf = block_sum<NT>(ovf, sh.tmp);
+      pad = block_sum<NT>(pad, sh.tmp);
+      const bool stageable2 =
+          tb - ta <= kSelectWindow && lo_key >= (1u << 20) && pad <= stage_cap;
+      C::sync();  // every CTA has read the first exchange
+      if (tid == 0) sh.xch[1] = ovf && !stageable2;
+      C::sync();
+      any_bad = 0;
+#pragma unroll
+      for (int q = 0; q < CL; ++q) any_bad |= C::remote(sh.xch, q)[1];
+      fast = !any_bad;
+    }
+  }
   if (!fast && rank == 0 && tid == 0) atomicAdd(dp.status + kStatusFallbacks, 1u);
 
   const uint32_t ea = ld.off + (uint32_t)((uint64_t)ld.d * rank / CL);
@@ -193,16 +251,18 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   // a pick, a tie or the bin holding the k-th largest key.
   bool staged = false, stage_timeout = false;
   uint32_t my_pad = 0;  // staged entries, padding included
-  const uint32_t lo_key = dp.lo_key[(size_t)p * dp.L + layer];
   if (fast && tb - ta <= kSelectWindow && lo_key >= (1u << 20)) {
     const uint32_t nw = tb - ta;
     constexpr int PER = kSelectWindow / NT;
-    uint32_t c[PER], sum = 0;
+    uint32_t c[PER], sum = 0, bulk = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const uint32_t q = tid * PER + i;
-      c[i] = q < nw ? (__ldg(cnt + ta + q) + 3u) & ~3u : 0u;
+      const uint32_t raw = q < nw ? __ldg(cnt + ta + q) : 0u;
+      c[i] = (raw + 3u) & ~3u;
       sum += c[i];
+      // entries the bulk copies bring: every run except an overflowed tile's
+      if (raw <= cap) bulk += c[i];
     }
     uint32_t ex = block_excl_scan<NT>(sum, sh.tmp, &my_pad);
 #pragma unroll
@@ -211,21 +271,50 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
       if (q < nw) sh.tpre[q] = ex;
       ex += c[i];
     }
-    staged = my_pad <= stage_cap;  // block-uniform
+    staged = my_pad <= stage_cap;  // block-uniform (== stageable)
+    bulk = block_sum<NT>(bulk, sh.tmp);  // (from this thread's own counts, not tpre)
     if (tid == 0) {
       sh.tpre[nw] = my_pad;
       mbar_init(&stage_bar, 1);
       mbar_init_fence();
-      if (staged) mbar_arrive_expect_tx(&stage_bar, my_pad * 8u);  // before any copy
+      if (staged) mbar_arrive_expect_tx(&stage_bar, bulk * 8u);  // before any copy
     }
     __syncthreads();
     if (staged) {
       for (uint32_t q = tid; q < nw; q += NT) {
         const uint32_t n = sh.tpre[q + 1] - sh.tpre[q];
-        if (n == 0) continue;
+        if (n == 0 || __ldg(cnt + ta + q) > cap) continue;
         const uint64_t slot = cbase + (uint64_t)(ta + q - ld.tile_begin) * cap;
         bulk_load(stage_val + sh.tpre[q], dp.cand_val + slot, n * 4u, &stage_bar);
         bulk_load(stage_idx + sh.tpre[q], dp.cand_idx + slot, n * 4u, &stage_bar);
+      }
+      if (ovf) {
+        // overflowed tiles: the CTA recompacts the entries with key >= lo_key
+        // from the tile's acc, in index order (each thread a contiguous run)
+        constexpr uint32_t PT = kTile / NT;
+        for (uint32_t q = 0; q < nw; ++q) {
+          const uint32_t n = __ldg(cnt + ta + q);  // block-uniform
+          if (n <= cap) continue;
+          const TileDesc tq = dp.tiles[ta + q];
+          const uint32_t e0 = tq.start + tid * PT;
+          const uint32_t mine = tid * PT < tq.len ? min(PT, tq.len - tid * PT) : 0u;
+          uint32_t c = 0;
+          for (uint32_t j = 0; j < mine; ++j) c += mag_key(r[e0 + j]) >= lo_key;
+          uint32_t found;
+          uint32_t at = block_excl_scan<NT>(c, sh.tmp, &found);
+          const uint32_t room = sh.tpre[q + 1] - sh.tpre[q];
+          if (tid == 0 && found != n) atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
+          for (uint32_t j = 0; j < mine; ++j) {  // (the run is in L1 from the count)
+            const float x = r[e0 + j];
+            if (mag_key(x) >= lo_key) {
+              if (at < room) {
+                stage_val[sh.tpre[q] + at] = x;
+                stage_idx[sh.tpre[q] + at] = e0 + j;
+              }
+              ++at;
+            }
+          }
+        }
       }
       const bool ok = mbar_wait_bounded(&stage_bar, 0, kSelectSpinLimit);
       if (__syncthreads_or(!ok)) {
@@ -251,15 +340,17 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
   // Unstaged shares: every pass walks the candidates (or, on the exhaustive
   // path, the layer's acc) from global memory.
   auto traverse = [&](auto&& fn) {
-    if (fast) {
-      stream_candidates([&](bool valid, uint32_t, uint32_t idx, float val) { fn(valid, idx, val); });
-    } else {
-      for (uint32_t b = ea; b < eb; b += NT) {
-        const uint32_t e = b + tid;
-        const bool valid = e < eb;
-        const float val = valid ? r[e] : 0.f;
-        fn(valid, e, val);
-      }
+    stream_candidates([&](bool valid, uint32_t, uint32_t idx, float val) { fn(valid, idx, val); });
+  };
+  // Exhaustive path: the CTA's element share [ea, eb) of the layer's acc, in
+  // rounds of NT * kExhV elements; each thread takes kExhV consecutive
+  // elements per round (index order = thread order within a round).
+  constexpr uint32_t kExhV = 4;
+  auto exh_load = [&](uint32_t base, float (&v)[kExhV]) {
+#pragma unroll
+    for (uint32_t j = 0; j < kExhV; ++j) {
+      const uint32_t e = base + tid * kExhV + j;
+      v[j] = e < eb ? r[e] : 0.f;
     }
   };
 
@@ -281,17 +372,28 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
         if (mshift >= 32 || (key >> mshift) == mval)
           atomicAdd(&sh.hist[(key >> dshift) & dmask], 1u);
       }
-    } else traverse([&](bool valid, uint32_t, float val) {
-      const uint32_t key = mag_key(val);
-      const bool m = valid && (mshift >= 32 || (key >> mshift) == mval);
-      const uint32_t dig = m ? ((key >> dshift) & dmask) : 0xFFFFFFFFu;
-      if (fast) {  // candidates sit in the sparse tail: few collisions
-        if (m) atomicAdd(&sh.hist[dig], 1u);
-      } else {     // a whole layer: keys crowd into few bins, add once per warp and bin
-        const unsigned peers = __match_any_sync(kFull, dig);
-        if (m && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
+    } else if (fast) {
+      traverse([&](bool valid, uint32_t, float val) {
+        // candidates sit in the sparse tail: few collisions
+        const uint32_t key = mag_key(val);
+        if (valid && (mshift >= 32 || (key >> mshift) == mval))
+          atomicAdd(&sh.hist[(key >> dshift) & dmask], 1u);
+      });
+    } else {
+      // a whole layer: keys crowd into few bins, add once per warp and bin
+      for (uint32_t base = ea; base < eb; base += NT * kExhV) {
+        float v[kExhV];
+        exh_load(base, v);
+#pragma unroll
+        for (uint32_t j = 0; j < kExhV; ++j) {
+          const uint32_t key = mag_key(v[j]);
+          const bool m = base + tid * kExhV + j < eb && (mshift >= 32 || (key >> mshift) == mval);
+          const uint32_t dig = m ? ((key >> dshift) & dmask) : 0xFFFFFFFFu;
+          const unsigned peers = __match_any_sync(kFull, dig);
+          if (m && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
+        }
       }
-    });
+    }
     __syncthreads();
     if constexpr (CL > 1) {
       uint32_t* dst = C::remote(merged[level], 0);
@@ -364,12 +466,26 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
     na = tot >> 16;
     nb = tot & 0xFFFFu;
     __syncthreads();
-  } else {
+  } else if (fast) {
     traverse([&](bool valid, uint32_t, float val) {
       const uint32_t s = mag_key(val) >> fshift;
       na += valid && s > fpfx;
       nb += valid && s == fpfx;
     });
+    na = block_sum<NT>(na, sh.tmp);
+    nb = block_sum<NT>(nb, sh.tmp);
+  } else {
+    for (uint32_t base = ea; base < eb; base += NT * kExhV) {
+      float v[kExhV];
+      exh_load(base, v);
+#pragma unroll
+      for (uint32_t j = 0; j < kExhV; ++j) {
+        const bool valid = base + tid * kExhV + j < eb;
+        const uint32_t s = mag_key(v[j]) >> fshift;
+        na += valid && s > fpfx;
+        nb += valid && s == fpfx;
+      }
+    }
     na = block_sum<NT>(na, sh.tmp);
     nb = block_sum<NT>(nb, sh.tmp);
   }
@@ -425,7 +541,7 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
       const uint32_t x = __float_as_uint(stage_val[i]);
       if (x != 0xFFFFFFFFu) r[x] = 0.0f;
     }
-  } else {
+  } else if (fast) {
     traverse([&](bool valid, uint32_t idx, float val) {
       const uint32_t s = mag_key(val) >> fshift;
       const bool st = valid && s > fpfx;
@@ -438,6 +554,43 @@ __global__ void __launch_bounds__(NT) k_select(DevPlan dp, WorkerPtrs wp, const 
       a_run += tot >> 16;
       b_run += tot & 0xFFFFu;
     });
+  } else {
+    // one block scan per round of NT * kExhV elements (< 2^16, so strict and
+    // tie counts pack into one word); the next round's loads are issued
+    // before this round's stores, which would otherwise hold them back
+    float v[kExhV];
+    exh_load(ea, v);
+    for (uint32_t base = ea; base < eb; base += NT * kExhV) {
+      float nv[kExhV];
+      exh_load(base + NT * kExhV, nv);
+      uint32_t cst = 0, cti = 0;
+#pragma unroll
+      for (uint32_t j = 0; j < kExhV; ++j) {
+        const bool valid = base + tid * kExhV + j < eb;
+        const uint32_t s = mag_key(v[j]) >> fshift;
+        cst += valid && s > fpfx;
+        cti += valid && s == fpfx;
+      }
+      uint32_t tot;
+      const uint32_t ex = block_excl_scan<NT>((cst << 16) | cti, sh.tmp, &tot);
+      uint32_t at = a_run + (ex >> 16), bt = b_run + (ex & 0xFFFFu);
+#pragma unroll
+      for (uint32_t j = 0; j < kExhV; ++j) {
+        const uint32_t e = base + tid * kExhV + j;
+        const uint32_t s = mag_key(v[j]) >> fshift;
+        if (e < eb && s > fpfx) {
+          emit(at + min(need, bt), e, v[j], true);
+          ++at;
+        } else if (e < eb && s == fpfx) {
+          if (bt < need) emit(at + bt, e, v[j], true);
+          ++bt;
+        }
+      }
+      a_run += tot >> 16;
+      b_run += tot & 0xFFFFu;
+#pragma unroll
+      for (uint32_t j = 0; j < kExhV; ++j) v[j] = nv[j];
+    }
   }
   if (stage_timeout && tid == 0)  // give copies still in flight a bounded chance to land
     mbar_wait_bounded(&stage_bar, 0, kSelectSpinLimit);

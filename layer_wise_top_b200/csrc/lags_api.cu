@@ -176,7 +176,7 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
   }
   // staging capacity of each select launch: 1.5x the largest expected
   // candidate count of one CTA (the sample rank scaled to the layer) plus 512
-  auto stage_for = [plan](const std::vector<uint32_t>& list, uint32_t ctas) {
+  auto stage_for = [plan, num_workers](const std::vector<uint32_t>& list, uint32_t ctas) {
     double most = 0.0;
     for (uint32_t l : list) {
       const LayerDesc& ld = plan->layers[l];
@@ -185,6 +185,10 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
       most = std::max(most, 1.5 * expected_candidates(ld) / ctas + 3.0 * tiles);
     }
     uint64_t cap = ((uint64_t)std::ceil(most + 512.0) + 255) / 256 * 256;
+    // a launch whose CTAs all run at once with one per SM (148 SMs) gives each
+    // the largest stage at no cost: crowded segments (a global top-k over
+    // tensors of different scales) then stay on the candidate lists
+    if ((uint64_t)list.size() * ctas * (uint64_t)num_workers <= 148) cap = kSelectStageMax;
     return (uint32_t)std::min<uint64_t>(std::max<uint64_t>(cap, kSelectStageMin), kSelectStageMax);
   };
   // aggregation: a tile of a sparse layer is expected to hold P * k * kTile / d
