@@ -2,9 +2,15 @@
 //
 // Before the fused pass streams a layer, one CTA per sparse (worker, layer)
 // draws a sample of m_l entries of acc = residual + lr*grad (the whole layer
-// when it is at most kSampleMax long, otherwise 256 runs of 64 contiguous
-// entries, one at a hashed offset inside each of 256 equal strata) and finds the magnitude key of the sample's r*-th
-// largest entry, rounded down to a level-1 radix bin edge.  The fused pass
+// when it is at most kSampleMax long, otherwise runs of contiguous entries,
+// one at a hashed offset inside each of m_l / run equal strata) and finds the
+// magnitude key of the sample's r*-th largest entry, rounded down to a
+// level-1 radix bin edge.  Segments longer than kSampleShortAbove use runs of
+// 16 (1024 strata): such a segment may span tensors of different scales, and
+// a run must not stand for a whole stratum of differently scaled values.
+// With 64-entry runs, one run inside the 1,728-entry first layer of VGG-16 set
+// the threshold of a global top-k over the model above its 14,720th value.
+// Shorter segments keep runs of 64, which measured faster there.  The fused pass
 // then keeps every entry at or above that key as a candidate.  r* is chosen on
 // the host so that, for a sample drawn from the layer, the candidates hold the
 // layer's k largest entries with overwhelming probability; when they do not
@@ -29,7 +35,7 @@ __device__ __forceinline__ uint32_t mix32(uint32_t x) {
 __global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs wp, float lr) {
   extern __shared__ uint32_t s_keys[];  // kSampleMax
   __shared__ uint32_t s_hist[kBins];
-  __shared__ uint32_t s_chunk[kSampleMax / kSampleChunk];  // first element of each run
+  __shared__ uint32_t s_chunk[kSampleMax / kSampleRunShort];  // first element of each run
   __shared__ uint32_t s_tmp[kEstThreads + kEstThreads / 32 + 4];
 
   pdl_trigger();
@@ -39,11 +45,14 @@ __global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs
   const float* __restrict__ g = wp.g[p];
   const float* __restrict__ r = wp.r[p];
   const uint32_t m = ld.sample;
-  const uint32_t nchunk = m / kSampleChunk;
+  const uint32_t run = ld.d > kSampleShortAbove ? kSampleRunShort : kSampleRunLong;
+  const uint32_t run_shift = run == kSampleRunShort ? 4 : 6;  // log2(run)
+  static_assert(kSampleRunShort == 16 && kSampleRunLong == 64, "run_shift");
+  const uint32_t nchunk = m >> run_shift;
   pdl_wait();
 
   for (uint32_t i = threadIdx.x; i < kBins; i += kEstThreads) s_hist[i] = 0;
-  // sample positions: the whole layer, or nchunk runs of kSampleChunk spread
+  // sample positions: the whole layer, or nchunk runs of `run` entries spread
   // evenly over it
   if (m != ld.d)
     for (uint32_t c = threadIdx.x; c < nchunk; c += kEstThreads) {
@@ -51,7 +60,7 @@ __global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs
       // equal strata, so every region of the layer is sampled in proportion
       const uint32_t a = (uint32_t)((uint64_t)c * ld.d / nchunk);
       const uint32_t b = (uint32_t)((uint64_t)(c + 1) * ld.d / nchunk);
-      s_chunk[c] = ld.off + a + mix32(c * 0x9E3779B9u + layer) % (b - a - kSampleChunk + 1);
+      s_chunk[c] = ld.off + a + mix32(c * 0x9E3779B9u + layer) % (b - a - run + 1);
     }
   __syncthreads();
   constexpr uint32_t U = 8;  // loads per array in flight per thread
@@ -63,7 +72,7 @@ __global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs
       gv[u] = 0.f;
       rv[u] = 0.f;
       if (i < m) {
-        const uint32_t e = m == ld.d ? ld.off + i : s_chunk[i / kSampleChunk] + i % kSampleChunk;
+        const uint32_t e = m == ld.d ? ld.off + i : s_chunk[i >> run_shift] + (i & (run - 1));
         gv[u] = __ldg(g + e);
         rv[u] = __ldg(r + e);
       }

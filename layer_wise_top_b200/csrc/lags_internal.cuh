@@ -20,7 +20,12 @@ constexpr uint32_t kEfVecPerThread = kTile / 4 / kEfThreads;  // float4 per thre
 
 // Largest sample the threshold estimate draws per (worker, layer).
 constexpr uint32_t kSampleMax = 16384;
-constexpr uint32_t kSampleChunk = 64;  // contiguous elements per sample chunk
+// contiguous elements per sample run: short runs for segments longer than
+// kSampleShortAbove (whole-model segments span tensors of different scales),
+// long runs (fewer, larger reads) for the rest
+constexpr uint32_t kSampleRunShort = 16;
+constexpr uint32_t kSampleRunLong = 64;
+constexpr uint32_t kSampleShortAbove = 1u << 23;
 constexpr uint32_t kEstThreads = 512;
 
 // Cluster size used to select layers whose expected candidates exceed what one
