@@ -120,13 +120,14 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   }
   my = block_sum<NT>(my, sh.tmp);
   ovf = block_sum<NT>(ovf, sh.tmp);
-  pad = block_sum<NT>(pad, sh.tmp);
+  if (ovf) pad = block_sum<NT>(pad, sh.tmp);  // (block-uniform; only needed then)
   // A tile whose candidates overflowed its slots is still usable when this
   // CTA stages its share: the CTA then recompacts that tile's candidates from
   // its acc (held in the residual buffer) instead of copying the slots.  Only
   // an overflow in a share that cannot be staged forces the exhaustive path.
   const uint32_t lo_key = dp.lo_key[(size_t)p * dp.L + layer];
-  const bool stageable = tb - ta <= kSelectWindow && lo_key >= (1u << 20) && pad <= stage_cap;
+  const bool stageable =
+      ovf && tb - ta <= kSelectWindow && lo_key >= (1u << 20) && pad <= stage_cap;
   if (tid == 0) {
     sh.xch[0] = my;
     sh.xch[1] = ovf && !stageable;
