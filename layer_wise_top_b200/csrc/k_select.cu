@@ -2,15 +2,23 @@
 //
 // One thread-block cluster of CL CTAs per sparse (worker, layer); each CTA owns
 // a contiguous, index-ordered share of the layer.  The CTAs count the layer's
-// candidates; if the sampled threshold held (at least k_l candidates and no
-// tile overflowed its slots) they work on the candidate lists, otherwise on
-// the full acc of the layer (held in the residual buffer after the fused
-// pass).  Either way the result is the exact top-k of the layer.  CL is 1, 8
-// or (for layers whose candidates need more shared memory than 8 CTAs hold)
-// 16, a non-portable cluster size used only where the occupancy query says it
-// fits.  A CTA whose candidates fit in shared memory stages them there with
-// plain bulk copies (cp.async.bulk, one per tile and array, completing on one
-// mbarrier); every pass below then reads shared memory only.
+// candidates; if the sampled threshold held (at least k_l candidates, and
+// every tile that overflowed its slots lies in a share that can be staged)
+// they work on the candidate lists, otherwise on the full acc of the layer
+// (held in the residual buffer after the fused pass).  Either way the result
+// is the exact top-k of the layer.
+//
+// CL is 1, 8, or 16. 16 is used for layers whose candidates need more shared
+// memory than 8 CTAs hold, and it is a non-portable cluster size used only
+// where the occupancy query says it fits.  Shares are equal tile ranges; a
+// crowded clustered segment (overflow that equal shares cannot stage) is
+// split again into shares of equal candidate counts.
+//
+// A CTA whose candidates fit in shared memory stages them there, with plain
+// bulk copies (cp.async.bulk, one per tile and array, completing on one
+// mbarrier).  An overflowed tile is instead recompacted from its acc by the
+// whole CTA.  Every pass below then reads shared memory only.  The exhaustive
+// path walks the acc in rounds of 4 consecutive entries per thread.
 //
 //  1. radix select on the magnitude key (bits 30..20, 19..9, 8..0): every CTA
 //     builds a shared-memory histogram of its share (warp-aggregated with
