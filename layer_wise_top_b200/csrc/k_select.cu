@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
       __syncthreads();
       for (uint32_t b = 0; b < wtotal; b += NT) {
         const uint32_t v = b + tid;
-        const bool valid = v < wtotal;
+        bool valid = v < wtotal;
         uint32_t idx = 0;
         float val = 0.f;
         if (valid) {
@@ -240,10 +240,17 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
             const uint32_t mid = (lo + hi + 1) >> 1;
             if (sh.tpre[mid] <= v) lo = mid; else hi = mid - 1;
           }
-          const uint64_t slot =
-              cbase + (uint64_t)(w0 + lo - ld.tile_begin) * cap + (v - sh.tpre[lo]);
-          idx = __ldg(dp.cand_idx + slot);
-          val = __ldg(dp.cand_val + slot);
+          const uint32_t in_tile = v - sh.tpre[lo];
+          if (in_tile < cap) {
+            const uint64_t slot = cbase + (uint64_t)(w0 + lo - ld.tile_begin) * cap + in_tile;
+            idx = __ldg(dp.cand_idx + slot);
+            val = __ldg(dp.cand_val + slot);
+          } else {
+            // an overflowed tile walked from its slots (only after a staging
+            // timeout): the slots end at cap, so report and skip the rest
+            atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
+            valid = false;
+          }
         }
         fn(valid, seen + v, idx, val);
       }
