@@ -3,7 +3,7 @@ checks it against the oracle and against full-size invariants (torch on the
 GPU as an independent checker).  Test infrastructure."""
 from __future__ import annotations
 
-from typing import Callable, Dict, Iterable, List, Optional, Sequence
+from typing import Callable, Iterable, List, Optional, Sequence
 
 import numpy as np
 import torch

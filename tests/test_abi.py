@@ -2,11 +2,9 @@
 include/lags.h declares, and plan creation validates and lays out correctly.
 No compute call is made here (no GPU)."""
 import ctypes
-import math
 import os
 import re
 
-import numpy as np
 import pytest
 
 import layer_wise_top_b200 as L

@@ -1,7 +1,6 @@
 """Adaptive per-layer densities (host planner in the C ABI) against the
 oracle's restatement, a hand-worked fixture, special cases and the
 "message hidden by the end of backward" property."""
-import math
 
 import numpy as np
 import pytest

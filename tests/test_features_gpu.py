@@ -6,7 +6,7 @@ import pytest
 
 import oracle.lags_oracle as lo
 import synth
-from synth.configs import WORKLOADS, Tensor
+from synth.configs import WORKLOADS
 
 pytestmark = pytest.mark.gpu
 

@@ -6,7 +6,6 @@ top-k: picks ascending and inside the layer, each value equal to acc at its
 index, picked residuals +0 and all others acc, every picked magnitude at
 least every unpicked one, ties to the lower index, and the dense update equal
 to the picks (P = 1) and +0 elsewhere.  About 105 GB of device memory."""
-import numpy as np
 import pytest
 
 import synth

@@ -1,7 +1,6 @@
 """Merged-message planner (reading R9): the C planner and the oracle's
 dynamic program against a hand-worked fixture, brute force over every cut of
 small models, and the special cases the timing model fixes."""
-import itertools
 
 import numpy as np
 import pytest

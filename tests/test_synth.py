@@ -4,7 +4,6 @@ import numpy as np
 import pytest
 
 import synth
-from conftest import read_golden
 from synth.configs import WORKLOADS
 
 
