@@ -35,6 +35,10 @@ METRIC = "LAGS sparsify+aggregate Gelem/s per step; achieved HBM GB/s vs peak"
 # the elements, so its traffic grows in proportion).
 EF_TRAFFIC_BYTES = 1_885_774_000 + 895_709_696
 EF_TRAFFIC_ELEMENTS = 235_517_088
+# DRAM bytes of one k_dense_sum launch (profiles/k_dense_sum_vgg16.md, VGG-16
+# shapes, 16 workers); other workloads scale it by their element count.
+DENSE_TRAFFIC_BYTES = 942_080_512 + 12_375_808
+DENSE_TRAFFIC_ELEMENTS = 235_517_088
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 POOL_BUDGET_BYTES = 48 * 1024 ** 3
@@ -324,7 +328,11 @@ def run_dense(args):
             l2=f"inputs larger than L2: {4 * P * N / 1e9:.2f} GB read per step"),
         "roofline": {"kernel": "k_dense_sum", "bound": "hbm", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak,
+                     "traffic": DENSE_TRAFFIC_BYTES * (P * N) / DENSE_TRAFFIC_ELEMENTS,
+                     "traffic_source": ("ncu capture of this workload" if P * N ==
+                                        DENSE_TRAFFIC_ELEMENTS else
+                                        "ncu capture of the VGG-16 shapes, scaled by elements"),
                      "algorithmic_bytes_per_launch": sum_bytes, "avg_launch_ms": sum_ms,
                      "share_of_step": sum_ms / (ms_max / K)},
         "cpu_baseline": None, "e2e": None, "gpu_launches": 2 * K, "clocks": clk,
