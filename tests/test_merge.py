@@ -92,3 +92,13 @@ def test_rejects_bad_arguments():
         L.lags_merge_layers([1, -1], [0.0, 0.0], 0.0, 0.0)
     with pytest.raises(L.LagsError):
         L.lags_merge_layers([1], [0.0], -1.0, 0.0)
+
+
+def test_check_buckets_accepts_only_ordered_partitions():
+    from layer_wise_top_b200.dist import check_buckets
+    check_buckets([(0, 2), (2, 3), (3, 7)], 7)
+    check_buckets(L.lags_merge_layers([8] * 5, [1e-3] * 5, 1e-5, 1e-9)[0], 5)
+    for bad in ([(0, 2), (3, 7)], [(0, 2), (2, 2), (2, 7)], [(1, 7)], [(0, 6)],
+                [(0, 4), (2, 7)]):
+        with pytest.raises(ValueError):
+            check_buckets(bad, 7)
