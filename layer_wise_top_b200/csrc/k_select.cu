@@ -555,7 +555,9 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
     __syncwarp();
     for (uint32_t i = wb + lane; i < we; i += 32) {
       const uint32_t x = __float_as_uint(stage_val[i]);
-      if (x != 0xFFFFFFFFu) r[x] = 0.0f;
+      if (x == 0xFFFFFFFFu) continue;
+      if (x - ld.off < ld.d) r[x] = 0.0f;  // an emitted index lies in the layer
+      else atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
     }
   } else if (fast) {
     traverse([&](bool valid, uint32_t idx, float val) {
