@@ -62,7 +62,10 @@ typedef enum {
   LAGS_ERR_CUDA = 3,               /* a CUDA runtime call or launch failed */
   LAGS_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not sm_100 (B200) */
   LAGS_ERR_WORKSPACE = 5,          /* workspace missing or smaller than required */
-  LAGS_ERR_BAD_PICKS = 6           /* (status word) pick lists not ascending/in layer */
+  LAGS_ERR_BAD_PICKS = 6,          /* (status word) pick lists not ascending/in layer */
+  LAGS_ERR_TIMEOUT = 7,            /* (status word) a kernel's bounded wait gave up */
+  LAGS_ERR_INTERNAL = 8,           /* (status word) a kernel failed a self-check */
+  LAGS_ERR_WRONG_DEVICE = 9        /* the current device is not the plan's */
 } lags_status;
 
 /* Largest number of simulated workers one plan accepts. */
@@ -75,8 +78,9 @@ typedef enum {
 
 /* Bits of the device status word returned by lags_status_poll(). */
 #define LAGS_FLAG_BAD_PICKS 0x1u /* lags_aggregate saw an unsorted or out-of-layer index */
-#define LAGS_FLAG_TIMEOUT 0x4u   /* a kernel's bounded wait on its own bulk copies gave up;
-                                    the outputs of that call are incomplete */
+#define LAGS_FLAG_TIMEOUT 0x4u   /* the selection's bounded wait on its own bulk copies gave
+                                    up; the selection then read its candidates from global
+                                    memory, and its picks may be incomplete */
 #define LAGS_FLAG_INTERNAL 0x2u  /* a selection kernel failed a self-check (a library bug);
                                     the write it guarded was skipped */
 
@@ -132,6 +136,16 @@ LAGS_API lags_status lags_plan_info(const lags_plan* plan, int64_t* N, int64_t* 
                            size_t* workspace_bytes);
 
 /*
+ * lags_plan_aggregate_workspace_bytes - the smaller workspace that serves a
+ * plan used only to aggregate (lags_aggregate, lags_aggregate_apply,
+ * lags_status_poll), e.g. the job-wide plan of a data-parallel rank that
+ * sparsifies its own workers with another plan.  It leaves out the selection's
+ * candidate slots, most of the full workspace.  Host only.
+ *   bytes  host, receives the size (<= workspace_bytes of lags_plan_info).
+ */
+LAGS_API lags_status lags_plan_aggregate_workspace_bytes(const lags_plan* plan, size_t* bytes);
+
+/*
  * lags_plan_layer - placement of layer l: its first element in a worker buffer
  * (offset), its pick count k_l and the first slot of its picks in a worker's
  * pick list (pick_offset).  Picks of layer l occupy
@@ -144,8 +158,12 @@ LAGS_API lags_status lags_plan_layer(const lags_plan* plan, int32_t l, int64_t* 
  * lags_plan_set_workspace - bind caller-owned device memory to the plan and
  * upload the plan's tables into it (enqueued on `stream`; the host tables are
  * owned by the plan, so nothing has to outlive the call on the caller side).
- *   workspace  device, 256-byte aligned, >= workspace_bytes of lags_plan_info.
- * Also checks that the current device is an sm_100 part.  Call it again after
+ *   workspace  device, 256-byte aligned, >= workspace_bytes of lags_plan_info
+ *              (full plan), or >= lags_plan_aggregate_workspace_bytes (the plan
+ *              then only aggregates: lags_sparsify returns LAGS_ERR_WORKSPACE).
+ * Also checks that the current device is an sm_100 part and makes it the
+ * plan's device: later calls on the plan return LAGS_ERR_WRONG_DEVICE, before
+ * enqueuing anything, when another device is current.  Call it again after
  * freeing or moving the workspace.  Not for use inside stream capture.
  */
 LAGS_API lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t bytes,
@@ -202,14 +220,17 @@ LAGS_API lags_status lags_apply(const lags_plan* plan, float* weights, const flo
 
 /*
  * lags_status_poll - synchronise `stream`, read and clear the plan's device
- * status word.
+ * status word.  The word collects the flags of every call on the plan since
+ * the last poll.
  *   flags              host, receives LAGS_FLAG_* bits (may be NULL)
  *   exact_fallbacks    host, receives how many (worker, layer) segments since
  *                      the last poll were selected by the exhaustive path
  *                      because the sampled candidate threshold did not hold
  *                      (results are exact either way; may be NULL)
- * Returns LAGS_ERR_BAD_PICKS if that flag was set, else LAGS_OK (or
- * LAGS_ERR_CUDA).
+ * Returns, when a flag is set: LAGS_ERR_TIMEOUT (LAGS_FLAG_TIMEOUT: picks may
+ * be incomplete), else LAGS_ERR_INTERNAL (LAGS_FLAG_INTERNAL: a library bug),
+ * else LAGS_ERR_BAD_PICKS; otherwise LAGS_OK.  The outputs are written in
+ * every case.  LAGS_ERR_CUDA if the copy fails.
  */
 LAGS_API lags_status lags_status_poll(lags_plan* plan, uint32_t* flags, uint32_t* exact_fallbacks,
                              void* stream);
@@ -228,13 +249,29 @@ LAGS_API lags_status lags_status_poll(lags_plan* plan, uint32_t* flags, uint32_t
  *   - All calls share the array, which keeps the last call's contents; each
  *     call uploads its plan's tables and clears what must start at zero.
  *     Calls whose work overlaps on the GPU race on it.
- *   - The first call on a device resolves the array's address there and
- *     configures the kernels: make it before any stream capture.
- *   - The status word it writes is not read by lags_status_poll.
+ *   - The first call on a device (of this function or of
+ *     lags_static_status_poll) resolves the array's address there and
+ *     configures the kernels.  Under CUDA's lazy module loading (the default)
+ *     that first call is also when the driver loads the array's code and
+ *     reserves its 16 MiB on the device, so make it at start-up: outside any
+ *     context that must not allocate, and before any stream capture.
+ *   - Its status words live in the same array, at a fixed place, and collect
+ *     the flags of every call on the device until lags_static_status_poll
+ *     reads and clears them (lags_status_poll does not see them).
  */
 LAGS_API lags_status lags_sparsify_static(lags_plan* plan, const float* const* grads,
                                           float* const* residuals, float lr, uint32_t* out_idx,
                                           float* out_val, void* stream);
+
+/*
+ * lags_static_status_poll - lags_status_poll for lags_sparsify_static: copy the
+ * status words of the static array of the current device into host memory
+ * (synchronising `stream`), then clear them.  Allocates nothing.
+ *   flags, exact_fallbacks   as lags_status_poll (either may be NULL).
+ * Returns as lags_status_poll.
+ */
+LAGS_API lags_status lags_static_status_poll(uint32_t* flags, uint32_t* exact_fallbacks,
+                                             void* stream);
 
 /*
  * lags_plan_set_events - timing instrumentation.  When `before` and `after`
@@ -247,6 +284,20 @@ LAGS_API lags_status lags_sparsify_static(lags_plan* plan, const float* const* g
  * graph records them again.
  */
 LAGS_API lags_status lags_plan_set_events(lags_plan* plan, void* before, void* after);
+
+/*
+ * lags_plan_set_stage_wait_limit - failure-injection knob for tests of the
+ * timeout path.  The selection kernel stages a layer's candidates in shared
+ * memory with bulk copies and polls their completion barrier at most
+ * `polls` times (default LAGS_STAGE_WAIT_POLLS) before it gives up, sets
+ * LAGS_FLAG_TIMEOUT and selects from global memory instead; it then still
+ * waits (up to the default limit) for its copies before it exits.  0 makes
+ * every staged selection give up at once: the status poll then reports the
+ * timeout, while the picks of layers without overflowed candidate tiles stay
+ * exact.  Takes effect from the next lags_sparsify on the plan.
+ */
+#define LAGS_STAGE_WAIT_POLLS 4194304u
+LAGS_API lags_status lags_plan_set_stage_wait_limit(lags_plan* plan, uint32_t polls);
 
 /*
  * lags_adaptive_densities - per-layer densities from each layer's

@@ -17,6 +17,10 @@ LAGS_ERR_CUDA = 3
 LAGS_ERR_UNSUPPORTED_DEVICE = 4
 LAGS_ERR_WORKSPACE = 5
 LAGS_ERR_BAD_PICKS = 6
+LAGS_ERR_TIMEOUT = 7
+LAGS_ERR_INTERNAL = 8
+LAGS_ERR_WRONG_DEVICE = 9
+LAGS_STAGE_WAIT_POLLS = 4194304
 LAGS_MAX_WORKERS = 256
 LAGS_MAX_ELEMENTS = (1 << 32) - 65536
 LAGS_FLAG_BAD_PICKS = 0x1
@@ -28,13 +32,20 @@ EXPORTED = ("lags_plan_create", "lags_plan_destroy", "lags_plan_info", "lags_pla
             "lags_status_poll", "lags_plan_set_events", "lags_sparsify_static",
             "lags_aggregate_apply", "lags_plan_kernel_launches", "lags_adaptive_densities",
             "lags_plan_create_range", "lags_merge_layers", "lags_dense_sum",
-            "lags_dense_finish", "lags_error_string")
+            "lags_dense_finish", "lags_plan_aggregate_workspace_bytes",
+            "lags_plan_set_stage_wait_limit", "lags_static_status_poll", "lags_error_string")
 
 
 class LagsError(RuntimeError):
-    def __init__(self, status: int, where: str):
+    """A non-OK lags_status.  A status poll that fails also carries the
+    flags and exhaustive-path count it read."""
+
+    def __init__(self, status: int, where: str, flags: int = 0, fallbacks: int = 0):
         self.status = status
-        super().__init__(f"{where}: {lags_error_string(status)} (status {status})")
+        self.flags = flags
+        self.fallbacks = fallbacks
+        extra = f", flags {flags:#x}" if flags else ""
+        super().__init__(f"{where}: {lags_error_string(status)} (status {status}{extra})")
 
 
 def _load() -> ctypes.CDLL:
@@ -73,6 +84,10 @@ def _load() -> ctypes.CDLL:
     lib.lags_plan_set_events.argtypes = [vp, vp, vp]
     lib.lags_sparsify_static.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp),
                                          ctypes.c_float, vp, vp, vp]
+    lib.lags_static_status_poll.argtypes = [ctypes.POINTER(ctypes.c_uint32),
+                                            ctypes.POINTER(ctypes.c_uint32), vp]
+    lib.lags_plan_aggregate_workspace_bytes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t)]
+    lib.lags_plan_set_stage_wait_limit.argtypes = [vp, ctypes.c_uint32]
     lib.lags_error_string.argtypes = [st]
     lib.lags_error_string.restype = ctypes.c_char_p
     for name in EXPORTED[:-1]:
@@ -132,6 +147,18 @@ def lags_plan_info(plan) -> Tuple[int, int, int]:
     _check(_LIB.lags_plan_info(plan, ctypes.byref(n), ctypes.byref(k), ctypes.byref(ws)),
            "lags_plan_info")
     return n.value, k.value, ws.value
+
+
+def lags_plan_aggregate_workspace_bytes(plan) -> int:
+    n = ctypes.c_size_t()
+    _check(_LIB.lags_plan_aggregate_workspace_bytes(plan, ctypes.byref(n)),
+           "lags_plan_aggregate_workspace_bytes")
+    return n.value
+
+
+def lags_plan_set_stage_wait_limit(plan, polls: int) -> None:
+    _check(_LIB.lags_plan_set_stage_wait_limit(plan, int(polls)),
+           "lags_plan_set_stage_wait_limit")
 
 
 def lags_plan_layer(plan, l: int) -> Tuple[int, int, int]:
@@ -246,9 +273,23 @@ def lags_plan_set_events(plan, before: int, after: int) -> None:
            "lags_plan_set_events")
 
 
-def lags_status_poll(plan, stream: int = 0) -> Tuple[int, int]:
-    """Returns (flags, exact_fallbacks); raises on LAGS_ERR_BAD_PICKS."""
-    f, fb = ctypes.c_uint32(), ctypes.c_uint32()
-    _check(_LIB.lags_status_poll(plan, ctypes.byref(f), ctypes.byref(fb),
-                                 ctypes.c_void_p(stream)), "lags_status_poll")
+def _poll_result(status: int, f, fb, where: str) -> Tuple[int, int]:
+    if status != LAGS_OK:
+        raise LagsError(status, where, f.value, fb.value)
     return f.value, fb.value
+
+
+def lags_status_poll(plan, stream: int = 0) -> Tuple[int, int]:
+    """Returns (flags, exact_fallbacks); raises LagsError (with .flags) when a
+    flag reports a timeout, a failed self-check or malformed pick lists."""
+    f, fb = ctypes.c_uint32(), ctypes.c_uint32()
+    st = _LIB.lags_status_poll(plan, ctypes.byref(f), ctypes.byref(fb), ctypes.c_void_p(stream))
+    return _poll_result(st, f, fb, "lags_status_poll")
+
+
+def lags_static_status_poll(stream: int = 0) -> Tuple[int, int]:
+    """lags_status_poll for lags_sparsify_static (the current device's static
+    status words)."""
+    f, fb = ctypes.c_uint32(), ctypes.c_uint32()
+    st = _LIB.lags_static_status_poll(ctypes.byref(f), ctypes.byref(fb), ctypes.c_void_p(stream))
+    return _poll_result(st, f, fb, "lags_static_status_poll")

@@ -15,7 +15,6 @@
 //    pick list and its residual becomes +0.
 #include "block_ops.cuh"
 #include "lags_internal.cuh"
-#include "tma.cuh"
 
 namespace lags {
 
@@ -171,229 +170,6 @@ __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, Worker
     }
   }
   if (threadIdx.x == 0) dp.tile_cnt[(size_t)p * dp.T + t] = s_total;
-}
-
-// ---------------------------------------------------------------------------
-// Bulk-copy streaming variant of the same pass: a persistent grid, one CTA of
-// kStreamThreads per SM, walks the (worker, tile) items.  One thread keeps
-// kStreamStages tiles of gradient and residual in flight with cp.async.bulk
-// into a shared-memory ring (completion tracked by one mbarrier per stage);
-// all threads then form acc from shared memory and store it to the residual
-// with 128-bit stores.  Results are identical to k_ef_capture.
-constexpr uint32_t kStreamThreads = 512;
-constexpr uint32_t kStreamStages = 3;
-constexpr uint32_t kStreamV = kTile / 4 / kStreamThreads;  // float4 per thread = 4
-constexpr uint32_t kSpinLimit = 1u << 22;                  // polls before giving up
-
-struct StreamShared {
-  float g[kStreamStages][kTile];
-  float r[kStreamStages][kTile];
-  uint64_t full[kStreamStages];
-};
-
-__global__ void __launch_bounds__(kStreamThreads, 1)
-    k_ef_stream(DevPlan dp, WorkerPtrs wp, float lr, uint32_t* __restrict__ out_idx,
-                float* __restrict__ out_val) {
-  constexpr int V = kStreamV;
-  constexpr int NWARP = kStreamThreads / 32;
-  static_assert(V * NWARP == 64, "two (v, warp) totals per lane of warp 0");
-  extern __shared__ __align__(128) unsigned char stream_smem[];
-  StreamShared& sh = *reinterpret_cast<StreamShared*>(stream_smem);
-  __shared__ uint32_t s_wtot[V * NWARP];
-  __shared__ uint32_t s_base[V * NWARP];
-  __shared__ uint32_t s_total;
-
-  const uint32_t items = dp.T * dp.P;
-  const uint32_t G = gridDim.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t Nal = dp.N & ~3u;  // bulk copies never read past the last full float4
-
-  if (tid == 0) {
-    for (uint32_t s = 0; s < kStreamStages; ++s) mbar_init(&sh.full[s], 1);
-    mbar_init_fence();
-  }
-  __syncthreads();
-
-  auto issue = [&](uint32_t item, uint32_t s) {  // thread 0 only
-    const uint32_t p = item / dp.T, t = item % dp.T;
-    const TileDesc td = dp.tiles[t];
-    const uint32_t a0 = td.start & ~3u;
-    const uint32_t a1 = min((td.start + td.len + 3u) & ~3u, Nal);
-    const uint32_t bytes = a1 > a0 ? (a1 - a0) * 4u : 0u;
-    mbar_arrive_expect_tx(&sh.full[s], 2u * bytes);
-    if (bytes) {
-      bulk_load(sh.g[s], wp.g[p] + a0, bytes, &sh.full[s]);
-      bulk_load(sh.r[s], wp.r[p] + a0, bytes, &sh.full[s]);
-    }
-  };
-  if (tid == 0)
-    for (uint32_t j = 0; j < kStreamStages; ++j)
-      if (blockIdx.x + j * G < items) issue(blockIdx.x + j * G, j);
-
-  for (uint32_t j = 0;; ++j) {
-    const uint32_t item = blockIdx.x + j * G;
-    if (item >= items) break;
-    const uint32_t s = j % kStreamStages;
-    const bool ok = mbar_wait_bounded(&sh.full[s], (j / kStreamStages) & 1u, kSpinLimit);
-    if (__syncthreads_or(!ok)) {
-      // a copy never completed: report it, give the copies in flight a bounded
-      // chance to land, and leave without touching the outputs further
-      if (tid == 0) {
-        atomicOr(dp.status + kStatusFlags, LAGS_FLAG_TIMEOUT);
-        for (uint32_t q = 0; q < kStreamStages; ++q) {
-          const uint32_t jq = j + q;
-          if (blockIdx.x + jq * G < items)
-            mbar_wait_bounded(&sh.full[jq % kStreamStages], (jq / kStreamStages) & 1u,
-                              kSpinLimit);
-        }
-      }
-      __syncthreads();
-      return;
-    }
-
-    const uint32_t p = item / dp.T, t = item % dp.T;
-    const TileDesc td = dp.tiles[t];
-    const LayerDesc ld = dp.layers[td.layer];
-    const float* __restrict__ g = wp.g[p];
-    float* __restrict__ r = wp.r[p];
-    const uint32_t start = td.start, end = td.start + td.len;
-    const uint32_t a0 = start & ~3u;
-    const uint32_t a1 = min((end + 3u) & ~3u, Nal);
-    const float* sg = sh.g[s];
-    const float* sr = sh.r[s];
-
-    float4 a[V];
-#pragma unroll
-    for (int v = 0; v < V; ++v) {
-      const uint32_t e0 = a0 + 4u * (v * kStreamThreads + tid);
-      float4 gv = make_float4(0.f, 0.f, 0.f, 0.f), rv = gv;
-      if (e0 < end) {
-        if (e0 + 4 <= a1) {
-          gv = *reinterpret_cast<const float4*>(sg + (e0 - a0));
-          rv = *reinterpret_cast<const float4*>(sr + (e0 - a0));
-        } else {
-          float gj[4] = {0.f, 0.f, 0.f, 0.f}, rj[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t e = e0 + q;
-            if (e >= end) continue;
-            if (e < a1) {
-              gj[q] = sg[e - a0];
-              rj[q] = sr[e - a0];
-            } else {  // the last < 4 elements of a buffer whose length is not a multiple of 4
-              gj[q] = g[e];
-              rj[q] = r[e];
-            }
-          }
-          gv = make_float4(gj[0], gj[1], gj[2], gj[3]);
-          rv = make_float4(rj[0], rj[1], rj[2], rj[3]);
-        }
-      }
-      a[v].x = __fadd_rn(rv.x, __fmul_rn(lr, gv.x));
-      a[v].y = __fadd_rn(rv.y, __fmul_rn(lr, gv.y));
-      a[v].z = __fadd_rn(rv.z, __fmul_rn(lr, gv.z));
-      a[v].w = __fadd_rn(rv.w, __fmul_rn(lr, gv.w));
-    }
-
-    if (ld.k == ld.d) {
-      const uint64_t ob = (uint64_t)p * dp.K + ld.koff;
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        const uint32_t e0 = a0 + 4u * (v * kStreamThreads + tid);
-        if (e0 >= end) continue;
-        const bool full = e0 >= start && e0 + 4 <= end;
-        if (full) st_stream(r + e0, make_float4(0.f, 0.f, 0.f, 0.f));
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t e = e0 + q;
-          if (e < start || e >= end) continue;
-          out_idx[ob + (e - ld.off)] = e;
-          out_val[ob + (e - ld.off)] = comp(a[v], q);
-          if (!full) r[e] = 0.0f;
-        }
-      }
-    } else {
-      const uint32_t lo = dp.lo_key[(size_t)p * dp.L + td.layer];
-      uint32_t masks = 0;
-      uint32_t excl[V];
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        const uint32_t e0 = a0 + 4u * (v * kStreamThreads + tid);
-        uint32_t m4 = 0;
-        if (e0 < end) {
-          const bool full = e0 >= start && e0 + 4 <= end;
-          if (full) st_stream(r + e0, a[v]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t e = e0 + q;
-            if (e < start || e >= end) continue;
-            const float x = comp(a[v], q);
-            if (!full) r[e] = x;
-            if (mag_key(x) >= lo) m4 |= 1u << q;
-          }
-        }
-        masks |= m4 << (4 * v);
-        const uint32_t c = __popc(m4);
-        excl[v] = 0;
-        if (__ballot_sync(kFull, c != 0u)) {
-          const uint32_t incl = warp_incl_scan(c);
-          excl[v] = incl - c;
-          if (lane == 31) s_wtot[v * NWARP + warp] = incl;
-        } else if (lane == 0) {
-          s_wtot[v * NWARP + warp] = 0;
-        }
-      }
-      __syncthreads();
-      if (warp == 0) {
-        const uint32_t x0 = s_wtot[2 * lane], x1 = s_wtot[2 * lane + 1];
-        const uint32_t incl = warp_incl_scan(x0 + x1);
-        const uint32_t ex = incl - x0 - x1;
-        s_base[2 * lane] = ex;
-        s_base[2 * lane + 1] = ex + x0;
-        if (lane == 31) s_total = incl;
-      }
-      __syncthreads();
-      const uint32_t cap = ld.slot_cap;
-      const uint64_t slot0 =
-          (uint64_t)p * dp.C + ld.slot_base + (uint64_t)(t - ld.tile_begin) * cap;
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        const uint32_t m4 = (masks >> (4 * v)) & 0xFu;
-        if (!m4) continue;
-        const uint32_t e0 = a0 + 4u * (v * kStreamThreads + tid);
-        uint32_t pos = s_base[v * NWARP + warp] + excl[v];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (!((m4 >> q) & 1u)) continue;
-          if (pos < cap) {
-            dp.cand_val[slot0 + pos] = comp(a[v], q);
-            dp.cand_idx[slot0 + pos] = e0 + q;
-          }
-          ++pos;
-        }
-      }
-      if (tid == 0) dp.tile_cnt[(size_t)p * dp.T + t] = s_total;
-    }
-    __syncthreads();  // stage s fully read: refill it
-    if (tid == 0 && item + kStreamStages * G < items) issue(item + kStreamStages * G, s);
-  }
-}
-
-cudaError_t configure_ef_stream() {
-  return cudaFuncSetAttribute(k_ef_stream, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)sizeof(StreamShared));
-}
-
-cudaError_t launch_ef_stream(const DevPlan& dp, const WorkerPtrs& wp, float lr,
-                             uint32_t* out_idx, float* out_val, cudaStream_t s) {
-  int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  const uint32_t items = dp.T * dp.P;
-  const uint32_t grid = items < (uint32_t)sms ? items : (uint32_t)sms;
-  k_ef_stream<<<grid, kStreamThreads, sizeof(StreamShared), s>>>(dp, wp, lr, out_idx, out_val);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_ef_capture(const DevPlan& dp, const WorkerPtrs& wp, float lr,

@@ -36,6 +36,9 @@
 // No CTA ever waits on another outside the hardware cluster barrier.
 #include <cooperative_groups.h>
 
+#include <mutex>
+#include <vector>
+
 #include "block_ops.cuh"
 #include "lags_internal.cuh"
 #include "tma.cuh"
@@ -330,11 +333,18 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
               ++at;
             }
           }
+          // if the self-check failed with fewer entries than counted, the rest
+          // of the run is padding, never uninitialised shared memory
+          for (uint32_t j = min(found, room) + tid; j < room; j += NT) {
+            stage_val[sh.tpre[q] + j] = 0.0f;
+            stage_idx[sh.tpre[q] + j] = 0xFFFFFFFFu;
+          }
         }
       }
-      const bool ok = mbar_wait_bounded(&stage_bar, 0, kSelectSpinLimit);
+      const bool ok = mbar_wait_bounded(&stage_bar, 0, dp.stage_spin);
       if (__syncthreads_or(!ok)) {
         // the copies did not complete: report, and select from global memory
+        // (the share's acc, see walk_share below)
         if (tid == 0) atomicOr(dp.status + kStatusFlags, LAGS_FLAG_TIMEOUT);
         staged = false;
         stage_timeout = true;
@@ -355,8 +365,29 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   // emission's scattered stores, which measured 6x slower.)
   // Unstaged shares: every pass walks the candidates (or, on the exhaustive
   // path, the layer's acc) from global memory.
+  // After a staging timeout the share's candidates are taken from its acc
+  // instead of the slots (a tile that overflowed its slots has only part of
+  // its candidates there): every entry of the share with key >= lo_key, one
+  // entry per thread and round, in index order.  Slower, same candidates.
+  uint32_t sa = 0, sb = 0;
+  if (stage_timeout && ta < tb) {
+    sa = __ldg(&dp.tiles[ta].start);
+    sb = __ldg(&dp.tiles[tb - 1].start) + __ldg(&dp.tiles[tb - 1].len);
+  }
+  auto walk_share = [&](auto&& fn) {
+    for (uint32_t b = sa; b < sb; b += NT) {
+      const uint32_t e = b + tid;
+      const float x = e < sb ? r[e] : 0.0f;
+      fn(e < sb && mag_key(x) >= lo_key, e, x);
+    }
+  };
   auto traverse = [&](auto&& fn) {
-    stream_candidates([&](bool valid, uint32_t, uint32_t idx, float val) { fn(valid, idx, val); });
+    if (stage_timeout) {
+      walk_share(fn);
+    } else {
+      stream_candidates(
+          [&](bool valid, uint32_t, uint32_t idx, float val) { fn(valid, idx, val); });
+    }
   };
   // Exhaustive path: the CTA's element share [ea, eb) of the layer's acc, in
   // rounds of NT * kExhV elements; each thread takes kExhV consecutive
@@ -636,14 +667,20 @@ cudaError_t configure_select() {
 
 namespace {
 // Whether the current device can run one 16-CTA select cluster with `smem`
-// bytes of dynamic shared memory per CTA (cached per device and size).
+// bytes of dynamic shared memory per CTA (cached per device and size, under a
+// lock: several host threads may launch on several devices).
 bool huge_clusters_fit(size_t smem) {
-  static int cached_dev = -1;
-  static size_t cached_smem = 0;
-  static bool cached_fit = false;
+  struct Fit {
+    size_t smem;
+    bool fit;
+  };
+  static std::mutex mu;
+  static std::vector<Fit> cache[64];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  if (dev == cached_dev && smem == cached_smem) return cached_fit;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Fit& f : cache[dev])
+    if (f.smem == smem) return f.fit;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kSelectClusterHuge);
   cfg.blockDim = dim3(kSelectThreads);
@@ -659,10 +696,9 @@ bool huge_clusters_fit(size_t smem) {
   const cudaError_t e = cudaOccupancyMaxActiveClusters(
       &clusters, k_select<kSelectClusterHuge, kSelectThreads>, &cfg);
   if (e != cudaSuccess) cudaGetLastError();  // clear; use 8-CTA clusters instead
-  cached_dev = dev;
-  cached_smem = smem;
-  cached_fit = e == cudaSuccess && clusters > 0;
-  return cached_fit;
+  const bool fit = e == cudaSuccess && clusters > 0;
+  cache[dev].push_back(Fit{smem, fit});
+  return fit;
 }
 }  // namespace
 

@@ -16,7 +16,6 @@
 namespace lags {
 cudaError_t configure_estimate();
 cudaError_t configure_select();
-cudaError_t configure_ef_stream();
 cudaError_t configure_aggregate();
 }  // namespace lags
 
@@ -69,6 +68,13 @@ double expected_candidates(const LayerDesc& ld) {
 }
 
 lags_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LAGS_OK : LAGS_ERR_CUDA; }
+
+// Calls that enqueue work on a plan's workspace run on the device it was bound on.
+lags_status check_device(const lags_plan* plan) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LAGS_ERR_CUDA;
+  return dev == plan->device ? LAGS_OK : LAGS_ERR_WRONG_DEVICE;
+}
 
 bool fill_workers(const lags_plan* plan, const float* const* grads, float* const* residuals,
                   WorkerPtrs* wp, lags_status* err) {
@@ -234,8 +240,15 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
   plan->C = slots;
   const uint64_t P = (uint64_t)num_workers, T = plan->tiles.size();
   size_t cur = 0;
+  // what aggregation reads: tables, per-tile first picks, status words
   plan->o_layers = section(cur, plan->layers.size() * sizeof(LayerDesc));
   plan->o_tiles = section(cur, T * sizeof(TileDesc));
+  plan->o_chunks = section(cur, (plan->pick_chunks.size() + 1) * sizeof(uint2));
+  plan->o_groups = section(cur, (plan->agg_groups.size() + 1) * sizeof(uint2));
+  plan->o_first = section(cur, P * T * 4);
+  plan->o_status = section(cur, kStatusWords * 4);
+  plan->agg_ws_bytes = (cur + kAlign - 1) / kAlign * kAlign;
+  // what only the selection reads
   plan->o_large = section(cur, (plan->sel_large.size() + 1) * 4);
   plan->o_small = section(cur, (plan->sel_small.size() + 1) * 4);
   plan->o_huge = section(cur, (plan->sel_huge.size() + 1) * 4);
@@ -244,10 +257,6 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
   plan->o_cnt = section(cur, P * T * 4);
   plan->o_cval = section(cur, P * (plan->C + 1) * 4);
   plan->o_cidx = section(cur, P * (plan->C + 1) * 4);
-  plan->o_first = section(cur, P * T * 4);
-  plan->o_chunks = section(cur, (plan->pick_chunks.size() + 1) * sizeof(uint2));
-  plan->o_groups = section(cur, (plan->agg_groups.size() + 1) * sizeof(uint2));
-  plan->o_status = section(cur, kStatusWords * 4);
   plan->ws_bytes = (cur + kAlign - 1) / kAlign * kAlign;
   *out_plan = plan;
   return LAGS_OK;
@@ -268,6 +277,12 @@ lags_status lags_plan_info(const lags_plan* plan, int64_t* N, int64_t* K,
   return LAGS_OK;
 }
 
+lags_status lags_plan_aggregate_workspace_bytes(const lags_plan* plan, size_t* bytes) {
+  if (!plan || !bytes) return LAGS_ERR_INVALID_ARG;
+  *bytes = plan->agg_ws_bytes;
+  return LAGS_OK;
+}
+
 lags_status lags_plan_layer(const lags_plan* plan, int32_t l, int64_t* offset, int64_t* k,
                             int64_t* pick_offset) {
   if (!plan || l < 0 || l >= plan->L) return LAGS_ERR_INVALID_ARG;
@@ -281,7 +296,8 @@ lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t byt
                                     void* stream) {
   if (!plan || !workspace) return LAGS_ERR_INVALID_ARG;
   if (!aligned(workspace, kAlign)) return LAGS_ERR_ALIGNMENT;
-  if (bytes < plan->ws_bytes) return LAGS_ERR_WORKSPACE;
+  if (bytes < plan->agg_ws_bytes) return LAGS_ERR_WORKSPACE;
+  const bool full = bytes >= plan->ws_bytes;
   int dev = 0, major = 0, minor = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LAGS_ERR_CUDA;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
@@ -289,7 +305,6 @@ lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t byt
     return LAGS_ERR_CUDA;
   if (major != 10 || minor != 0) return LAGS_ERR_UNSUPPORTED_DEVICE;
   if (configure_estimate() != cudaSuccess || configure_select() != cudaSuccess ||
-      configure_ef_stream() != cudaSuccess ||
       configure_aggregate() != cudaSuccess)
     return LAGS_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
@@ -300,10 +315,12 @@ lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t byt
   cudaError_t e = cudaSuccess;
   if (e == cudaSuccess) e = up(plan->o_layers, plan->layers.data(), plan->layers.size() * sizeof(LayerDesc));
   if (e == cudaSuccess) e = up(plan->o_tiles, plan->tiles.data(), plan->tiles.size() * sizeof(TileDesc));
-  if (e == cudaSuccess) e = up(plan->o_large, plan->sel_large.data(), plan->sel_large.size() * 4);
-  if (e == cudaSuccess) e = up(plan->o_small, plan->sel_small.data(), plan->sel_small.size() * 4);
-  if (e == cudaSuccess) e = up(plan->o_huge, plan->sel_huge.data(), plan->sel_huge.size() * 4);
-  if (e == cudaSuccess) e = up(plan->o_sparse, plan->sparse.data(), plan->sparse.size() * 4);
+  if (full) {
+    if (e == cudaSuccess) e = up(plan->o_large, plan->sel_large.data(), plan->sel_large.size() * 4);
+    if (e == cudaSuccess) e = up(plan->o_small, plan->sel_small.data(), plan->sel_small.size() * 4);
+    if (e == cudaSuccess) e = up(plan->o_huge, plan->sel_huge.data(), plan->sel_huge.size() * 4);
+    if (e == cudaSuccess) e = up(plan->o_sparse, plan->sparse.data(), plan->sparse.size() * 4);
+  }
   if (e == cudaSuccess)
     e = up(plan->o_chunks, plan->pick_chunks.data(), plan->pick_chunks.size() * sizeof(uint2));
   if (e == cudaSuccess)
@@ -314,6 +331,7 @@ lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t byt
   if (e != cudaSuccess) return LAGS_ERR_CUDA;
   bind_dev_plan(plan, base, &plan->dp);
   plan->ws = workspace;
+  plan->ws_full = full;
   plan->device = dev;
   return LAGS_OK;
 }
@@ -321,11 +339,12 @@ lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t byt
 lags_status lags_sparsify(lags_plan* plan, const float* const* grads, float* const* residuals,
                           float lr, uint32_t* out_idx, float* out_val, void* stream) {
   if (!plan || !grads || !residuals || !out_idx || !out_val) return LAGS_ERR_INVALID_ARG;
-  if (!plan->ws) return LAGS_ERR_WORKSPACE;
+  if (!plan->ws || !plan->ws_full) return LAGS_ERR_WORKSPACE;
   if (!aligned(out_idx, 4) || !aligned(out_val, 4)) return LAGS_ERR_ALIGNMENT;
   WorkerPtrs wp;
   lags_status err = LAGS_OK;
   if (!fill_workers(plan, grads, residuals, &wp, &err)) return err;
+  if ((err = check_device(plan)) != LAGS_OK) return err;
   cudaStream_t s = (cudaStream_t)stream;
   const bool timed = plan->ev_before && plan->ev_after;
   // under stream capture the timing events become event-record nodes of the
@@ -338,7 +357,7 @@ lags_status lags_sparsify(lags_plan* plan, const float* const* grads, float* con
   }
   cudaError_t e = launch_estimate(plan->dp, wp, lr, s);
   if (e == cudaSuccess && timed) e = cudaEventRecordWithFlags(plan->ev_before, s, rec_flags);
-  if (e == cudaSuccess) e = launch_ef(plan->dp, wp, lr, out_idx, out_val, s);
+  if (e == cudaSuccess) e = launch_ef_capture(plan->dp, wp, lr, out_idx, out_val, s);
   if (e == cudaSuccess && timed) e = cudaEventRecordWithFlags(plan->ev_after, s, rec_flags);
   if (e == cudaSuccess) e = launch_select(plan->dp, wp, out_idx, out_val, s);
   return cuda_status(e);
@@ -349,6 +368,8 @@ lags_status lags_aggregate(lags_plan* plan, const uint32_t* idx, const float* va
   if (!plan || !idx || !val || !dense_out) return LAGS_ERR_INVALID_ARG;
   if (!plan->ws) return LAGS_ERR_WORKSPACE;
   if (!aligned(idx, 4) || !aligned(val, 4) || !aligned(dense_out, 16)) return LAGS_ERR_ALIGNMENT;
+  const lags_status dev_ok = check_device(plan);
+  if (dev_ok != LAGS_OK) return dev_ok;
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = launch_pick_bounds(plan->dp, idx, s);
   if (e == cudaSuccess) e = launch_aggregate(plan->dp, idx, val, dense_out, nullptr, s);
@@ -361,6 +382,8 @@ lags_status lags_aggregate_apply(lags_plan* plan, const uint32_t* idx, const flo
   if (!plan->ws) return LAGS_ERR_WORKSPACE;
   if (!aligned(idx, 4) || !aligned(val, 4) || !aligned(dense_out, 16) || !aligned(weights, 16))
     return LAGS_ERR_ALIGNMENT;
+  const lags_status dev_ok = check_device(plan);
+  if (dev_ok != LAGS_OK) return dev_ok;
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = launch_pick_bounds(plan->dp, idx, s);
   if (e == cudaSuccess) e = launch_aggregate(plan->dp, idx, val, dense_out, weights, s);
@@ -480,6 +503,10 @@ lags_status lags_apply(const lags_plan* plan, float* weights, const float* dense
                        void* stream) {
   if (!plan || !weights || !dense_out) return LAGS_ERR_INVALID_ARG;
   if (!aligned(weights, 16) || !aligned(dense_out, 16)) return LAGS_ERR_ALIGNMENT;
+  if (plan->device >= 0) {  // (apply reads no workspace; a bound plan keeps its device)
+    const lags_status dev_ok = check_device(plan);
+    if (dev_ok != LAGS_OK) return dev_ok;
+  }
   return cuda_status(launch_apply((uint32_t)plan->N0, (uint32_t)plan->N, weights, dense_out,
                                   (cudaStream_t)stream));
 }
@@ -492,10 +519,19 @@ lags_status lags_plan_set_events(lags_plan* plan, void* before, void* after) {
   return LAGS_OK;
 }
 
+lags_status lags_plan_set_stage_wait_limit(lags_plan* plan, uint32_t polls) {
+  if (!plan) return LAGS_ERR_INVALID_ARG;
+  plan->stage_spin = polls;
+  plan->dp.stage_spin = polls;
+  return LAGS_OK;
+}
+
 lags_status lags_status_poll(lags_plan* plan, uint32_t* flags, uint32_t* exact_fallbacks,
                              void* stream) {
   if (!plan) return LAGS_ERR_INVALID_ARG;
   if (!plan->ws) return LAGS_ERR_WORKSPACE;
+  const lags_status dev_ok = check_device(plan);
+  if (dev_ok != LAGS_OK) return dev_ok;
   cudaStream_t s = (cudaStream_t)stream;
   uint32_t words[2] = {0, 0};
   uint32_t* dev = plan->dp.status;
@@ -505,7 +541,7 @@ lags_status lags_status_poll(lags_plan* plan, uint32_t* flags, uint32_t* exact_f
   if (e != cudaSuccess) return LAGS_ERR_CUDA;
   if (flags) *flags = words[kStatusFlags];
   if (exact_fallbacks) *exact_fallbacks = words[kStatusFallbacks];
-  return (words[kStatusFlags] & LAGS_FLAG_BAD_PICKS) ? LAGS_ERR_BAD_PICKS : LAGS_OK;
+  return lags_status_of_flags(words[kStatusFlags]);
 }
 
 const char* lags_error_string(lags_status status) {
@@ -517,6 +553,10 @@ const char* lags_error_string(lags_status status) {
     case LAGS_ERR_UNSUPPORTED_DEVICE: return "current device is not sm_100 (B200)";
     case LAGS_ERR_WORKSPACE: return "workspace missing or too small";
     case LAGS_ERR_BAD_PICKS: return "pick list not ascending or outside its layer";
+    case LAGS_ERR_TIMEOUT:
+      return "a kernel's bounded wait on its own copies gave up; picks may be incomplete";
+    case LAGS_ERR_INTERNAL: return "a kernel failed a self-check (library bug)";
+    case LAGS_ERR_WRONG_DEVICE: return "the current device is not the plan's device";
   }
   return "unknown status";
 }

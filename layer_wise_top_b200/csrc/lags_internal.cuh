@@ -42,7 +42,7 @@ constexpr uint32_t kSelectWindow = 2048;  // tiles whose prefix sits in smem at 
 // reads them from global memory on every pass instead.
 constexpr uint32_t kSelectStageMin = 1024;
 constexpr uint32_t kSelectStageMax = 20480;  // multiple of 4 (16-byte staged runs)
-constexpr uint32_t kSelectSpinLimit = 1u << 22;  // polls of the staging mbarrier
+constexpr uint32_t kSelectSpinLimit = LAGS_STAGE_WAIT_POLLS;  // polls of the staging mbarrier
 
 
 // Radix digits of the magnitude key (bits 30..0 of the fp32 pattern).
@@ -111,14 +111,13 @@ struct DevPlan {
   uint64_t C;  // candidate slots per worker
   uint32_t stage_small, stage_large, stage_huge;  // select staging capacity per launch
   uint32_t agg_tile_acc;  // aggregation launches carry a shared tile accumulator
+  uint32_t stage_spin;    // polls of the select's first staging wait before it gives up
 };
 
 // Launchers (each returns the launch's cudaError_t).
 cudaError_t launch_estimate(const DevPlan& dp, const WorkerPtrs& wp, float lr, cudaStream_t s);
 cudaError_t launch_ef_capture(const DevPlan& dp, const WorkerPtrs& wp, float lr,
                               uint32_t* out_idx, float* out_val, cudaStream_t s);
-cudaError_t launch_ef_stream(const DevPlan& dp, const WorkerPtrs& wp, float lr,
-                             uint32_t* out_idx, float* out_val, cudaStream_t s);
 cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out_idx,
                           float* out_val, cudaStream_t s);
 cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStream_t s);
@@ -130,15 +129,6 @@ cudaError_t launch_dense_sum(const DenseGrads& gp, uint32_t P, uint64_t N, float
 cudaError_t launch_dense_finish(const float* sum, uint64_t N, uint32_t P, float* dense,
                                 float* weights, cudaStream_t s);
 
-// The fused error-feedback pass used by lags_sparsify.
-inline cudaError_t launch_ef(const DevPlan& dp, const WorkerPtrs& wp, float lr, uint32_t* out_idx,
-                             float* out_val, cudaStream_t s) {
-#ifdef LAGS_EF_BULK_COPY
-  return launch_ef_stream(dp, wp, lr, out_idx, out_val, s);
-#else
-  return launch_ef_capture(dp, wp, lr, out_idx, out_val, s);
-#endif
-}
 
 // ------------------------------------------------------------------ launches
 // Programmatic dependent launch: each kernel of a step is launched so that it

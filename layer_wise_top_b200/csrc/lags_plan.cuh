@@ -19,12 +19,16 @@ struct lags_plan {
   std::vector<uint2> agg_groups;   // (first tile, tiles) per aggregation CTA
   std::vector<int64_t> off, k, koff;
   // workspace sections (byte offsets)
+  // (the sections aggregation uses come first: a workspace of agg_ws_bytes
+  // serves a plan that only aggregates)
   size_t o_layers = 0, o_tiles = 0, o_large = 0, o_small = 0, o_huge = 0, o_sparse = 0, o_lo = 0,
          o_cnt = 0,
          o_cval = 0, o_cidx = 0, o_first = 0, o_chunks = 0, o_groups = 0, o_status = 0,
-         ws_bytes = 0;
+         agg_ws_bytes = 0, ws_bytes = 0;
   void* ws = nullptr;
+  bool ws_full = false;  // the bound workspace also serves lags_sparsify
   int device = -1;
+  uint32_t stage_spin = lags::kSelectSpinLimit;  // polls of the select's first staging wait
   cudaEvent_t ev_before = nullptr, ev_after = nullptr;
   uint32_t stage_small = 0, stage_large = 0, stage_huge = 0;  // select staging per launch
   uint32_t agg_tile_acc = 0;  // some tile expects more picks than the owner search handles
@@ -67,4 +71,14 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.stage_large = plan->stage_large;
   dp.stage_huge = plan->stage_huge;
   dp.agg_tile_acc = plan->agg_tile_acc;
+  dp.stage_spin = plan->stage_spin;
+}
+
+// The status a poll returns for the flags it read: a timeout first (its picks
+// may be incomplete), then a failed self-check, then malformed pick lists.
+inline lags_status lags_status_of_flags(uint32_t flags) {
+  if (flags & LAGS_FLAG_TIMEOUT) return LAGS_ERR_TIMEOUT;
+  if (flags & LAGS_FLAG_INTERNAL) return LAGS_ERR_INTERNAL;
+  if (flags & LAGS_FLAG_BAD_PICKS) return LAGS_ERR_BAD_PICKS;
+  return LAGS_OK;
 }

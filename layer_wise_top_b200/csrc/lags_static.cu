@@ -8,17 +8,27 @@
 // thresholds, the per-tile candidate counts and the candidate slots) in one
 // array with static storage that is part of the library image on each device.
 //
-//  - Limit: a plan whose workspace exceeds kStaticScratchBytes (16 MiB) is
-//    rejected with LAGS_ERR_WORKSPACE before anything is enqueued.
-//  - Every GPU that loads liblags.so holds the 16 MiB until the process exits.
+//  - Limit: a plan whose workspace exceeds kStaticPlanBytes (16 MiB less the
+//    status block at the end of the array) is rejected with
+//    LAGS_ERR_WORKSPACE before anything is enqueued.
+//  - Every GPU on which the array is loaded holds its 16 MiB until the
+//    process exits.
 //  - All calls share the one array and it keeps the last call's contents:
-//    each call re-uploads its plan's tables and clears the status words.
-//    Calls whose work overlaps on the GPU (different streams without ordering,
-//    or several host threads) race on the array.
-//  - The first call on a device resolves the array's device address there
-//    (cudaGetSymbolAddress, with that device current) and configures the
-//    kernels; make that first call before any stream capture.
-//  - It calls no cudaMalloc, cudaFree or other allocating routine.
+//    each call re-uploads its plan's tables, and everything the kernels need
+//    zeroed is written by them before it is read.  Calls whose work overlaps
+//    on the GPU (different streams without ordering, or several host threads)
+//    race on the array.
+//  - The status words sit at a fixed place at the end of the array, are
+//    cleared once when the device is set up, collect the flags of every call
+//    and are read and cleared by lags_static_status_poll.
+//  - The first call on a device (either entry point) resolves the array's
+//    device address there (cudaGetSymbolAddress, with that device current),
+//    configures the kernels and clears the status words.  With CUDA's lazy
+//    module loading that is also when the driver loads this file's device
+//    code and reserves the array on the device, so the first call belongs at
+//    start-up, outside code that must not allocate and before any capture.
+//  - Neither entry point calls cudaMalloc, cudaFree or another allocating
+//    routine.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -32,7 +42,6 @@
 namespace lags {
 cudaError_t configure_estimate();
 cudaError_t configure_select();
-cudaError_t configure_ef_stream();
 }  // namespace lags
 
 using namespace lags;
@@ -40,6 +49,9 @@ using namespace lags;
 namespace {
 
 constexpr size_t kStaticScratchBytes = 16u << 20;
+constexpr size_t kStaticStatusBytes = 256;  // >= kStatusWords * 4
+constexpr size_t kStaticPlanBytes = kStaticScratchBytes - kStaticStatusBytes;
+static_assert(kStatusWords * 4 <= kStaticStatusBytes, "status block");
 constexpr int kMaxDevices = 64;
 
 // Host code must not use g_static_scratch as an address: on the host it names
@@ -50,8 +62,9 @@ std::mutex g_setup_mutex;
 char* g_scratch_dev[kMaxDevices] = {};
 
 // Once per device, with that device current: the scratch array's device
-// address, the sm_100 check and the kernel attributes.
-lags_status scratch_for_current_device(char** out) {
+// address, the sm_100 check, the kernel attributes and cleared status words
+// (enqueued on `s`).
+lags_status scratch_for_current_device(cudaStream_t s, char** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LAGS_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return LAGS_ERR_UNSUPPORTED_DEVICE;
@@ -65,8 +78,9 @@ lags_status scratch_for_current_device(char** out) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr)
       return LAGS_ERR_CUDA;
-    if (configure_estimate() != cudaSuccess || configure_select() != cudaSuccess ||
-      configure_ef_stream() != cudaSuccess)
+    if (configure_estimate() != cudaSuccess || configure_select() != cudaSuccess)
+      return LAGS_ERR_CUDA;
+    if (cudaMemsetAsync((char*)ptr + kStaticPlanBytes, 0, kStaticStatusBytes, s) != cudaSuccess)
       return LAGS_ERR_CUDA;
     g_scratch_dev[dev] = (char*)ptr;
   }
@@ -82,7 +96,7 @@ extern "C" lags_status lags_sparsify_static(lags_plan* plan, const float* const*
                                             float* const* residuals, float lr,
                                             uint32_t* out_idx, float* out_val, void* stream) {
   if (!plan || !grads || !residuals || !out_idx || !out_val) return LAGS_ERR_INVALID_ARG;
-  if (plan->ws_bytes > kStaticScratchBytes) return LAGS_ERR_WORKSPACE;
+  if (plan->ws_bytes > kStaticPlanBytes) return LAGS_ERR_WORKSPACE;
   if (!aligned_to(out_idx, 4) || !aligned_to(out_val, 4)) return LAGS_ERR_ALIGNMENT;
   WorkerPtrs wp;
   std::memset(&wp, 0, sizeof(wp));
@@ -92,11 +106,11 @@ extern "C" lags_status lags_sparsify_static(lags_plan* plan, const float* const*
     wp.g[p] = grads[p];
     wp.r[p] = residuals[p];
   }
+  cudaStream_t s = (cudaStream_t)stream;
   char* base = nullptr;
-  lags_status st = scratch_for_current_device(&base);
+  lags_status st = scratch_for_current_device(s, &base);
   if (st != LAGS_OK) return st;
 
-  cudaStream_t s = (cudaStream_t)stream;
   auto up = [&](size_t o, const void* src, size_t n) {
     return n ? cudaMemcpyAsync(base + o, src, n, cudaMemcpyHostToDevice, s) : cudaSuccess;
   };
@@ -106,13 +120,30 @@ extern "C" lags_status lags_sparsify_static(lags_plan* plan, const float* const*
   if (e == cudaSuccess) e = up(plan->o_small, plan->sel_small.data(), plan->sel_small.size() * 4);
   if (e == cudaSuccess) e = up(plan->o_huge, plan->sel_huge.data(), plan->sel_huge.size() * 4);
   if (e == cudaSuccess) e = up(plan->o_sparse, plan->sparse.data(), plan->sparse.size() * 4);
-  if (e == cudaSuccess) e = cudaMemsetAsync(base + plan->o_status, 0, kStatusWords * 4, s);
   if (e != cudaSuccess) return LAGS_ERR_CUDA;
 
   DevPlan dp;
   bind_dev_plan(plan, base, &dp);
+  dp.status = reinterpret_cast<uint32_t*>(base + kStaticPlanBytes);  // the fixed status block
   e = launch_estimate(dp, wp, lr, s);
-  if (e == cudaSuccess) e = launch_ef(dp, wp, lr, out_idx, out_val, s);
+  if (e == cudaSuccess) e = launch_ef_capture(dp, wp, lr, out_idx, out_val, s);
   if (e == cudaSuccess) e = launch_select(dp, wp, out_idx, out_val, s);
   return e == cudaSuccess ? LAGS_OK : LAGS_ERR_CUDA;
+}
+
+extern "C" lags_status lags_static_status_poll(uint32_t* flags, uint32_t* exact_fallbacks,
+                                               void* stream) {
+  cudaStream_t s = (cudaStream_t)stream;
+  char* base = nullptr;
+  lags_status st = scratch_for_current_device(s, &base);
+  if (st != LAGS_OK) return st;
+  uint32_t words[2] = {0, 0};
+  uint32_t* dev = reinterpret_cast<uint32_t*>(base + kStaticPlanBytes);
+  cudaError_t e = cudaMemcpyAsync(words, dev, sizeof(words), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dev, 0, sizeof(words), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return LAGS_ERR_CUDA;
+  if (flags) *flags = words[kStatusFlags];
+  if (exact_fallbacks) *exact_fallbacks = words[kStatusFallbacks];
+  return lags_status_of_flags(words[kStatusFlags]);
 }

@@ -53,11 +53,13 @@ class DataParallelLags:
                workers_per_rank: int, device: torch.device,
                group: Optional[dist.ProcessGroup] = None) -> "DataParallelLags":
         """Plans on `device`: one for the rank's workers (sparsify) and one for
-        all workers of the job (aggregation)."""
+        all workers of the job (aggregation only, so it binds the smaller
+        workspace without candidate slots)."""
         from .plan import Plan
         world = dist.get_world_size(group)
         local = Plan(layer_sizes, densities, workers_per_rank, device=device)
-        total = Plan(layer_sizes, densities, workers_per_rank * world, device=device)
+        total = Plan(layer_sizes, densities, workers_per_rank * world, device=device,
+                     aggregate_only=True)
         return cls(local, total, workers_per_rank, local.K, device, group)
 
     def exchange(self) -> None:
@@ -135,7 +137,7 @@ class LayerwiseLags:
         local = [Plan(layer_sizes, densities, workers_per_rank, device=device, layer_range=b)
                  for b in buckets]
         total = [Plan(layer_sizes, densities, workers_per_rank * world, device=device,
-                      layer_range=b) for b in buckets]
+                      layer_range=b, aggregate_only=True) for b in buckets]
         return cls(local, total, buckets, workers_per_rank, device, group)
 
     def step(self, grads: List[torch.Tensor], residuals: List[torch.Tensor], lr: float,

@@ -34,7 +34,8 @@ class Plan:
 
     def __init__(self, layer_sizes: Sequence[int], densities: Sequence[float], P: int,
                  device: Optional[torch.device] = None,
-                 layer_range: Optional[Tuple[int, int]] = None):
+                 layer_range: Optional[Tuple[int, int]] = None,
+                 aggregate_only: bool = False):
         self.device = torch.device(device if device is not None else "cuda")
         if layer_range is None:
             lb, le = 0, len(layer_sizes)
@@ -49,6 +50,11 @@ class Plan:
         self.layers = [B.lags_plan_layer(self.handle, l) for l in range(self.L)]
         self.sizes = [int(x) for x in layer_sizes[lb:le]]
         self.first = self.layers[0][0]  # first element of the plan's layers
+        # a plan that only aggregates binds the smaller workspace without the
+        # selection's candidate slots (sparsify then fails with LAGS_ERR_WORKSPACE)
+        self.aggregate_only = bool(aggregate_only)
+        if self.aggregate_only:
+            self.workspace_bytes = B.lags_plan_aggregate_workspace_bytes(self.handle)
         with torch.cuda.device(self.device):
             self.workspace = torch.empty(max(self.workspace_bytes, 256), dtype=torch.uint8,
                                          device=self.device)
@@ -122,8 +128,13 @@ class Plan:
         B.lags_plan_set_events(self.handle, before.cuda_event, after.cuda_event)
 
     def poll(self, stream: Optional[torch.cuda.Stream] = None):
-        """(flags, exact_fallbacks) since the last poll; synchronises the stream."""
+        """(flags, exact_fallbacks) since the last poll; synchronises the stream.
+        Raises LagsError (carrying the flags) when a flag reports an error."""
         return B.lags_status_poll(self.handle, _stream(stream, self.device))
+
+    def set_stage_wait_limit(self, polls: int) -> None:
+        """Failure-injection knob: polls of the selection's first staging wait."""
+        B.lags_plan_set_stage_wait_limit(self.handle, polls)
 
 
 class DenseKernels:

@@ -21,7 +21,7 @@ def declared():
 
 def test_exports_every_declared_symbol():
     names = declared()
-    assert len(names) == 19, names
+    assert len(names) == 22, names
     lib = ctypes.CDLL(L.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -29,9 +29,56 @@ def test_exports_every_declared_symbol():
 
 
 def test_error_strings():
-    for code in range(7):
+    for code in range(10):
         assert L.lags_error_string(code) not in ("", "unknown status")
+    assert len({L.lags_error_string(c) for c in range(10)}) == 10
     assert L.lags_error_string(99) == "unknown status"
+
+
+def test_status_codes_match_header():
+    with open(os.path.join(ROOT, "include", "lags.h")) as f:
+        text = f.read()
+    for name in ("LAGS_ERR_TIMEOUT", "LAGS_ERR_INTERNAL", "LAGS_ERR_WRONG_DEVICE",
+                 "LAGS_ERR_BAD_PICKS", "LAGS_ERR_WORKSPACE"):
+        m = re.search(rf"\b{name}\s*=\s*(\d+)", text)
+        assert m and int(m.group(1)) == getattr(L, name), name
+    for name in ("LAGS_FLAG_TIMEOUT", "LAGS_FLAG_INTERNAL", "LAGS_FLAG_BAD_PICKS"):
+        m = re.search(rf"#define {name} (0x[0-9a-fA-F]+)u", text)
+        assert m and int(m.group(1), 16) == getattr(L, name), name
+    m = re.search(r"#define LAGS_STAGE_WAIT_POLLS (\d+)u", text)
+    assert m and int(m.group(1)) == L.LAGS_STAGE_WAIT_POLLS
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_aggregate_only_workspace_is_a_smaller_prefix(name):
+    # the job-wide plan of a data-parallel rank only aggregates: its workspace
+    # leaves out the candidate slots, the bulk of the full workspace
+    w = WORKLOADS[name]
+    h = L.lags_plan_create(w.sizes, w.densities, w.P)
+    try:
+        full = L.lags_plan_info(h)[2]
+        agg = L.lags_plan_aggregate_workspace_bytes(h)
+        assert 0 < agg < full and agg % 256 == 0
+        # tiles (16 B each) and the per-(worker, tile) first picks (4 B) fit in it
+        tiles = sum((o + d - 1) // 8192 - o // 8192 + 1
+                    for o, d in zip(w.offsets, w.sizes))
+        assert agg >= 16 * tiles + 4 * w.P * tiles
+        if name != "resnet20":
+            assert agg < full / 4
+    finally:
+        L.lags_plan_destroy(h)
+
+
+def test_stage_wait_limit_knob_validates():
+    with pytest.raises(L.LagsError) as e:
+        L.lags_plan_set_stage_wait_limit(None, 0)
+    assert e.value.status == L.LAGS_ERR_INVALID_ARG
+    h = L.lags_plan_create([100], [0.1], 2)
+    try:
+        L.lags_plan_set_stage_wait_limit(h, 0)
+        L.lags_plan_set_stage_wait_limit(h, L.LAGS_STAGE_WAIT_POLLS)
+    finally:
+        L.lags_plan_destroy(h)
 
 
 @pytest.mark.parametrize("name", sorted(WORKLOADS))
