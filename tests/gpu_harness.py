@@ -83,47 +83,56 @@ def compare_layer(run: GpuRun, l: int, exp, where: str) -> None:
         f"{where}: weights"
 
 
-def check_invariants(run: GpuRun, workers: Iterable[int], check_dense: bool = True) -> None:
-    """Full-size properties that determine the result uniquely: for every layer
-    the picks are ascending and inside the layer, each value is acc at its
-    index, picked residuals are +0 and the others keep acc, every picked
-    magnitude is >= every unpicked one, and among entries tied at the smallest
-    picked magnitude the picked ones have the lowest indices.  The dense update
-    is recomputed in worker order with one rounding per add."""
+def check_invariants(run: GpuRun, workers: Iterable[int], check_dense: bool = True,
+                     max_elems: int = 1 << 27) -> None:
+    """Full-size properties that determine the result uniquely, checked for
+    the given workers of every layer (workers in groups of up to `max_elems`
+    layer elements, so whole layers are checked at once): the picks are
+    ascending and inside the layer, each value is acc at its index, picked
+    residuals are +0 and the others keep acc, every picked magnitude is >=
+    every unpicked one, and among entries tied at the smallest picked
+    magnitude the picked ones have the lowest indices.  The dense update is
+    recomputed in worker order with one rounding per add."""
     assert run.prev is not None, "run with keep_prev=True"
     lr = torch.tensor(run.lr, dtype=torch.float32, device="cuda")
     K = run.plan.K
     idx_all = run.idx.view(run.P, K)
     val_all = run.val.view(run.P, K)
-    for p in workers:
-        acc = run.prev[p] + lr * run.grads[p]  # two separate fp32 roundings
-        res = run.res[p]
-        for l, (off, k, koff) in enumerate(run.plan.layers):
-            d = run.plan.sizes[l]
-            li = idx_all[p, koff:koff + k].to(torch.int64) & 0xFFFFFFFF
-            lv = val_all[p, koff:koff + k]
-            assert bool((li >= off).all() and (li < off + d).all()), (p, l, "range")
+    workers = list(workers)
+    i32 = torch.int32
+    for l, (off, k, koff) in enumerate(run.plan.layers):
+        d = run.plan.sizes[l]
+        per = max(1, min(len(workers), max_elems // d))
+        for g0 in range(0, len(workers), per):
+            ws = workers[g0:g0 + per]
+            # acc = prev + lr * g: two separate fp32 roundings
+            a = torch.stack([run.prev[p][off:off + d] + lr * run.grads[p][off:off + d]
+                             for p in ws])
+            res = torch.stack([run.res[p][off:off + d] for p in ws])
+            li = idx_all[ws, koff:koff + k].to(torch.int64) & 0xFFFFFFFF
+            lv = val_all[ws, koff:koff + k]
+            where = (l, ws)
+            assert bool((li >= off).all() and (li < off + d).all()), (where, "range")
             if k > 1:
-                assert bool((li[1:] > li[:-1]).all()), (p, l, "ascending")
-            a = acc[off:off + d]
+                assert bool((li[:, 1:] > li[:, :-1]).all()), (where, "ascending")
             loc = li - off
-            assert torch.equal(lv.view(torch.int32), a[loc].view(torch.int32)), (p, l, "val")
-            rl = res[off:off + d]
-            mask = torch.zeros(d, dtype=torch.bool, device="cuda")
-            mask[loc] = True
-            assert bool((rl[mask].view(torch.int32) == 0).all()), (p, l, "zeroed")
-            assert torch.equal(rl[~mask].view(torch.int32), a[~mask].view(torch.int32)), \
-                (p, l, "residual")
+            assert torch.equal(lv.view(i32), torch.gather(a, 1, loc).view(i32)), (where, "val")
+            mask = torch.zeros_like(a, dtype=torch.bool)
+            mask.scatter_(1, loc, True)
+            assert bool((res.view(i32)[mask] == 0).all()), (where, "zeroed")
+            assert torch.equal(res.view(i32)[~mask], a.view(i32)[~mask]), (where, "residual")
             if k < d:
                 mag = a.abs()
-                tmin = mag[mask].min()
-                assert bool(tmin >= mag[~mask].max()), (p, l, "magnitude")
-                tie_unpicked = (~mask) & (mag == tmin)
-                if bool(tie_unpicked.any()):
-                    tie_picked = mask & (mag == tmin)
-                    first_unpicked = int(torch.nonzero(tie_unpicked)[0])
-                    last_picked = int(torch.nonzero(tie_picked)[-1])
-                    assert last_picked < first_unpicked, (p, l, "tie order")
+                inf = torch.tensor(float("inf"), device="cuda")
+                tmin = torch.where(mask, mag, inf).amin(1, keepdim=True)
+                umax = torch.where(mask, -inf, mag).amax(1, keepdim=True)
+                assert bool((tmin >= umax).all()), (where, "magnitude")
+                pos = torch.arange(d, device="cuda", dtype=torch.int64).expand_as(a)
+                at_min = mag == tmin
+                first_unpicked = torch.where(at_min & ~mask, pos, d).amin(1)
+                last_picked = torch.where(at_min & mask, pos, -1).amax(1)
+                assert bool((last_picked < first_unpicked).all()), (where, "tie order")
+            del a, res, mask
     if check_dense:
         dense = torch.zeros(run.plan.N, dtype=torch.float32, device="cuda")
         for p in range(run.P):
@@ -191,3 +200,49 @@ def check_layer_chunked(run: GpuRun, l: int, lr: float, chunk: int = 1 << 28) ->
             sel = idx[inside] - a
             acc[sel] = acc[sel] + val[inside]
         assert torch.equal(bits(run.dense[a:b]), bits(acc / fP)), f"dense chunk {a}"
+
+
+def same_bits_or_nan(got_u32, exp_f32):
+    """Bitwise equality, except that a NaN matches any NaN: IEEE 754 leaves the
+    payload and sign of an invalid operation's NaN (inf - inf) unspecified."""
+    exp_u32 = exp_f32.view(np.uint32)
+    got_f = got_u32.view(np.float32)
+    both_nan = np.isnan(got_f) & np.isnan(exp_f32)
+    return bool(np.all((got_u32 == exp_u32) | both_nan))
+
+
+def run_full_compare(sizes, densities, P, lr, steps, grad_fn, expect_fallbacks=None):
+    """Element-by-element parity of every output for `steps` steps."""
+    run = GpuRun(sizes, densities, P, lr)
+    hist = lo.run_workload(sizes, densities, P, lr, steps, grad_fn)
+    total_fb = 0
+    for s in range(steps):
+        for p in range(P):
+            run.grads[p].copy_(torch.from_numpy(grad_fn(p, s)))
+        run.step(fused=s % 2 == 1)  # odd steps: lags_aggregate_apply
+        flags, fb = run.plan.poll()
+        assert flags == 0
+        total_fb += fb
+        e_idx, e_val, e_res, e_dense, e_w = hist[s]
+        K = run.plan.K
+        assert np.array_equal(u32(run.idx).reshape(P, K), e_idx), f"step {s}: idx"
+        assert np.array_equal(u32(run.val).reshape(P, K), e_val.view(np.uint32)), f"step {s}: val"
+        for p in range(P):
+            assert np.array_equal(u32(run.res[p]), e_res[p].view(np.uint32)), f"step {s}: res {p}"
+        assert same_bits_or_nan(u32(run.dense), e_dense), f"step {s}: dense"
+        assert same_bits_or_nan(u32(run.weights), e_w), f"step {s}: weights"
+    if expect_fallbacks is not None:
+        assert expect_fallbacks(total_fb), total_fb
+    return total_fb
+
+
+def synth_grad_fn(w):
+    """grad_fn(p, s) of a workload: host gradients, generated once each."""
+    import synth
+    cache = {}
+
+    def fn(p, s):
+        if (p, s) not in cache:
+            cache[(p, s)] = synth.worker_grads_host(w, p, s)
+        return cache[(p, s)]
+    return fn
