@@ -3,14 +3,17 @@
 
 One step = error feedback + layer-wise exact top-k for all P simulated workers
 (lags_sparsify) and the deterministic sparse aggregation with the weight update
-(lags_aggregate_apply), over one batch of synthetic gradients already in HBM.  value = P*N elements per step / step time, in Gelem/s; under torchrun
-each rank runs its own replica (no collective on the data path) and value sums
-the elements of all ranks over the slowest rank's time.
+(lags_aggregate_apply), over one batch of synthetic gradients already in HBM.
+value = P*N elements per step / step time, in Gelem/s; under torchrun each rank
+runs its own replica (no collective on the data path) and value sums the
+elements of all ranks over the slowest rank's time.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config vgg16]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config gpt_1_3b]
     python bench.py --impl reference ...   # the CPU oracle on a bounded sample
 
-Prints one JSON line (rank 0).
+The default workload is the largest that fits one GPU: the 1.3B-parameter
+transformer (P = 8 workers, N = 1,311,178,752 elements, 126 GB streamed per
+step).  Prints one JSON line (rank 0).
 """
 from __future__ import annotations
 
@@ -29,19 +32,41 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "LAGS sparsify+aggregate Gelem/s per step; achieved HBM GB/s vs peak"
-# DRAM bytes (read + write) of one k_ef_capture launch from the ncu capture in
-# profiles/k_ef_capture_vgg16.md (VGG-16 workload, 235,517,088 elements).
-# Other workloads scale it by their element count (the pass is a stream over
-# the elements, so its traffic grows in proportion).
-EF_TRAFFIC_BYTES = 1_885_774_000 + 895_709_696
-EF_TRAFFIC_ELEMENTS = 235_517_088
-# DRAM bytes of one k_dense_sum launch (profiles/k_dense_sum_vgg16.md, VGG-16
-# shapes, 16 workers); other workloads scale it by their element count.
-DENSE_TRAFFIC_BYTES = 942_080_512 + 12_375_808
-DENSE_TRAFFIC_ELEMENTS = 235_517_088
+DEFAULT_CONFIG = "gpt_1_3b"
+# DRAM bytes (read + write) of one launch of a kernel, from single-launch ncu
+# captures (dram__bytes_read.sum + dram__bytes_write.sum) of the workload or
+# tensor range named by the key, with the worker-elements that launch
+# processed.  A workload without its own capture takes the capture of a range
+# of its own tensors (same kernel, same layer shapes), else another
+# workload's, scaled by worker-elements: the passes stream over the elements,
+# so their traffic grows in proportion.
+EF_TRAFFIC = {  # k_ef_capture
+    "vgg16": (1_885_774_000 + 895_709_696, 235_517_088),
+}
+DENSE_TRAFFIC = {  # k_dense_sum
+    "vgg16": (942_080_512 + 12_375_808, 235_517_088),
+}
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 POOL_BUDGET_BYTES = 48 * 1024 ** 3
+# oracle timing: per worker, consecutive tensors from the second one (the first
+# is the embedding of the transformer and LSTM workloads) up to this many elements
+ORACLE_SAMPLE_ELEMS = 56_000_000
+
+
+def traffic_for(table, name, elems):
+    """(bytes per launch, where they come from) for a launch over `elems`
+    worker-elements of workload `name` (a `--tensors` case is `name[a:b]`)."""
+    if name in table:
+        b, e = table[name]
+        if e == elems:
+            return b, f"ncu capture of this workload ({name})"
+    base = name.split("[")[0]
+    order = (lambda k: (not k.startswith(base + "["), k != base, k != "vgg16", k))
+    for key in sorted(table, key=order):
+        b, e = table[key]
+        return b * elems / e, f"ncu capture of {key}, scaled by worker-elements"
+    return None, "no capture"
 
 
 def parse_args():
@@ -50,7 +75,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="vgg16",
+    ap.add_argument("--config", default=DEFAULT_CONFIG,
                     choices=["resnet20", "vgg16", "resnet50", "lstm_ptb", "gpt_1_3b"])
     ap.add_argument("--tensors", default=None, metavar="A:B",
                     help="only tensors A..B-1 of the workload (a smaller case of the same "
@@ -74,6 +99,10 @@ def parse_args():
                     help="the dense S-SGD baseline instead of LAGS: worker-ordered sum of "
                          "lr*g (lags_dense_sum), NCCL all-reduce of the ranks' sums, division "
                          "and update (lags_dense_finish); the job's P workers split over ranks")
+    ap.add_argument("--adaptive", default=None, choices=["10gbe", "nvlink"],
+                    help="per-layer densities from each layer's communication-to-computation "
+                         "ratio: backward times measured on the device (synthetic backward), "
+                         "messages over the named link, planned by lags_adaptive_densities")
     ap.add_argument("--graph", action="store_true",
                     help="capture each step (one graph per gradient buffer of the pool) in a "
                          "CUDA graph and time graph replays")
@@ -158,11 +187,19 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-# ------------------------------------------------------------------- reference arm
-def oracle_sample_layers(w, budget_elems):
-    """Consecutive layers of one worker, from the first, up to ~budget elements."""
+# ------------------------------------------------------------------- oracle timing
+# The CPU oracle (plain numpy: one sort per worker-layer segment, worker-ordered
+# aggregation) timed on the host cores.  Gradients are generated into shared
+# memory before the clock starts; a spawn pool of one process per core then
+# sparsifies the (worker, layer) segments and the parent aggregates each layer
+# in worker order.  The step is step 0 of the workload (zero residuals).
+
+def oracle_sample_layers(w, budget_elems=ORACLE_SAMPLE_ELEMS):
+    """Consecutive tensors of one worker from the second (or the only) one, up
+    to about budget_elems elements."""
     layers, total = [], 0
-    for l, d in enumerate(w.sizes):
+    for l in range(1 if w.L > 1 else 0, w.L):
+        d = w.sizes[l]
         if layers and total + d > budget_elems:
             break
         layers.append(l)
@@ -170,50 +207,156 @@ def oracle_sample_layers(w, budget_elems):
     return layers, total
 
 
-def time_oracle(w, worker, step, layers):
-    """Oracle sparsify + aggregate of one worker's sampled layers (zero
-    residual, worker `worker`, step `step`); returns seconds and elements."""
+def _oracle_segment(shm_name, at, d, off, k, lr):
+    """One worker's sparsification of one layer (pool job): zero residual,
+    gradient read from shared memory.  Returns the picks."""
+    from multiprocessing import shared_memory
     import numpy as np
     import oracle.lags_oracle as lo
-    import synth
-    grads = {l: synth.layer_grads_host(w, worker, step, l) for l in layers}
-    t0 = time.perf_counter()
-    elems = 0
-    for l in layers:
-        d = w.sizes[l]
-        k = lo.k_of(d, w.densities[l])
-        off = w.offsets[l]
-        idx, val, _ = lo.sparsify_layer(off, k, [grads[l]], [np.zeros(d, np.float32)], w.lr)
-        lo.aggregate_layer(off, d, idx, val)
-        elems += d
-    return time.perf_counter() - t0, elems
+    shm = shared_memory.SharedMemory(name=shm_name)
+    try:
+        g = np.ndarray((d,), dtype=np.float32, buffer=shm.buf, offset=4 * at).copy()
+    finally:
+        shm.close()
+    idx, val, _ = lo.sparsify_layer(off, k, [g], [np.zeros(d, np.float32)], lr)
+    return idx[0], val[0]
+
+
+def _warm(_):
+    import oracle.lags_oracle  # noqa: F401
+    return os.getpid()
+
+
+class OracleTimer:
+    """Times the oracle's sparsify + aggregate over (worker, layer) segments
+    of a workload on `procs` host processes."""
+
+    def __init__(self, w, procs=None, densities=None):
+        import concurrent.futures as cf
+        import multiprocessing as mp
+        self.w = w
+        self.dens = list(densities) if densities is not None else w.densities
+        self.procs = procs or os.cpu_count() or 1
+        self.ex = cf.ProcessPoolExecutor(max_workers=self.procs,
+                                         mp_context=mp.get_context("spawn"))
+        list(self.ex.map(_warm, range(self.procs)))  # start and import outside the clock
+        self.shm = None
+
+    def close(self):
+        self.ex.shutdown()
+        if self.shm is not None:
+            self.shm.close()
+            self.shm.unlink()
+            self.shm = None
+
+    def _fill(self, segs, step):
+        """Generate the segments' gradients into shared memory (untimed)."""
+        from multiprocessing import shared_memory
+        import numpy as np
+        import synth
+        total = sum(self.w.sizes[l] for _, l in segs)
+        if self.shm is None or self.shm.size < 4 * total:
+            if self.shm is not None:
+                self.shm.close()
+                self.shm.unlink()
+            self.shm = shared_memory.SharedMemory(create=True, size=max(4 * total, 4))
+        at, where = 0, []
+        for p, l in segs:
+            d = self.w.sizes[l]
+            buf = np.ndarray((d,), dtype=np.float32, buffer=self.shm.buf, offset=4 * at)
+            t = self.w.tensors[l]
+            synth.fill_host(buf, self.w.offsets[l], self.w.seed, p, step, self.w.dist, t.scale)
+            where.append((p, l, at))
+            at += d
+        return where
+
+    def run(self, segs, step=0, procs=None):
+        """Seconds and worker-elements for one oracle pass over `segs`
+        [(worker, layer)] (all of one layer's workers are aggregated)."""
+        import oracle.lags_oracle as lo
+        w = self.w
+        where = self._fill(segs, step)
+        ks = {l: lo.k_of(w.sizes[l], self.dens[l]) for _, l in segs}
+        order = sorted(where, key=lambda x: -w.sizes[x[1]])  # largest first
+        t0 = time.perf_counter()
+        if procs == 1:
+            res = [(p, l, _oracle_segment(self.shm.name, at, w.sizes[l], w.offsets[l], ks[l],
+                                          w.lr)) for p, l, at in order]
+        else:
+            futs = [(p, l, self.ex.submit(_oracle_segment, self.shm.name, at, w.sizes[l],
+                                          w.offsets[l], ks[l], w.lr)) for p, l, at in order]
+            res = [(p, l, f.result()) for p, l, f in futs]
+        by_layer = {}
+        for p, l, (idx, val) in res:
+            by_layer.setdefault(l, []).append((p, idx, val))
+        import numpy as np
+        for l, picks in by_layer.items():
+            picks.sort(key=lambda x: x[0])  # worker order
+            lo.aggregate_layer(w.offsets[l], w.sizes[l], np.stack([x[1] for x in picks]),
+                               np.stack([x[2] for x in picks]))
+        secs = time.perf_counter() - t0
+        return secs, sum(w.sizes[l] for _, l in segs)
+
+
+def cpu_baseline(w, densities=None):
+    """The oracle on the host cores: all P workers' sample tensors in parallel
+    (one process per core), plus one worker's largest sample tensor on one
+    thread."""
+    layers, per_worker = oracle_sample_layers(w)
+    timer = OracleTimer(w, densities=densities)
+    try:
+        segs = [(p, l) for p in range(w.P) for l in layers]
+        secs, elems = timer.run(segs)
+        big = max(layers, key=lambda l: w.sizes[l])
+        s1, e1 = timer.run([(0, big)], procs=1)
+    finally:
+        timer.close()
+    return {"value": elems / secs / 1e9, "unit": "Gelem/s", "cores": timer.procs,
+            "kind": "oracle",
+            "sample": (f"step 0 (zero residuals) of all {w.P} workers' tensors "
+                       f"{layers[0]}..{layers[-1]} ({per_worker} elements per worker, "
+                       f"{elems} in all), sparsify + aggregate; numpy oracle in "
+                       f"{timer.procs} spawned processes over (worker, tensor) segments, "
+                       f"gradients pre-generated in shared memory"),
+            "seconds": secs,
+            "single_thread": {"value": e1 / s1 / 1e9, "unit": "Gelem/s", "seconds": s1,
+                              "sample": f"worker 0, tensor {big} ({e1} elements), one thread"}}
 
 
 def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, timed on the host cores
+    on the same workload, metric and unit.  Each step is a bounded sample of
+    the workload: all P workers of one tensor of the oracle sample (tensors
+    taken in turn), in parallel over the workers, then aggregated."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    from synth.configs import WORKLOADS
     w = workload(args)
-    layers, total = oracle_sample_layers(w, 4_000_000)
-    sample = (f"one worker per step (worker = step mod P), layers {layers[0]}..{layers[-1]} "
-              f"({total} elements), zero residual; numpy oracle, single thread")
-    for s in range(args.warmup):
-        time_oracle(w, s % w.P, s, layers)
-    secs, elems = 0.0, 0
-    for s in range(args.steps):
-        t, e = time_oracle(w, (args.warmup + s) % w.P, args.warmup + s, layers)
-        secs += t
-        elems += e
+    layers, _ = oracle_sample_layers(w)
+    timer = OracleTimer(w)
+    try:
+        for s in range(args.warmup):
+            timer.run([(p, layers[s % len(layers)]) for p in range(w.P)], step=s)
+        secs, elems = 0.0, 0
+        for s in range(args.steps):
+            t, e = timer.run([(p, layers[(args.warmup + s) % len(layers)]) for p in range(w.P)],
+                             step=args.warmup + s)
+            secs += t
+            elems += e
+    finally:
+        timer.close()
     value = elems / secs / 1e9
+    sample = (f"per step all {w.P} workers of one tensor of {layers[0]}..{layers[-1]} in "
+              f"turn (zero residuals; {elems} worker-elements over {args.steps} steps), "
+              f"sparsify + aggregate; numpy oracle in {timer.procs} spawned processes")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "Gelem/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": workload_config(w, sample_elements_per_step=total),
-        "cpu_baseline": {"kind": "oracle", "value": value, "unit": "Gelem/s", "cores": 1,
-                         "sample": sample},
+        "config": workload_config(w, sample_elements=elems),
+        "cpu_baseline": {"kind": "oracle", "value": value, "unit": "Gelem/s",
+                         "cores": timer.procs, "sample": sample},
         "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -222,21 +365,6 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------- our arm
-def cpu_baseline(w):
-    layers, total = oracle_sample_layers(w, 8_000_000)
-    secs, elems, step = 0.0, 0, 0
-    while secs < 12.0 and step < 16:
-        t, e = time_oracle(w, step % w.P, step, layers)
-        secs += t
-        elems += e
-        step += 1
-    return {"value": elems / secs / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
-            "sample": (f"{step} x one worker's layers {layers[0]}..{layers[-1]} ({total} "
-                       f"elements, zero residual), sparsify+aggregate, numpy single thread "
-                       f"on {os.cpu_count()} host cores"),
-            "seconds": secs}
-
-
 def run_dense(args):
     """Dense S-SGD baseline: same workload, metric and timing rules as LAGS."""
     import torch
@@ -329,10 +457,8 @@ def run_dense(args):
         "roofline": {"kernel": "k_dense_sum", "bound": "hbm", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak,
-                     "traffic": DENSE_TRAFFIC_BYTES * (P * N) / DENSE_TRAFFIC_ELEMENTS,
-                     "traffic_source": ("ncu capture of this workload" if P * N ==
-                                        DENSE_TRAFFIC_ELEMENTS else
-                                        "ncu capture of the VGG-16 shapes, scaled by elements"),
+                     "traffic": traffic_for(DENSE_TRAFFIC, w.name, P * N)[0],
+                     "traffic_source": traffic_for(DENSE_TRAFFIC, w.name, P * N)[1],
                      "algorithmic_bytes_per_launch": sum_bytes, "avg_launch_ms": sum_ms,
                      "share_of_step": sum_ms / (ms_max / K)},
         "cpu_baseline": None, "e2e": None, "gpu_launches": 2 * K, "clocks": clk,
@@ -363,6 +489,20 @@ def run_ours(args):
 
     w = workload(args)
     P, N = w.P, w.N
+    dens = w.densities
+    adaptive_cfg = None
+    if args.adaptive:
+        # densities from each layer's communication-to-computation ratio, with
+        # backward times measured on this device before the timed region
+        from layer_wise_top_b200 import adaptive
+        dens, secs = adaptive.plan_densities([t.shape for t in w.tensors], P, args.adaptive,
+                                             0.001, device=dev)
+        adaptive_cfg = {"link": args.adaptive, "alpha_s": adaptive.LINKS[args.adaptive][0],
+                        "beta_s_per_byte": adaptive.LINKS[args.adaptive][1],
+                        "backward_ms": sum(secs) * 1e3,
+                        "dense_layers": sum(1 for r in dens if r >= 1.0),
+                        "at_rho_min": sum(1 for r in dens if r <= 0.001),
+                        "density_mean": sum(dens) / len(dens)}
     dp = None
     lw = None
     buckets = None
@@ -383,22 +523,22 @@ def run_ours(args):
             # message model: NVLink all-gather of 8 B per pick per worker,
             # 20 us start-up, the measured 770 GB/s peer bandwidth
             import layer_wise_top_b200 as lags
-            h = lags.lags_plan_create(w.sizes, w.densities, 1)
+            h = lags.lags_plan_create(w.sizes, dens, 1)
             ks = [lags.lags_plan_layer(h, l)[1] for l in range(w.L)]
             lags.lags_plan_destroy(h)
             buckets, _ = lags.lags_merge_layers(
                 [8 * P * k for k in ks], [d * args.bwd_ps_per_elem * 1e-12 for d in w.sizes],
                 2e-5, 1.0 / 770e9)
-            lw = LayerwiseLags.create(w.sizes, w.densities, P // world, buckets, dev)
+            lw = LayerwiseLags.create(w.sizes, dens, P // world, buckets, dev)
             dp = lw
         else:
-            dp = DataParallelLags.create(w.sizes, w.densities, P // world, dev)
+            dp = DataParallelLags.create(w.sizes, dens, P // world, dev)
         P = P // world  # workers held by this rank
         plan = dp.local[0] if lw is not None else dp.local
     elif args.global_topk is not None:
         plan = Plan([N], [args.global_topk], P, device=dev)
     else:
-        plan = Plan(w.sizes, w.densities, P, device=dev)
+        plan = Plan(w.sizes, dens, P, device=dev)
     # plans whose fused pass is timed and whose status words are read
     local_plans = lw.local if lw is not None else [plan]
     status_plans = local_plans + (lw.total if lw is not None else [])
@@ -506,8 +646,18 @@ def run_ours(args):
     if graphs is not None:
         step = eager_step  # the e2e leg below times the eager calls
     if not args.no_e2e and dp is None:
-        host = [torch.empty(N, dtype=torch.float32, pin_memory=True) for _ in range(P)]
-        for p in range(P):
+        # one pinned host buffer per worker while they fit in a quarter of the
+        # host's free memory; otherwise workers share buffers in turn (worker p
+        # copies buffer p mod n).  Either way every worker's P*N*4 bytes cross
+        # the host link every step.
+        try:
+            import psutil
+            avail = psutil.virtual_memory().available
+        except Exception:  # pragma: no cover
+            avail = 64 << 30
+        n_host = max(1, min(P, int(avail * 0.25) // (N * 4)))
+        host = [torch.empty(N, dtype=torch.float32, pin_memory=True) for _ in range(n_host)]
+        for p in range(n_host):
             host[p].copy_(grads[0][p])
         w_host = torch.empty(N, dtype=torch.float32, pin_memory=True)
         dev_g = grads[0]
@@ -519,7 +669,7 @@ def run_ours(args):
         e0.record()
         for i in range(ke):
             for p in range(P):
-                dev_g[p].copy_(host[p], non_blocking=True)
+                dev_g[p].copy_(host[p % n_host], non_blocking=True)
             plan.sparsify(dev_g, res, w.lr, idx, val)
             plan.aggregate_apply(idx, val, dense, weights)
             w_host.copy_(weights, non_blocking=True)
@@ -531,7 +681,10 @@ def run_ours(args):
             dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
         e2e = {"value": world * P * N * ke / (float(e_ms.item()) / 1e3) / 1e9,
                "unit": "Gelem/s", "steps": ke, "h2d_bytes_per_step": P * N * 4,
-               "d2h_bytes_per_step": N * 4}
+               "d2h_bytes_per_step": N * 4, "pinned_host_buffers": n_host,
+               "path": "per step: P pinned host->device gradient copies, lags_sparsify, "
+                       "lags_aggregate_apply, device->host copy of the updated weights"}
+        del host, w_host
 
     # lags_apply alone (outside the step: the step applies the update fused
     # into the aggregation), 12 bytes per element
@@ -551,7 +704,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w)
+        cpu = cpu_baseline(w, dens)
 
     is_dp = dp is not None
     if world > 1 or is_dp:
@@ -589,15 +742,14 @@ def run_ours(args):
             selection=(f"global top-k over all {N} elements at density {args.global_topk}"
                        if args.global_topk is not None else "layer-wise top-k"),
             step="lags_sparsify + lags_aggregate_apply (aggregate and apply fused)"
-                 + (", replayed from CUDA graphs" if args.graph else "")),
+                 + (", replayed from CUDA graphs" if args.graph else ""),
+            **({"densities": "adaptive (per layer)", "adaptive": adaptive_cfg,
+                "K_per_worker": sum(pl.K for pl in local_plans)} if adaptive_cfg else {})),
         "roofline": {"kernel": "k_ef_capture", "bound": "hbm", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak,
-                     "traffic": EF_TRAFFIC_BYTES * (P * N) / EF_TRAFFIC_ELEMENTS,
-                     "traffic_source": ("ncu capture of this workload" if P * N ==
-                                        EF_TRAFFIC_ELEMENTS else
-                                        "ncu capture of the VGG-16 workload, scaled by "
-                                        "elements"),
+                     "traffic": traffic_for(EF_TRAFFIC, w.name, P * N)[0],
+                     "traffic_source": traffic_for(EF_TRAFFIC, w.name, P * N)[1],
                      "algorithmic_bytes_per_launch": k1_bytes, "avg_launch_ms": k1_avg,
                      "share_of_step": k1_avg / (ms_max / K)},
         "step_hbm": {
@@ -614,6 +766,9 @@ def run_ours(args):
         "clocks": clk,
         "status": {"flags": flags | flags2, "exact_fallback_segments": fallbacks + fallbacks2},
     }
+    if line["status"]["exact_fallback_segments"]:
+        print(f"warning: {line['status']['exact_fallback_segments']} (worker, layer) segments "
+              "took the exhaustive selection path (exact, slower)", file=sys.stderr)
     print(json.dumps(line), flush=True)
     return 0
 

@@ -19,11 +19,49 @@ def _bench(argv):
         sys.argv = old
 
 
-def test_default_workload_is_vgg16():
+def test_default_workload_is_the_largest_single_gpu_config():
     bench, args = _bench([])
     w = bench.workload(args)
-    assert w.name == "vgg16" and w.P == 16 and w.N == 14_719_818
+    assert w.name == "gpt_1_3b" and w.P == 8 and w.N == 1_311_178_752
     assert args.steps >= 1 and args.warmup >= 3
+
+
+def test_oracle_sample_is_bounded():
+    bench, _ = _bench([])
+    from synth.configs import WORKLOADS
+    for name, w in WORKLOADS.items():
+        layers, per_worker = bench.oracle_sample_layers(w)
+        assert layers == list(range(layers[0], layers[-1] + 1))
+        assert per_worker == sum(w.sizes[l] for l in layers)
+        assert per_worker <= max(bench.ORACLE_SAMPLE_ELEMS, max(w.sizes[l] for l in layers))
+    layers, per_worker = bench.oracle_sample_layers(WORKLOADS["gpt_1_3b"])
+    assert layers[:8] == list(range(1, 9))  # a whole transformer block
+    assert 50_339_840 <= per_worker <= bench.ORACLE_SAMPLE_ELEMS
+
+
+def test_traffic_scaling():
+    bench, _ = _bench([])
+    table = {"vgg16": (2000, 1000), "gpt_1_3b[1:9]": (300, 100)}
+    assert bench.traffic_for(table, "vgg16", 1000) == (2000, "ncu capture of this workload (vgg16)")
+    b, src = bench.traffic_for(table, "gpt_1_3b", 1000)
+    assert b == 3000 and "gpt_1_3b[1:9]" in src      # own tensor range preferred
+    b, src = bench.traffic_for(table, "lstm_ptb", 500)
+    assert b == 1000 and "vgg16" in src
+
+
+def test_oracle_timer_on_host_cores():
+    bench, _ = _bench([])
+    from synth.configs import WORKLOADS
+    w = WORKLOADS["resnet20"]
+    cpu = bench.cpu_baseline(w)
+    assert cpu["kind"] == "oracle" and cpu["cores"] >= 1 and cpu["value"] > 0
+    assert cpu["single_thread"]["value"] > 0
+    timer = bench.OracleTimer(w, procs=2)
+    try:
+        secs, elems = timer.run([(p, 3) for p in range(w.P)], step=1)
+    finally:
+        timer.close()
+    assert secs > 0 and elems == w.P * w.sizes[3]
 
 
 def test_tensor_range_slices_the_workload():
