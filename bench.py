@@ -662,20 +662,54 @@ def run_ours(args):
         for p in range(n_host):
             host[p].copy_(grads[0][p])
         w_host = torch.empty(N, dtype=torch.float32, pin_memory=True)
-        dev_g = grads[0]
+        # two device gradient sets when memory allows: step i+1's inputs cross
+        # the host link (copy stream) while step i computes, and step i's
+        # weights go back on a third stream (the link is full duplex)
+        free_b, _ = torch.cuda.mem_get_info(dev)
+        sets = [grads[0]]
+        if free_b > P * N * 4 + (4 << 30):
+            sets.append([torch.empty(N, dtype=torch.float32, device=dev) for _ in range(P)])
+        comp = torch.cuda.current_stream(dev)
+        h2d = torch.cuda.Stream(device=dev)
+        d2h = torch.cuda.Stream(device=dev)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         ke = max(3, min(K, 10))
+        ev_in = [torch.cuda.Event() for _ in range(ke)]
+        ev_done = [torch.cuda.Event() for _ in range(ke)]
+        ev_out = [torch.cuda.Event() for _ in range(ke)]
+
+        def load(i):  # step i's inputs into set i mod 2, once the set is free
+            with torch.cuda.stream(h2d):
+                if i >= len(sets):
+                    h2d.wait_event(ev_done[i - len(sets)])
+                for p in range(P):
+                    sets[i % len(sets)][p].copy_(host[p % n_host], non_blocking=True)
+                ev_in[i].record(h2d)
+
         barrier()
         torch.cuda.synchronize()
-        e0.record()
+        e0.record(comp)
+        h2d.wait_event(e0)
+        d2h.wait_event(e0)
+        load(0)
         for i in range(ke):
-            for p in range(P):
-                dev_g[p].copy_(host[p % n_host], non_blocking=True)
-            plan.sparsify(dev_g, res, w.lr, idx, val)
+            if i + 1 < ke and len(sets) > 1:
+                load(i + 1)
+            comp.wait_event(ev_in[i])
+            plan.sparsify(sets[i % len(sets)], res, w.lr, idx, val)
+            if i >= 1:
+                comp.wait_event(ev_out[i - 1])  # the read-back of the weights is done
             plan.aggregate_apply(idx, val, dense, weights)
-            w_host.copy_(weights, non_blocking=True)
-        e1.record()
+            ev_done[i].record(comp)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(ev_done[i])
+                w_host.copy_(weights, non_blocking=True)
+                ev_out[i].record(d2h)
+            if i + 1 < ke and len(sets) == 1:
+                load(i + 1)
+        comp.wait_event(ev_out[ke - 1])
+        e1.record(comp)
         torch.cuda.synchronize()
         barrier()
         e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
@@ -684,9 +718,12 @@ def run_ours(args):
         e2e = {"value": world * P * N * ke / (float(e_ms.item()) / 1e3) / 1e9,
                "unit": "Gelem/s", "steps": ke, "h2d_bytes_per_step": P * N * 4,
                "d2h_bytes_per_step": N * 4, "pinned_host_buffers": n_host,
-               "path": "per step: P pinned host->device gradient copies, lags_sparsify, "
-                       "lags_aggregate_apply, device->host copy of the updated weights"}
-        del host, w_host
+               "device_input_sets": len(sets),
+               "path": "per step: P pinned host->device gradient copies (the next step's "
+                       "overlapping this step's compute when two device input sets fit), "
+                       "lags_sparsify, lags_aggregate_apply, device->host copy of the "
+                       "updated weights on a third stream"}
+        del host, w_host, sets
 
     # lags_apply alone (outside the step: the step applies the update fused
     # into the aggregation), 12 bytes per element

@@ -199,10 +199,11 @@ LAGS_API lags_status lags_aggregate(lags_plan* plan, const uint32_t* idx, const 
                            float* dense_out, void* stream);
 
 /*
- * lags_aggregate_apply - lags_aggregate followed by lags_apply in one pass
- * over the update: dense_out is written exactly as lags_aggregate writes it and
- * weights end exactly as lags_apply leaves them (entries no worker picked
- * keep their weight, since w - (+0) == w), without reading dense_out back.
+ * lags_aggregate_apply - lags_aggregate followed by lags_apply without a
+ * pass over the whole update: dense_out is written exactly as lags_aggregate
+ * writes it and weights end exactly as lags_apply leaves them, but only the
+ * picked positions of weights are read and written (entries no worker picked
+ * keep their weight, since w - (+0) == w) and dense_out is not read back.
  *   weights    device float[N], 16-byte aligned, updated in place.
  * Other arguments, layout and errors: as lags_aggregate.
  */
@@ -383,8 +384,9 @@ LAGS_API lags_status lags_dense_finish(const float* sum, int64_t N, int32_t num_
 
 /*
  * lags_plan_kernel_launches - how many kernels one lags_sparsify, one
- * lags_aggregate (or lags_aggregate_apply) and one lags_apply call enqueue for
- * this plan (any output pointer may be NULL).
+ * lags_aggregate_apply and one lags_apply call enqueue for this plan (any
+ * output pointer may be NULL); lags_aggregate enqueues one fewer than
+ * lags_aggregate_apply.
  */
 LAGS_API lags_status lags_plan_kernel_launches(const lags_plan* plan, int32_t* sparsify,
                                                int32_t* aggregate, int32_t* apply);

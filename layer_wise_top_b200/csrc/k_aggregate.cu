@@ -9,9 +9,12 @@
 // the group in shared memory; the thread holding the lowest worker's pick of a
 // position finds the other workers' picks of it by binary search and adds them
 // in worker order.  Tiles expected to hold many picks form groups of one and
-// accumulate worker by worker in a shared tile instead.  No atomics, so the
-// result is bit-identical however the grid is scheduled.  With a weights
-// pointer the same kernel also applies the SGD update (weights -= dense).
+// accumulate worker by worker in a shared tile instead.  Either way each tile
+// of the update is composed in shared memory and written once, with aligned
+// 16-byte stores: the kernel streams the dense output at the HBM rate and
+// never writes a position twice.  No atomics, so the result is bit-identical
+// however the grid is scheduled.  With a weights pointer the same kernel also
+// applies the SGD update (weights -= dense) at the picked positions.
 //
 // Pick lists are read through the read-only path (they are inputs; plain
 // loads would be ordered behind the kernels' own scattered stores).
@@ -21,7 +24,6 @@
 // picks.  It also checks that the lists are ascending and inside their layer.
 #include "block_ops.cuh"
 #include "lags_internal.cuh"
-#include "tma.cuh"
 
 namespace lags {
 
@@ -66,108 +68,186 @@ __global__ void __launch_bounds__(256) k_pick_bounds(DevPlan dp, const uint32_t*
     for (uint32_t t = ti + 1; t < ld.tile_end; ++t) first[t] = ld.koff + ld.k;
 }
 
-// Picks of one tile staged in shared memory; a tile with more picks (layers
-// sent at high density by many workers) reads them from global memory.
-constexpr uint32_t kAggPickCap = 2048;
-// Up to this many picks in a tile, the thread holding a position's first pick
-// looks the position up in the other workers' lists (binary search); above it,
-// and when the launch has room for a tile accumulator, the CTA adds the
-// workers' picks into shared memory one worker at a time instead.
+// Up to this many picks in a one-tile group, the thread holding a position's
+// first pick looks the position up in the other workers' lists (binary
+// search); above it the CTA adds the workers' picks into the shared tile one
+// worker at a time instead.
 constexpr uint32_t kAggOwnerMax = 512;
-
-// Zeros the owner path sends to the dense output with bulk stores.
-constexpr uint32_t kAggZeroBytes = 4096;  // keeps 4 tile-accumulator CTAs per SM
+// The shared tile holds one tile of the dense update, placed so that shared
+// index j is element (tile start rounded down to 4) + j: float4 slot v of the
+// tile is then one aligned 16-byte store.  A tile spans at most kTile + 3
+// such positions.
+constexpr uint32_t kAggTileSlots = kTile / 4 + 1;  // float4 slots
+constexpr uint32_t kAggSlotsPerThread = (kAggTileSlots + kAggThreads - 1) / kAggThreads;
 
 struct AggShared {
-  float4 zero[kAggZeroBytes / 16];       // first: 16-byte aligned source of the bulk stores
+  float4 tile[kAggTileSlots];            // first: 16-byte aligned
   uint32_t loc[kAggPickCap];             // pick position inside the group, per worker ascending
   float val[kAggPickCap];
+  uint32_t seen[kTile / 32];             // positions of the current tile picked by some worker
+  uint32_t multi[kTile / 32];            // ... by more than one worker
   uint32_t base[LAGS_MAX_WORKERS + 1];   // first staged pick of each worker
-  uint32_t rng[2 * LAGS_MAX_WORKERS];
+  uint32_t rng[2 * LAGS_MAX_WORKERS];    // each worker's pick slots [a, b) of the group / tile
   uint32_t warp[kAggThreads / 32];
 };
-// Tile accumulator, only in launches that may need it.  A sum that started at
-// +0 is never -0, so acc != 0 tells exactly which positions need the division
-// and the weight update (0 / P == +0 and w - (+0) == w).
-struct AggTileAcc {
-  float acc[kTile];
-};
-// The accumulator follows AggShared in dynamic shared memory and is cleared
-// with 16-byte stores, so it starts on a 128-byte boundary.
-constexpr size_t kAggAccOffset = (sizeof(AggShared) + 127) / 128 * 128;
-static_assert(kAggAccOffset % 16 == 0, "tile accumulator alignment");
 
+__device__ __forceinline__ float f4_get(const float4& v, int j) {
+  return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+}
+
+// Writes tile [start, start + len) of the dense update from the shared tile
+// (positions relative to start & ~3) with aligned 16-byte streaming stores
+// (scalar stores at a tile's unaligned ends) and clears the shared tile behind
+// it.  With `divide`, the tile holds sums: each nonzero sum is divided by P
+// (a sum that started at +0 is never -0, so zero means "no pick": +0 / P = +0
+// and w - (+0) = w) and, with weights, applied to them.  Without `divide` the
+// tile holds finished values and the weights were updated by their owners.
+__device__ __forceinline__ void agg_write_tile(AggShared& sh, uint32_t start, uint32_t len,
+                                               float* __restrict__ dense,
+                                               float* __restrict__ weights, bool divide,
+                                               float fP) {
+  const uint32_t base = start & ~3u, end = start + len;
+  const uint32_t nv = (end - base + 3) / 4;
+  float4 wv[kAggSlotsPerThread];
+  bool upd[kAggSlotsPerThread];
+  // first the quotients (back into the shared tile) and every weight load of
+  // this thread, then the stores (a load issued after stores waits for them)
+#pragma unroll
+  for (uint32_t j = 0; j < kAggSlotsPerThread; ++j) {
+    const uint32_t v = threadIdx.x + j * kAggThreads;
+    upd[j] = false;
+    if (!divide || v >= nv) continue;
+    float4 a = sh.tile[v];
+    // (most slots hold no pick: divide only where a sum is)
+    if ((__float_as_uint(a.x) | __float_as_uint(a.y) | __float_as_uint(a.z) |
+         __float_as_uint(a.w)) == 0u)
+      continue;
+    a.x = a.x != 0.0f ? __fdiv_rn(a.x, fP) : 0.0f;
+    a.y = a.y != 0.0f ? __fdiv_rn(a.y, fP) : 0.0f;
+    a.z = a.z != 0.0f ? __fdiv_rn(a.z, fP) : 0.0f;
+    a.w = a.w != 0.0f ? __fdiv_rn(a.w, fP) : 0.0f;
+    sh.tile[v] = a;
+    // skip only +0: w - (-0) may differ from w
+    upd[j] = weights && (__float_as_uint(a.x) | __float_as_uint(a.y) | __float_as_uint(a.z) |
+                         __float_as_uint(a.w)) != 0u;
+    const uint32_t e0 = base + 4 * v;
+    if (upd[j]) {
+      if (e0 >= start && e0 + 4 <= end) {
+        wv[j] = *reinterpret_cast<const float4*>(weights + e0);
+      } else {
+        float t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (e0 + c >= start && e0 + c < end) t[c] = weights[e0 + c];
+        wv[j] = make_float4(t[0], t[1], t[2], t[3]);
+      }
+    }
+  }
+#pragma unroll
+  for (uint32_t j = 0; j < kAggSlotsPerThread; ++j) {
+    const uint32_t v = threadIdx.x + j * kAggThreads;
+    if (v >= nv) continue;
+    const uint32_t e0 = base + 4 * v;
+    const float4 a = sh.tile[v];
+    sh.tile[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 nw = wv[j];
+    if (upd[j]) {
+      nw.x = __fsub_rn(nw.x, a.x);
+      nw.y = __fsub_rn(nw.y, a.y);
+      nw.z = __fsub_rn(nw.z, a.z);
+      nw.w = __fsub_rn(nw.w, a.w);
+    }
+    if (e0 >= start && e0 + 4 <= end) {
+      __stcs(reinterpret_cast<float4*>(dense + e0), a);
+      if (upd[j]) *reinterpret_cast<float4*>(weights + e0) = nw;
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (e0 + c < start || e0 + c >= end) continue;
+        dense[e0 + c] = f4_get(a, c);
+        if (upd[j] && __float_as_uint(f4_get(a, c)) != 0u) weights[e0 + c] = f4_get(nw, c);
+      }
+    }
+  }
+}
+
+// One CTA per group of consecutive tiles of one layer (the plan sizes groups
+// to about a thousand expected picks).  The CTA loads the group's pick bounds,
+// stages every worker's picks of the group in shared memory and issues the
+// loads of the weights at the picked positions (consumed only at the end, so
+// their latency hides behind the dense stream).  Then, tile by tile:
+//   1. every pick marks its position in a bitmap; a second bitmap marks the
+//      positions that several workers picked;
+//   2. a position picked by one worker gets fl(+0 + v) in the shared tile
+//      from that pick; a position picked by several gets its worker-ordered
+//      sum from the pick of the lowest worker, which looks the position up in
+//      the other workers' staged lists (binary search);
+//   3. the CTA divides the tile by P and writes all of it once, coalesced.
+// The pick that wrote a position (its "owner") writes the quotient itself, so
+// the tile write divides nothing.  With weights, every staged pick leaves a
+// record for k_weight_updates: (position, quotient) for owners, a skip mark
+// for the others; the weights' scattered read-modify-writes then run in a
+// pass of their own instead of slowing the dense stream.  Groups of one
+// high-density tile instead add the workers' picks into the shared tile
+// worker by worker (a barrier between workers), then divide, apply the
+// weights and write.
 __global__ void __launch_bounds__(kAggThreads, 4)
     k_aggregate(DevPlan dp, const uint32_t* __restrict__ idx, const float* __restrict__ val,
-                float* __restrict__ dense, float* __restrict__ weights, bool have_acc) {
+                float* __restrict__ dense, float* __restrict__ weights) {
   extern __shared__ __align__(16) unsigned char agg_smem[];
   AggShared& sh = *reinterpret_cast<AggShared*>(agg_smem);
-  AggTileAcc& ta = *reinterpret_cast<AggTileAcc*>(agg_smem + kAggAccOffset);
   pdl_trigger();
-  // a group of consecutive tiles of one layer: elements [gs, gs + glen)
   const uint2 grp = dp.agg_groups[blockIdx.x];
   const uint32_t t = grp.x, nt = grp.y;
   const TileDesc td0 = dp.tiles[t];
   const TileDesc tdl = dp.tiles[t + nt - 1];
   const LayerDesc ld = dp.layers[td0.layer];
-  const TileDesc td{td0.start, tdl.start + tdl.len - td0.start, td0.layer, 0};
+  const uint32_t gs = td0.start, glen = tdl.start + tdl.len - td0.start;
   const uint32_t P = dp.P;
   const float fP = (float)P;
   const uint64_t K = dp.K;
   const int tid = threadIdx.x;
-  // source of the bulk zero stores (this CTA's own shared memory)
-  for (uint32_t i = tid; i < kAggZeroBytes / 16; i += kAggThreads)
-    sh.zero[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  fence_proxy_async_shared();  // visible to the bulk copies after the next barrier
+  for (uint32_t v = tid; v < kAggTileSlots; v += kAggThreads)
+    sh.tile[v] = make_float4(0.f, 0.f, 0.f, 0.f);
   pdl_wait();
 
+  if (weights && tid == 0) dp.wcnt[blockIdx.x] = 0;  // (the owner path below sets it)
   if (ld.k == ld.d) {
     // dense layer: every worker sent every entry; slot = koff + (e - off)
-    const uint64_t s0 = ld.koff + (td.start - ld.off);
-    for (uint32_t i = tid; i < td.len; i += kAggThreads) {
+    const uint64_t s0 = ld.koff + (gs - ld.off);
+    for (uint32_t i = tid; i < glen; i += kAggThreads) {
       float s = 0.0f;
       for (uint32_t p = 0; p < P; ++p) s = __fadd_rn(s, __ldg(val + p * K + s0 + i));
       const float dv = __fdiv_rn(s, fP);
-      dense[td.start + i] = dv;
-      if (weights) weights[td.start + i] = __fsub_rn(weights[td.start + i], dv);
+      dense[gs + i] = dv;
+      if (weights) weights[gs + i] = __fsub_rn(weights[gs + i], dv);
     }
     return;
   }
 
   const uint32_t kend = ld.koff + ld.k;
-  uint32_t cnt = 0;
-  if (tid < (int)P) {
-    const uint32_t* first = dp.pick_first + (size_t)tid * dp.T;
-    uint32_t a = __ldg(first + t);
-    uint32_t b = (t + nt < ld.tile_end) ? __ldg(first + t + nt) : kend;
-    a = min(max(a, ld.koff), kend);  // keeps a bad pick list inside the layer
-    b = min(max(b, a), kend);
-    sh.rng[2 * tid] = a;
-    sh.rng[2 * tid + 1] = b;
-    cnt = b - a;
-  }
+  // each worker's picks of [first, first + n) tiles (a bad pick list is kept
+  // inside its layer)
+  auto load_bounds = [&](uint32_t first, uint32_t n) -> uint32_t {
+    uint32_t c = 0;
+    if (tid < (int)P) {
+      const uint32_t* f = dp.pick_first + (size_t)tid * dp.T;
+      uint32_t a = __ldg(f + first);
+      uint32_t b = (first + n < ld.tile_end) ? __ldg(f + first + n) : kend;
+      a = min(max(a, ld.koff), kend);
+      b = min(max(b, a), kend);
+      sh.rng[2 * tid] = a;
+      sh.rng[2 * tid + 1] = b;
+      c = b - a;
+    }
+    return c;
+  };
   uint32_t total;
-  const uint32_t before = block_excl_scan<kAggThreads>(cnt, sh.warp, &total);
+  const uint32_t before = block_excl_scan<kAggThreads>(load_bounds(t, nt), sh.warp, &total);
   if (tid < (int)P) sh.base[tid] = before;
   if (tid == 0) sh.base[P] = total;
   __syncthreads();
   const bool staged = total <= kAggPickCap;
-  // the tile accumulator covers one tile: groups of several tiles use the
-  // owner search (the plan groups only tiles expected to hold few picks)
-  const bool owner_path = staged && (total <= kAggOwnerMax || !have_acc || nt > 1);
-  const uint32_t head = min(td.len, (4u - (td.start & 3u)) & 3u);
-  const uint32_t nvec = (td.len - head) / 4;
-  if (owner_path && tid == 0 && nvec > 0) {
-    // the group's 16-byte-aligned middle is cleared by the bulk-copy engine
-    // while the CTA stages and sums its picks; waited for before the sums
-    char* dst = reinterpret_cast<char*>(dense + td.start + head);
-    const uint64_t bytes = (uint64_t)nvec * 16;
-    for (uint64_t o = 0; o < bytes; o += kAggZeroBytes) {
-      const uint64_t n = bytes - o < kAggZeroBytes ? bytes - o : kAggZeroBytes;
-      bulk_store(dst + o, sh.zero, (uint32_t)n);
-    }
-    bulk_commit();
-  }
   auto worker_of = [&](uint32_t i) {  // staged pick i: last worker p with base[p] <= i
     uint32_t p = 0, hi = P - 1;
     while (p < hi) {
@@ -176,166 +256,185 @@ __global__ void __launch_bounds__(kAggThreads, 4)
     }
     return p;
   };
+  constexpr uint32_t OI = kAggPickCap / kAggThreads;  // staged picks per thread
   if (staged) {
-    for (uint32_t i = tid; i < total; i += kAggThreads) {
-      const uint32_t p = worker_of(i);
-      const uint64_t slot = p * K + sh.rng[2 * p] + (i - sh.base[p]);
-      const uint32_t x = __ldg(idx + slot) - td.start;
-      sh.loc[i] = x < td.len ? x : 0xFFFFFFFFu;
-      sh.val[i] = __ldg(val + slot);
+    // all of a thread's loads in flight before the shared stores
+    uint32_t sx[OI];
+    float sv[OI];
+#pragma unroll
+    for (uint32_t j = 0; j < OI; ++j) {
+      const uint32_t i = tid + j * kAggThreads;
+      sx[j] = 0xFFFFFFFFu;
+      sv[j] = 0.0f;
+      if (i < total) {
+        const uint32_t p = worker_of(i);
+        const uint64_t slot = p * K + sh.rng[2 * p] + (i - sh.base[p]);
+        sx[j] = __ldg(idx + slot) - gs;
+        sv[j] = __ldg(val + slot);
+      }
+    }
+#pragma unroll
+    for (uint32_t j = 0; j < OI; ++j) {
+      const uint32_t i = tid + j * kAggThreads;
+      if (i < total) {
+        sh.loc[i] = sx[j] < glen ? sx[j] : 0xFFFFFFFFu;
+        sh.val[i] = sv[j];
+      }
     }
   }
-  if (owner_path) {
-    // ---- few picks: zeros everywhere, then each position's first owner ----
-    // Owned positions, their sums and their old weights are all gathered
-    // before this thread's first store: a load issued after stores waits for
-    // them to drain.
-    __syncthreads();  // staged picks visible to all threads
-    constexpr uint32_t OI = kAggPickCap / kAggThreads;  // staged picks per thread
-    uint32_t own_x[OI];
-    float own_v[OI], own_w[OI];
+  __syncthreads();  // staged picks visible to all threads
+
+  float* tile = reinterpret_cast<float*>(sh.tile);
+  if (staged && (nt > 1 || total <= kAggOwnerMax)) {
+    // this thread's staged picks i = tid + 256 j: position in the group,
+    // worker and the weight there (loaded now, used after the last tile)
+    static_assert(OI == 8 && LAGS_MAX_WORKERS <= 256, "eight 8-bit worker ids per thread");
+    uint32_t px[OI];
+    uint64_t pw = 0;  // byte j: worker of pick j
+    uint32_t own = 0;  // bit j: this thread writes pick j's position
 #pragma unroll
     for (uint32_t j = 0; j < OI; ++j) {
-      own_x[j] = 0xFFFFFFFFu;
-      own_v[j] = 0.0f;
-      own_w[j] = 0.0f;
       const uint32_t i = tid + j * kAggThreads;
-      if (i >= total) continue;
-      const uint32_t x = sh.loc[i];
-      if (x >= td.len) continue;
-      const uint32_t p = worker_of(i);
-      bool first_owner = true;
-      float s = 0.0f;
-      for (uint32_t q = 0; q < P && first_owner; ++q) {
-        if (q == p) {
-          s = __fadd_rn(s, sh.val[i]);
-          continue;
-        }
-        uint32_t a = sh.base[q], b = sh.base[q + 1];
-        while (a < b) {  // lower bound of x in worker q's staged picks
-          const uint32_t m = (a + b) >> 1;
-          if (sh.loc[m] < x) a = m + 1; else b = m;
-        }
-        if (a < sh.base[q + 1] && sh.loc[a] == x) {
-          if (q < p) first_owner = false;
-          else s = __fadd_rn(s, sh.val[a]);
+      px[j] = 0xFFFFFFFFu;
+      if (i < total) {
+        px[j] = sh.loc[i];
+        pw |= (uint64_t)worker_of(i) << (8 * j);
+      }
+    }
+    for (uint32_t q = 0; q < nt; ++q) {
+      const TileDesc tq = nt == 1 ? td0 : dp.tiles[t + q];
+      const uint32_t lo = tq.start - gs;
+      const uint32_t shift = tq.start & 3u;  // shared index of the tile's first element
+      for (uint32_t w = tid; w < kTile / 32; w += kAggThreads) {
+        sh.seen[w] = 0;
+        sh.multi[w] = 0;
+      }
+      __syncthreads();
+      // 1. which positions of the tile do several workers pick?
+#pragma unroll
+      for (uint32_t j = 0; j < OI; ++j) {
+        const uint32_t x = px[j] - lo;
+        if (x < tq.len) {
+          const uint32_t bit = 1u << (x & 31);
+          if (atomicOr(&sh.seen[x >> 5], bit) & bit) atomicOr(&sh.multi[x >> 5], bit);
         }
       }
-      if (first_owner) {
-        own_x[j] = x;
-        own_v[j] = __fdiv_rn(s, fP);
+      __syncthreads();
+      // 2. one pick per position writes its worker-ordered sum
+#pragma unroll
+      for (uint32_t j = 0; j < OI; ++j) {
+        const uint32_t x = px[j] - lo;
+        if (x >= tq.len) continue;
+        const uint32_t i = tid + j * kAggThreads;
+        float s;
+        if (!(sh.multi[x >> 5] & (1u << (x & 31)))) {
+          s = __fadd_rn(0.0f, sh.val[i]);
+        } else {
+          // several workers: the lowest one sums them in worker order
+          const uint32_t p = (uint32_t)(pw >> (8 * j)) & 0xFFu, gx = px[j];
+          bool first_owner = true;
+          s = 0.0f;
+          for (uint32_t r = 0; r < P && first_owner; ++r) {
+            if (r == p) {
+              s = __fadd_rn(s, sh.val[i]);
+              continue;
+            }
+            uint32_t u = sh.base[r], e = sh.base[r + 1];
+            while (u < e) {  // lower bound of gx in worker r's staged picks
+              const uint32_t m = (u + e) >> 1;
+              if (sh.loc[m] < gx) u = m + 1; else e = m;
+            }
+            if (u < sh.base[r + 1] && sh.loc[u] == gx) {
+              if (r < p) first_owner = false;
+              else s = __fadd_rn(s, sh.val[u]);
+            }
+          }
+          if (!first_owner) continue;
+        }
+        const float qv = __fdiv_rn(s, fP);  // (+0 / P = +0)
+        tile[shift + x] = qv;
+        own |= 1u << j;
+        // kept for the weight record in the pick's own value slot (only the
+        // owner ever reads an owner's value)
+        sh.val[i] = qv;
       }
+      __syncthreads();
+      // 3. the whole tile, once
+      agg_write_tile(sh, tq.start, tq.len, dense, nullptr, false, fP);
+      __syncthreads();  // the shared tile is clear again
     }
     if (weights) {
+      // one record per staged pick: owners whose quotient is not +0 (w - (+0)
+      // == w; w - (-0) may differ from w) update their weight
+      uint2* rec = dp.wrec + (size_t)blockIdx.x * kAggPickCap;
 #pragma unroll
-      for (uint32_t j = 0; j < OI; ++j)
-        if (own_x[j] != 0xFFFFFFFFu) own_w[j] = weights[td.start + own_x[j]];
-    }
-    // the unaligned ends of the group (the middle went to the bulk copies)
-    for (uint32_t i = tid; i < head; i += kAggThreads) dense[td.start + i] = 0.0f;
-    for (uint32_t i = head + 4 * nvec + tid; i < td.len; i += kAggThreads) dense[td.start + i] = 0.0f;
-    if (tid == 0 && nvec > 0) {
-      bulk_wait_all();             // the bulk zeros have landed ...
-      fence_proxy_async_global();  // ... and are ordered before generic stores
-    }
-    __syncthreads();  // orders the zeros before the sums written below
-#pragma unroll
-    for (uint32_t j = 0; j < OI; ++j) {
-      if (own_x[j] == 0xFFFFFFFFu) continue;
-      dense[td.start + own_x[j]] = own_v[j];
-      if (weights) weights[td.start + own_x[j]] = __fsub_rn(own_w[j], own_v[j]);
+      for (uint32_t j = 0; j < OI; ++j) {
+        const uint32_t i = tid + j * kAggThreads;
+        if (i >= total) break;
+        const float qj = sh.val[i];
+        const bool upd = ((own >> j) & 1u) && __float_as_uint(qj) != 0u;
+        rec[i] = upd ? make_uint2(gs + px[j], __float_as_uint(qj)) : make_uint2(0xFFFFFFFFu, 0u);
+      }
+      if (tid == 0) dp.wcnt[blockIdx.x] = total;
     }
     return;
   }
 
-  if (have_acc && nt == 1) {
-    // ---- many picks: worker-ordered accumulation in a shared tile ----
-    float4* acc4 = reinterpret_cast<float4*>(ta.acc);
-    for (uint32_t i = tid; i < kTile / 4; i += kAggThreads) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    __syncthreads();
+  // ---- many picks: worker-ordered accumulation in the shared tile, one tile
+  // at a time (a group of one tile with staged picks reads them from shared
+  // memory, otherwise from global memory) ----
+  for (uint32_t q = 0; q < nt; ++q) {
+    const TileDesc tq = nt == 1 ? td0 : dp.tiles[t + q];
+    const uint32_t shift = tq.start & 3u;
+    const bool from_stage = staged && nt == 1;
+    if (!from_stage) {
+      load_bounds(t + q, 1);
+      __syncthreads();
+    }
     for (uint32_t p = 0; p < P; ++p) {
-      if (staged) {
+      if (from_stage) {
         for (uint32_t j = sh.base[p] + tid; j < sh.base[p + 1]; j += kAggThreads) {
           const uint32_t x = sh.loc[j];
-          if (x < td.len) ta.acc[x] = __fadd_rn(ta.acc[x], sh.val[j]);
+          if (x < tq.len) tile[shift + x] = __fadd_rn(tile[shift + x], sh.val[j]);
         }
       } else {
         const uint64_t row = p * K;
         for (uint32_t j = sh.rng[2 * p] + tid; j < sh.rng[2 * p + 1]; j += kAggThreads) {
-          const uint32_t x = __ldg(idx + row + j) - td.start;
-          if (x < td.len) ta.acc[x] = __fadd_rn(ta.acc[x], __ldg(val + row + j));
+          const uint32_t x = __ldg(idx + row + j) - tq.start;
+          if (x < tq.len) tile[shift + x] = __fadd_rn(tile[shift + x], __ldg(val + row + j));
         }
       }
       __syncthreads();
     }
-    auto value_at = [&](uint32_t i) -> float {
-      const float a = ta.acc[i];
-      return a != 0.0f ? __fdiv_rn(a, fP) : 0.0f;
-    };
-    for (uint32_t i = tid; i < head; i += kAggThreads) {
-      const float q = value_at(i);
-      dense[td.start + i] = q;
-      if (weights && __float_as_uint(q) != 0u)  // skip only +0: w - (-0) may differ from w
-        weights[td.start + i] = __fsub_rn(weights[td.start + i], q);
-    }
-    float4* d4 = reinterpret_cast<float4*>(dense + td.start + head);
-    float4* w4 = weights ? reinterpret_cast<float4*>(weights + td.start + head) : nullptr;
-    // a thread's weight loads all go out before its first store (a load
-    // issued after stores waits for them)
-    constexpr uint32_t GV = (kTile / 4 + kAggThreads - 1) / kAggThreads;
-    float4 wv[GV];
-    bool upd[GV];
-#pragma unroll
-    for (uint32_t j = 0; j < GV; ++j) {
-      const uint32_t v = tid + j * kAggThreads, i = head + 4 * v;
-      upd[j] = w4 && v < nvec &&
-               (ta.acc[i] != 0.f || ta.acc[i + 1] != 0.f || ta.acc[i + 2] != 0.f ||
-                ta.acc[i + 3] != 0.f);
-      if (upd[j]) wv[j] = w4[v];  // 16-byte aligned: weights and dense share the layout
-    }
-#pragma unroll
-    for (uint32_t j = 0; j < GV; ++j) {
-      const uint32_t v = tid + j * kAggThreads, i = head + 4 * v;
-      if (v >= nvec) continue;
-      const float4 q = make_float4(value_at(i), value_at(i + 1), value_at(i + 2), value_at(i + 3));
-      __stcs(d4 + v, q);
-      if (upd[j]) {
-        wv[j].x = __fsub_rn(wv[j].x, q.x);
-        wv[j].y = __fsub_rn(wv[j].y, q.y);
-        wv[j].z = __fsub_rn(wv[j].z, q.z);
-        wv[j].w = __fsub_rn(wv[j].w, q.w);
-        w4[v] = wv[j];
-      }
-    }
-    for (uint32_t i = head + 4 * nvec + tid; i < td.len; i += kAggThreads) {
-      const float q = value_at(i);
-      dense[td.start + i] = q;
-      if (weights && __float_as_uint(q) != 0u)  // skip only +0: w - (-0) may differ from w
-        weights[td.start + i] = __fsub_rn(weights[td.start + i], q);
-    }
-    return;
-  }
-
-  // ---- more picks than the stage holds and no tile accumulator: accumulate
-  // worker by worker in the output itself, a barrier between workers ----
-  for (uint32_t i = tid; i < td.len; i += kAggThreads) dense[td.start + i] = 0.0f;
-  __syncthreads();
-  for (uint32_t p = 0; p < P; ++p) {
-    const uint64_t row = p * K;
-    for (uint32_t j = sh.rng[2 * p] + tid; j < sh.rng[2 * p + 1]; j += kAggThreads) {
-      const uint32_t x = __ldg(idx + row + j) - td.start;
-      if (x < td.len) dense[td.start + x] = __fadd_rn(dense[td.start + x], __ldg(val + row + j));
-    }
+    agg_write_tile(sh, tq.start, tq.len, dense, weights, true, fP);
     __syncthreads();
   }
-  for (uint32_t i = tid; i < td.len; i += kAggThreads) {
-    const float s = dense[td.start + i];
-    if (s != 0.0f) {  // +0 stays +0 (0 / P), and w - (+0) == w
-      const float dv = __fdiv_rn(s, fP);
-      dense[td.start + i] = dv;
-      if (weights) weights[td.start + i] = __fsub_rn(weights[td.start + i], dv);
-    }
+}
+
+// The weight updates the aggregation recorded: w = fl32(w - q) at every
+// owner's position, one CTA per aggregation group, every weight load of a
+// thread issued before its stores.
+__global__ void __launch_bounds__(kAggThreads) k_weight_updates(DevPlan dp,
+                                                                 float* __restrict__ weights) {
+  pdl_trigger();
+  pdl_wait();
+  const uint32_t n = dp.wcnt[blockIdx.x];
+  if (n == 0) return;
+  const uint2* rec = dp.wrec + (size_t)blockIdx.x * kAggPickCap;
+  constexpr uint32_t OI = kAggPickCap / kAggThreads;
+  uint2 r[OI];
+  float w[OI];
+#pragma unroll
+  for (uint32_t j = 0; j < OI; ++j) {
+    const uint32_t i = threadIdx.x + j * kAggThreads;
+    r[j] = i < n ? __ldg(rec + i) : make_uint2(0xFFFFFFFFu, 0u);
   }
+#pragma unroll
+  for (uint32_t j = 0; j < OI; ++j)
+    if (r[j].x != 0xFFFFFFFFu) w[j] = weights[r[j].x];
+#pragma unroll
+  for (uint32_t j = 0; j < OI; ++j)
+    if (r[j].x != 0xFFFFFFFFu) weights[r[j].x] = __fsub_rn(w[j], __uint_as_float(r[j].y));
 }
 
 __global__ void __launch_bounds__(256) k_apply(uint32_t first, uint32_t end,
@@ -373,14 +472,17 @@ cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStrea
 
 cudaError_t configure_aggregate() {
   return cudaFuncSetAttribute(k_aggregate, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)(kAggAccOffset + sizeof(AggTileAcc)));
+                              (int)sizeof(AggShared));
 }
 
 cudaError_t launch_aggregate(const DevPlan& dp, const uint32_t* idx, const float* val,
                              float* dense, float* weights, cudaStream_t s) {
-  const size_t smem = dp.agg_tile_acc ? kAggAccOffset + sizeof(AggTileAcc) : sizeof(AggShared);
-  return launch_pdl(k_aggregate, dim3(dp.n_groups), dim3(kAggThreads), smem, s, 1, dp, idx, val,
-                    dense, weights, dp.agg_tile_acc != 0);
+  return launch_pdl(k_aggregate, dim3(dp.n_groups), dim3(kAggThreads), sizeof(AggShared), s, 1,
+                    dp, idx, val, dense, weights);
+}
+
+cudaError_t launch_weight_updates(const DevPlan& dp, float* weights, cudaStream_t s) {
+  return launch_pdl(k_weight_updates, dim3(dp.n_groups), dim3(kAggThreads), 0, s, 1, dp, weights);
 }
 
 cudaError_t launch_apply(uint32_t first, uint32_t end, float* w, const float* dense,

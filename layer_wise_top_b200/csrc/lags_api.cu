@@ -197,14 +197,6 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
     if ((uint64_t)list.size() * ctas * (uint64_t)num_workers <= 148) cap = kSelectStageMax;
     return (uint32_t)std::min<uint64_t>(std::max<uint64_t>(cap, kSelectStageMin), kSelectStageMax);
   };
-  // aggregation: a tile of a sparse layer is expected to hold P * k * kTile / d
-  // picks; past a few hundred, worker-ordered accumulation in a shared tile
-  // beats looking each position up in every worker's list
-  for (uint32_t l : plan->sparse) {
-    const LayerDesc& ld = plan->layers[l];
-    if ((double)num_workers * ld.k * std::min<double>(kTile, ld.d) / ld.d > 256.0)
-      plan->agg_tile_acc = 1;
-  }
   plan->stage_small = stage_for(plan->sel_small, 1);
   plan->stage_large = stage_for(plan->sel_large, kSelectCluster);
   plan->stage_huge = stage_for(plan->sel_huge, kSelectClusterHuge);
@@ -246,6 +238,8 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
   plan->o_chunks = section(cur, (plan->pick_chunks.size() + 1) * sizeof(uint2));
   plan->o_groups = section(cur, (plan->agg_groups.size() + 1) * sizeof(uint2));
   plan->o_first = section(cur, P * T * 4);
+  plan->o_wrec = section(cur, plan->agg_groups.size() * (size_t)kAggPickCap * sizeof(uint2));
+  plan->o_wcnt = section(cur, (plan->agg_groups.size() + 1) * 4);
   plan->o_status = section(cur, kStatusWords * 4);
   plan->agg_ws_bytes = (cur + kAlign - 1) / kAlign * kAlign;
   // what only the selection reads
@@ -387,6 +381,7 @@ lags_status lags_aggregate_apply(lags_plan* plan, const uint32_t* idx, const flo
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = launch_pick_bounds(plan->dp, idx, s);
   if (e == cudaSuccess) e = launch_aggregate(plan->dp, idx, val, dense_out, weights, s);
+  if (e == cudaSuccess) e = launch_weight_updates(plan->dp, weights, s);
   return cuda_status(e);
 }
 
@@ -494,7 +489,7 @@ lags_status lags_plan_kernel_launches(const lags_plan* plan, int32_t* sparsify,
   if (sparsify)
     *sparsify = (any_sparse ? 1 : 0) + 1 + (plan->sel_small.empty() ? 0 : 1) +
                 (plan->sel_large.empty() ? 0 : 1) + (plan->sel_huge.empty() ? 0 : 1);
-  if (aggregate) *aggregate = 2;
+  if (aggregate) *aggregate = 3;  // (lags_aggregate_apply; lags_aggregate enqueues 2)
   if (apply) *apply = 1;
   return LAGS_OK;
 }

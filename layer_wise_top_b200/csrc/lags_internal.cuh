@@ -45,6 +45,10 @@ constexpr uint32_t kSelectStageMax = 20480;  // multiple of 4 (16-byte staged ru
 constexpr uint32_t kSelectSpinLimit = LAGS_STAGE_WAIT_POLLS;  // polls of the staging mbarrier
 
 
+// Picks of one aggregation group staged in shared memory (more: the group
+// takes the worker-ordered accumulation path, reading them from global memory).
+constexpr uint32_t kAggPickCap = 2048;
+
 // Radix digits of the magnitude key (bits 30..0 of the fp32 pattern).
 constexpr int kDigitShift0 = 20;  // level 0: bits 30..20, 2048 bins
 constexpr int kDigitShift1 = 9;   // level 1: bits 19..9,  2048 bins
@@ -103,6 +107,8 @@ struct DevPlan {
   uint32_t* pick_first;       // [P][T] first pick slot of each tile (aggregate)
   const uint2* pick_chunks;   // (sparse layer, first slot) per 256 pick slots
   const uint2* agg_groups;    // (first tile, tiles) per aggregation CTA
+  uint2* wrec;                // [groups][kAggPickCap] (position, quotient) weight updates
+  uint32_t* wcnt;             // [groups] records of each group (0: none)
   uint32_t* status;           // kStatusWords
   uint32_t L, T, P;
   uint32_t n_large, n_small, n_huge, n_sparse, n_chunks, n_groups;
@@ -110,7 +116,6 @@ struct DevPlan {
   uint64_t K;
   uint64_t C;  // candidate slots per worker
   uint32_t stage_small, stage_large, stage_huge;  // select staging capacity per launch
-  uint32_t agg_tile_acc;  // aggregation launches carry a shared tile accumulator
   uint32_t stage_spin;    // polls of the select's first staging wait before it gives up
 };
 
@@ -124,6 +129,7 @@ cudaError_t launch_pick_bounds(const DevPlan& dp, const uint32_t* idx, cudaStrea
 cudaError_t launch_aggregate(const DevPlan& dp, const uint32_t* idx, const float* val,
                              float* dense, float* weights, cudaStream_t s);
 cudaError_t launch_apply(uint32_t first, uint32_t end, float* w, const float* dense, cudaStream_t s);
+cudaError_t launch_weight_updates(const DevPlan& dp, float* weights, cudaStream_t s);
 cudaError_t launch_dense_sum(const DenseGrads& gp, uint32_t P, uint64_t N, float lr, float* sum,
                              cudaStream_t s);
 cudaError_t launch_dense_finish(const float* sum, uint64_t N, uint32_t P, float* dense,

@@ -23,7 +23,8 @@ struct lags_plan {
   // serves a plan that only aggregates)
   size_t o_layers = 0, o_tiles = 0, o_large = 0, o_small = 0, o_huge = 0, o_sparse = 0, o_lo = 0,
          o_cnt = 0,
-         o_cval = 0, o_cidx = 0, o_first = 0, o_chunks = 0, o_groups = 0, o_status = 0,
+         o_cval = 0, o_cidx = 0, o_first = 0, o_chunks = 0, o_groups = 0, o_wrec = 0, o_wcnt = 0,
+         o_status = 0,
          agg_ws_bytes = 0, ws_bytes = 0;
   void* ws = nullptr;
   bool ws_full = false;  // the bound workspace also serves lags_sparsify
@@ -31,7 +32,6 @@ struct lags_plan {
   uint32_t stage_spin = lags::kSelectSpinLimit;  // polls of the select's first staging wait
   cudaEvent_t ev_before = nullptr, ev_after = nullptr;
   uint32_t stage_small = 0, stage_large = 0, stage_huge = 0;  // select staging per launch
-  uint32_t agg_tile_acc = 0;  // some tile expects more picks than the owner search handles
   lags::DevPlan dp{};  // device view once a workspace is bound
 };
 
@@ -54,6 +54,8 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.pick_first = (uint32_t*)(base + plan->o_first);
   dp.pick_chunks = (const uint2*)(base + plan->o_chunks);
   dp.agg_groups = (const uint2*)(base + plan->o_groups);
+  dp.wrec = (uint2*)(base + plan->o_wrec);
+  dp.wcnt = (uint32_t*)(base + plan->o_wcnt);
   dp.status = (uint32_t*)(base + plan->o_status);
   dp.L = (uint32_t)plan->L;
   dp.T = (uint32_t)plan->tiles.size();
@@ -70,7 +72,6 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.stage_small = plan->stage_small;
   dp.stage_large = plan->stage_large;
   dp.stage_huge = plan->stage_huge;
-  dp.agg_tile_acc = plan->agg_tile_acc;
   dp.stage_spin = plan->stage_spin;
 }
 
