@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(256) k_pick_bounds(DevPlan dp, const uint32_t*
   pdl_wait();
   if (j >= ld.k) return;
   const uint64_t i = (uint64_t)ld.koff + j;
-  const uint32_t* pi = idx + (uint64_t)p * dp.K;
+  const uint32_t* pi = after_wait(idx) + (uint64_t)p * dp.K;
   const uint32_t x = __ldg(pi + i);
   const uint32_t lend = ld.off + ld.d;
   if (x < ld.off || x >= lend) {
@@ -84,8 +84,8 @@ struct AggShared {
   float4 tile[kAggTileSlots];            // first: 16-byte aligned
   uint32_t loc[kAggPickCap];             // pick position inside the group, per worker ascending
   float val[kAggPickCap];
-  uint32_t seen[kTile / 32];             // positions of the current tile picked by some worker
-  uint32_t multi[kTile / 32];            // ... by more than one worker
+  uint32_t seen[2][kTile / 32];          // positions of a tile picked by some worker
+  uint32_t multi[2][kTile / 32];         // ... by more than one worker (two sets: tiles alternate)
   uint32_t base[LAGS_MAX_WORKERS + 1];   // first staged pick of each worker
   uint32_t rng[2 * LAGS_MAX_WORKERS];    // each worker's pick slots [a, b) of the group / tile
   uint32_t warp[kAggThreads / 32];
@@ -192,7 +192,7 @@ __device__ __forceinline__ void agg_write_tile(AggShared& sh, uint32_t start, ui
 // worker by worker (a barrier between workers), then divide, apply the
 // weights and write.
 __global__ void __launch_bounds__(kAggThreads, 4)
-    k_aggregate(DevPlan dp, const uint32_t* __restrict__ idx, const float* __restrict__ val,
+    k_aggregate(DevPlan dp, const uint32_t* __restrict__ idx0, const float* __restrict__ val0,
                 float* __restrict__ dense, float* __restrict__ weights) {
   extern __shared__ __align__(16) unsigned char agg_smem[];
   AggShared& sh = *reinterpret_cast<AggShared*>(agg_smem);
@@ -210,6 +210,9 @@ __global__ void __launch_bounds__(kAggThreads, 4)
   for (uint32_t v = tid; v < kAggTileSlots; v += kAggThreads)
     sh.tile[v] = make_float4(0.f, 0.f, 0.f, 0.f);
   pdl_wait();
+  const uint32_t* __restrict__ idx = after_wait(idx0);
+  const float* __restrict__ val = after_wait(val0);
+  const uint32_t* __restrict__ pick_first = after_wait(dp.pick_first);
 
   if (weights && tid == 0) dp.wcnt[blockIdx.x] = 0;  // (the owner path below sets it)
   if (ld.k == ld.d) {
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(kAggThreads, 4)
   auto load_bounds = [&](uint32_t first, uint32_t n) -> uint32_t {
     uint32_t c = 0;
     if (tid < (int)P) {
-      const uint32_t* f = dp.pick_first + (size_t)tid * dp.T;
+      const uint32_t* f = pick_first + (size_t)tid * dp.T;
       uint32_t a = __ldg(f + first);
       uint32_t b = (first + n < ld.tile_end) ? __ldg(f + first + n) : kend;
       a = min(max(a, ld.koff), kend);
@@ -301,25 +304,36 @@ __global__ void __launch_bounds__(kAggThreads, 4)
         pw |= (uint64_t)worker_of(i) << (8 * j);
       }
     }
+    // Two barriers per tile: the bitmaps alternate between tiles (a set is
+    // cleared while the other is in use), and the write of tile q is
+    // separated from the owners' writes of tile q + 1 by that tile's first
+    // barrier.
+    for (uint32_t w = tid; w < kTile / 32; w += kAggThreads) {
+      sh.seen[0][w] = 0;
+      sh.multi[0][w] = 0;
+    }
+    __syncthreads();
     for (uint32_t q = 0; q < nt; ++q) {
       const TileDesc tq = nt == 1 ? td0 : dp.tiles[t + q];
       const uint32_t lo = tq.start - gs;
       const uint32_t shift = tq.start & 3u;  // shared index of the tile's first element
-      for (uint32_t w = tid; w < kTile / 32; w += kAggThreads) {
-        sh.seen[w] = 0;
-        sh.multi[w] = 0;
-      }
-      __syncthreads();
+      uint32_t* seen = sh.seen[q & 1];
+      uint32_t* multi = sh.multi[q & 1];
       // 1. which positions of the tile do several workers pick?
 #pragma unroll
       for (uint32_t j = 0; j < OI; ++j) {
         const uint32_t x = px[j] - lo;
         if (x < tq.len) {
           const uint32_t bit = 1u << (x & 31);
-          if (atomicOr(&sh.seen[x >> 5], bit) & bit) atomicOr(&sh.multi[x >> 5], bit);
+          if (atomicOr(&seen[x >> 5], bit) & bit) atomicOr(&multi[x >> 5], bit);
         }
       }
       __syncthreads();
+      // the other set was last read before this tile's barrier: clear it
+      for (uint32_t w = tid; w < kTile / 32; w += kAggThreads) {
+        sh.seen[(q + 1) & 1][w] = 0;
+        sh.multi[(q + 1) & 1][w] = 0;
+      }
       // 2. one pick per position writes its worker-ordered sum
 #pragma unroll
       for (uint32_t j = 0; j < OI; ++j) {
@@ -327,7 +341,7 @@ __global__ void __launch_bounds__(kAggThreads, 4)
         if (x >= tq.len) continue;
         const uint32_t i = tid + j * kAggThreads;
         float s;
-        if (!(sh.multi[x >> 5] & (1u << (x & 31)))) {
+        if (!(multi[x >> 5] & (1u << (x & 31)))) {
           s = __fadd_rn(0.0f, sh.val[i]);
         } else {
           // several workers: the lowest one sums them in worker order
@@ -359,9 +373,9 @@ __global__ void __launch_bounds__(kAggThreads, 4)
         sh.val[i] = qv;
       }
       __syncthreads();
-      // 3. the whole tile, once
+      // 3. the whole tile, once (clearing it behind; the next tile's owners
+      // write after its first barrier)
       agg_write_tile(sh, tq.start, tq.len, dense, nullptr, false, fP);
-      __syncthreads();  // the shared tile is clear again
     }
     if (weights) {
       // one record per staged pick: owners whose quotient is not +0 (w - (+0)
@@ -418,9 +432,9 @@ __global__ void __launch_bounds__(kAggThreads) k_weight_updates(DevPlan dp,
                                                                  float* __restrict__ weights) {
   pdl_trigger();
   pdl_wait();
-  const uint32_t n = dp.wcnt[blockIdx.x];
+  const uint32_t n = after_wait(dp.wcnt)[blockIdx.x];
   if (n == 0) return;
-  const uint2* rec = dp.wrec + (size_t)blockIdx.x * kAggPickCap;
+  const uint2* rec = after_wait(dp.wrec) + (size_t)blockIdx.x * kAggPickCap;
   constexpr uint32_t OI = kAggPickCap / kAggThreads;
   uint2 r[OI];
   float w[OI];
@@ -444,6 +458,8 @@ __global__ void __launch_bounds__(256) k_apply(uint32_t first, uint32_t end,
   // float4 over the aligned middle, a scalar tail
   pdl_trigger();
   pdl_wait();
+  w = after_wait(w);
+  dense = after_wait(dense);
   const uint32_t a0 = min(end, (first + 3u) & ~3u);
   const uint32_t n4 = (end - a0) / 4;
   const uint32_t gid = blockIdx.x * blockDim.x + threadIdx.x;

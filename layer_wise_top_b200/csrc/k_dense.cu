@@ -23,7 +23,8 @@ __global__ void __launch_bounds__(kDenseThreads) k_dense_sum(DenseGrads gp, uint
                                                              uint64_t N, float lr,
                                                              float* __restrict__ sum) {
   pdl_trigger();
-  pdl_wait();
+  pdl_wait();  // (the gradients come from the caller's work, which does not
+               // trigger dependents early: no read below can precede it)
   const uint64_t n4 = N / 4;
   const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
   const uint64_t gid = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -59,6 +60,7 @@ __global__ void __launch_bounds__(kDenseThreads) k_dense_finish(const float* __r
                                                                 float* __restrict__ weights) {
   pdl_trigger();
   pdl_wait();
+  sum = after_wait(sum);
   const uint64_t n4 = N / 4;
   const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
   const uint64_t gid = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;

@@ -36,33 +36,45 @@ __device__ __forceinline__ float comp(const float4& v, int j) {
 // Three CTAs per SM: the 16 float4 loads of a thread stay in flight together
 // (about 80 registers), which measured 1.2x faster than four CTAs with loads
 // interleaved with arithmetic and than two CTAs with all loads in flight.
+//
+// Warp w owns the contiguous 1024 entries [w * 1024, (w + 1) * 1024) of the
+// tile (lane l takes float4 v * 32 + l of them, so every load and store of a
+// warp covers 512 contiguous bytes).  A warp's candidates are then contiguous
+// in index order, and a candidate's slot is the candidates of the warps before
+// it plus its rank inside its warp: one block barrier per tile, to publish the
+// warps' totals.
 __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, WorkerPtrs wp, float lr,
                                                            uint32_t* __restrict__ out_idx,
                                                            float* __restrict__ out_val) {
   constexpr int V = kEfVecPerThread;
   constexpr int NWARP = kEfThreads / 32;
-  __shared__ uint32_t s_wtot[V * NWARP];  // candidates per (v, warp), v-major
-  __shared__ uint32_t s_base[V * NWARP];
-  __shared__ uint32_t s_total;
+  static_assert(NWARP <= 32, "warp totals fit one warp");
+  __shared__ uint32_t s_wtot[NWARP];  // candidates of each warp
 
   pdl_trigger();
   const uint32_t t = blockIdx.x, p = blockIdx.y;
   const TileDesc td = dp.tiles[t];
   const LayerDesc ld = dp.layers[td.layer];
-  const float* __restrict__ g = wp.g[p];
-  float* __restrict__ r = wp.r[p];
+  const float* g0 = wp.g[p];
+  float* r0 = wp.r[p];
   const uint32_t start = td.start, end = td.start + td.len;
-  const uint32_t base = start & ~3u;
   const uint32_t N = dp.N;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // first element of this thread's float4 v: the warp's run, then lane order
+  const uint32_t wbase = (start & ~3u) + 4u * (uint32_t)(warp * V * 32 + lane);
   pdl_wait();
+  const float* __restrict__ g = after_wait(g0);
+  float* __restrict__ r = after_wait(r0);
+  // the layer's candidate threshold (written by k_estimate): loaded with the
+  // tile, not after it (unused in dense layers, which have none)
+  const uint32_t lo = after_wait(dp.lo_key)[(size_t)p * dp.L + td.layer];
 
   float4 a[V];
   float4 gv[V];
   // every load of the tile is issued before any arithmetic
 #pragma unroll
   for (int v = 0; v < V; ++v) {
-    const uint32_t e0 = base + 4u * (v * kEfThreads + threadIdx.x);
+    const uint32_t e0 = wbase + 128u * v;
     gv[v] = make_float4(0.f, 0.f, 0.f, 0.f);
     a[v] = gv[v];
     if (e0 < end) {
@@ -90,7 +102,7 @@ __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, Worker
     const uint64_t ob = (uint64_t)p * dp.K + ld.koff;
 #pragma unroll
     for (int v = 0; v < V; ++v) {
-      const uint32_t e0 = base + 4u * (v * kEfThreads + threadIdx.x);
+      const uint32_t e0 = wbase + 128u * v;
       if (e0 >= end) continue;
       if (e0 >= start && e0 + 4 <= end) {
         st_stream(r + e0, make_float4(0.f, 0.f, 0.f, 0.f));
@@ -108,12 +120,12 @@ __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, Worker
   }
 
   // sparse layer: write acc back and capture candidates in index order
-  const uint32_t lo = dp.lo_key[(size_t)p * dp.L + td.layer];
   uint32_t masks = 0;
-  uint32_t excl[V];
+  uint32_t excl[V];   // candidates of this warp before this thread's float4 v
+  uint32_t run = 0;   // candidates of this warp in float4s v' < v (warp-uniform)
 #pragma unroll
   for (int v = 0; v < V; ++v) {
-    const uint32_t e0 = base + 4u * (v * kEfThreads + threadIdx.x);
+    const uint32_t e0 = wbase + 128u * v;
     uint32_t m4 = 0;
     if (e0 < end) {
       const bool full = e0 >= start && e0 + 4 <= end;
@@ -129,26 +141,20 @@ __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, Worker
     }
     masks |= m4 << (4 * v);
     const uint32_t c = __popc(m4);
-    excl[v] = 0;
+    excl[v] = run;
     if (__ballot_sync(kFull, c != 0u)) {
       const uint32_t incl = warp_incl_scan(c);
-      excl[v] = incl - c;
-      if (lane == 31) s_wtot[v * NWARP + warp] = incl;
-    } else if (lane == 0) {
-      s_wtot[v * NWARP + warp] = 0;
+      excl[v] = run + incl - c;
+      run += __shfl_sync(kFull, incl, 31);
     }
   }
+  if (lane == 0) s_wtot[warp] = run;
   __syncthreads();
-  if (warp == 0) {
-    // 64 (v, warp) totals, two per lane, scanned in v-major order
-    const uint32_t x0 = s_wtot[2 * lane], x1 = s_wtot[2 * lane + 1];
-    const uint32_t incl = warp_incl_scan(x0 + x1);
-    const uint32_t ex = incl - x0 - x1;
-    s_base[2 * lane] = ex;
-    s_base[2 * lane + 1] = ex + x0;
-    if (lane == 31) s_total = incl;
-  }
-  __syncthreads();
+  // this warp's first slot: the candidates of the warps before it
+  const uint32_t wt = lane < NWARP ? s_wtot[lane] : 0u;
+  const uint32_t wincl = warp_incl_scan(wt);
+  const uint32_t before = __shfl_sync(kFull, wincl - wt, warp);
+  const uint32_t total = __shfl_sync(kFull, wincl, NWARP - 1);
 
   const uint32_t cap = ld.slot_cap;
   const uint64_t slot0 =
@@ -157,8 +163,8 @@ __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, Worker
   for (int v = 0; v < V; ++v) {
     const uint32_t m4 = (masks >> (4 * v)) & 0xFu;
     if (!m4) continue;
-    const uint32_t e0 = base + 4u * (v * kEfThreads + threadIdx.x);
-    uint32_t pos = s_base[v * NWARP + warp] + excl[v];
+    const uint32_t e0 = wbase + 128u * v;
+    uint32_t pos = before + excl[v];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       if (!((m4 >> j) & 1u)) continue;
@@ -169,7 +175,7 @@ __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, Worker
       ++pos;
     }
   }
-  if (threadIdx.x == 0) dp.tile_cnt[(size_t)p * dp.T + t] = s_total;
+  if (threadIdx.x == 0) dp.tile_cnt[(size_t)p * dp.T + t] = total;
 }
 
 cudaError_t launch_ef_capture(const DevPlan& dp, const WorkerPtrs& wp, float lr,

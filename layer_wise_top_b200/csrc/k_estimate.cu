@@ -42,14 +42,16 @@ __global__ void __launch_bounds__(kEstThreads) k_estimate(DevPlan dp, WorkerPtrs
   const uint32_t layer = dp.sparse[blockIdx.x];
   const uint32_t p = blockIdx.y;
   const LayerDesc ld = dp.layers[layer];
-  const float* __restrict__ g = wp.g[p];
-  const float* __restrict__ r = wp.r[p];
+  const float* g0 = wp.g[p];
+  const float* r0 = wp.r[p];
   const uint32_t m = ld.sample;
   const uint32_t run = ld.d > kSampleShortAbove ? kSampleRunShort : kSampleRunLong;
   const uint32_t run_shift = run == kSampleRunShort ? 4 : 6;  // log2(run)
   static_assert(kSampleRunShort == 16 && kSampleRunLong == 64, "run_shift");
   const uint32_t nchunk = m >> run_shift;
   pdl_wait();
+  const float* __restrict__ g = after_wait(g0);
+  const float* __restrict__ r = after_wait(r0);
 
   for (uint32_t i = threadIdx.x; i < kBins; i += kEstThreads) s_hist[i] = 0;
   // sample positions: the whole layer, or nchunk runs of `run` entries spread

@@ -105,8 +105,11 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   const uint32_t p = blockIdx.y;
   const LayerDesc ld = dp.layers[layer];
   const int tid = threadIdx.x, lane = tid & 31;
-  float* __restrict__ r = wp.r[p];
+  float* r0 = wp.r[p];
   pdl_wait();
+  float* __restrict__ r = after_wait(r0);
+  const float* __restrict__ cand_val = after_wait(dp.cand_val);
+  const uint32_t* __restrict__ cand_idx = after_wait(dp.cand_idx);
 
   for (int i = tid; i < (int)kBins; i += NT) {
     sh.hist[i] = 0;
@@ -121,7 +124,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   uint32_t ta = ld.tile_begin + (uint32_t)((uint64_t)nt * rank / CL);
   uint32_t tb = ld.tile_begin + (uint32_t)((uint64_t)nt * (rank + 1) / CL);
   const uint32_t cap = ld.slot_cap;
-  const uint32_t* cnt = dp.tile_cnt + (size_t)p * dp.T;
+  const uint32_t* cnt = after_wait(dp.tile_cnt) + (size_t)p * dp.T;
   uint32_t my = 0, ovf = 0, pad = 0;
   for (uint32_t t = ta + tid; t < tb; t += NT) {
     const uint32_t c = __ldg(cnt + t);
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   // CTA stages its share: the CTA then recompacts that tile's candidates from
   // its acc (held in the residual buffer) instead of copying the slots.  Only
   // an overflow in a share that cannot be staged forces the exhaustive path.
-  const uint32_t lo_key = dp.lo_key[(size_t)p * dp.L + layer];
+  const uint32_t lo_key = after_wait(dp.lo_key)[(size_t)p * dp.L + layer];
   const bool stageable =
       ovf && tb - ta <= kSelectWindow && lo_key >= (1u << 20) && pad <= stage_cap;
   if (tid == 0) {
@@ -246,8 +249,8 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
           const uint32_t in_tile = v - sh.tpre[lo];
           if (in_tile < cap) {
             const uint64_t slot = cbase + (uint64_t)(w0 + lo - ld.tile_begin) * cap + in_tile;
-            idx = __ldg(dp.cand_idx + slot);
-            val = __ldg(dp.cand_val + slot);
+            idx = __ldg(cand_idx + slot);
+            val = __ldg(cand_val + slot);
           } else {
             // an overflowed tile walked from its slots (only after a staging
             // timeout): the slots end at cap, so report and skip the rest
@@ -304,8 +307,8 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
         const uint32_t n = sh.tpre[q + 1] - sh.tpre[q];
         if (n == 0 || __ldg(cnt + ta + q) > cap) continue;
         const uint64_t slot = cbase + (uint64_t)(ta + q - ld.tile_begin) * cap;
-        bulk_load(stage_val + sh.tpre[q], dp.cand_val + slot, n * 4u, &stage_bar);
-        bulk_load(stage_idx + sh.tpre[q], dp.cand_idx + slot, n * 4u, &stage_bar);
+        bulk_load(stage_val + sh.tpre[q], cand_val + slot, n * 4u, &stage_bar);
+        bulk_load(stage_idx + sh.tpre[q], cand_idx + slot, n * 4u, &stage_bar);
       }
       if (ovf) {
         // overflowed tiles: the CTA recompacts the entries with key >= lo_key

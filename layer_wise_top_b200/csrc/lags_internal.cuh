@@ -149,6 +149,20 @@ __device__ __forceinline__ void pdl_trigger() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Data the step's earlier kernels wrote must be read after pdl_wait().  Loads
+// through the read-only path (__ldg) are invariant to the compiler, and the
+// cache-hinted loads are asm without a memory clobber, so either may be moved
+// above the wait; a plain "memory" clobber does not hold them.  Every kernel
+// therefore reads such data through pointers passed through after_wait()
+// behind its pdl_wait(): the compiler learns their value only there, so no
+// load through them can be issued before the wait.
+template <typename T>
+__device__ __forceinline__ T* after_wait(T* p) {
+  uint64_t v = reinterpret_cast<uint64_t>(p);
+  asm volatile("" : "+l"(v));
+  return reinterpret_cast<T*>(v);
+}
+
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t s, int cluster, Args&&... args) {
