@@ -65,6 +65,15 @@ struct Cluster {
       return 0;
     }
   }
+  // split cluster barrier: arrive once this CTA no longer reads its peers'
+  // shared memory, wait before leaving (so no peer's memory goes away while
+  // it is read); no-ops for a single CTA
+  __device__ __forceinline__ static void arrive() {
+    if constexpr (CL > 1) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  }
+  __device__ __forceinline__ static void wait() {
+    if constexpr (CL > 1) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+  }
   template <typename T>
   __device__ __forceinline__ static T* remote(T* p, uint32_t r) {
     if constexpr (CL > 1) {
@@ -550,6 +559,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
     a_run += x[2];
     b_run += x[3];
   }
+  C::arrive();  // the last read of a peer's shared memory (see C::wait below)
 
   // ---- ordered emission: pos = strict_before + min(need, ties_before) ----
   const uint64_t ob = (uint64_t)p * dp.K + ld.koff;
@@ -646,7 +656,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   }
   if (stage_timeout && tid == 0)  // give copies still in flight a bounded chance to land
     mbar_wait_bounded(&stage_bar, 0, kSelectSpinLimit);
-  C::sync();  // no CTA leaves while another may still read its shared memory
+  C::wait();  // no CTA leaves while another may still read its shared memory
 }
 
 // Dynamic shared memory of a select launch staging `cap` candidates.
