@@ -648,16 +648,19 @@ def run_ours(args):
     if graphs is not None:
         step = eager_step  # the e2e leg below times the eager calls
     if not args.no_e2e and dp is None:
-        # one pinned host buffer per worker while they fit in a quarter of the
-        # host's free memory; otherwise workers share buffers in turn (worker p
-        # copies buffer p mod n).  Either way every worker's P*N*4 bytes cross
-        # the host link every step.
+        # one pinned host buffer per worker while they fit in this rank's share
+        # of a quarter of the host's free memory (the ranks of the node split
+        # it); otherwise workers share buffers in turn (worker p copies buffer
+        # p mod n).  Either way every worker's P*N*4 bytes cross the host link
+        # every step.
         try:
             import psutil
             avail = psutil.virtual_memory().available
         except Exception:  # pragma: no cover
             avail = 64 << 30
-        n_host = max(1, min(P, int(avail * 0.25) // (N * 4)))
+        local_ranks = max(1, int(os.environ.get("LOCAL_WORLD_SIZE", str(world))))
+        share = int(avail * 0.25) // local_ranks
+        n_host = max(1, min(P, share // (N * 4)))
         host = [torch.empty(N, dtype=torch.float32, pin_memory=True) for _ in range(n_host)]
         for p in range(n_host):
             host[p].copy_(grads[0][p])

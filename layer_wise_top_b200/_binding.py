@@ -142,6 +142,12 @@ def lags_plan_destroy(plan) -> None:
     _check(_LIB.lags_plan_destroy(plan), "lags_plan_destroy")
 
 
+def raw_plan_destroy():
+    """The C entry point itself, for destructors that may run at interpreter
+    exit (after this module's globals are cleared); its status is ignored."""
+    return _LIB.lags_plan_destroy
+
+
 def lags_plan_info(plan) -> Tuple[int, int, int]:
     n, k, ws = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_size_t()
     _check(_LIB.lags_plan_info(plan, ctypes.byref(n), ctypes.byref(k), ctypes.byref(ws)),

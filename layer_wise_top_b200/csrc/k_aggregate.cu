@@ -260,27 +260,33 @@ __global__ void __launch_bounds__(kAggThreads, 4)
     return p;
   };
   constexpr uint32_t OI = kAggPickCap / kAggThreads;  // staged picks per thread
+  // staged pick i = tid + 256 j belongs to this thread: its position in the
+  // group and its worker stay in registers for the owner path below
+  static_assert(OI == 8 && LAGS_MAX_WORKERS <= 256, "eight 8-bit worker ids per thread");
+  uint32_t px[OI];
+  uint64_t pw = 0;  // byte j: worker of pick j
   if (staged) {
     // all of a thread's loads in flight before the shared stores
-    uint32_t sx[OI];
     float sv[OI];
 #pragma unroll
     for (uint32_t j = 0; j < OI; ++j) {
       const uint32_t i = tid + j * kAggThreads;
-      sx[j] = 0xFFFFFFFFu;
+      px[j] = 0xFFFFFFFFu;
       sv[j] = 0.0f;
       if (i < total) {
         const uint32_t p = worker_of(i);
+        pw |= (uint64_t)p << (8 * j);
         const uint64_t slot = p * K + sh.rng[2 * p] + (i - sh.base[p]);
-        sx[j] = __ldg(idx + slot) - gs;
+        px[j] = __ldg(idx + slot) - gs;
         sv[j] = __ldg(val + slot);
       }
     }
 #pragma unroll
     for (uint32_t j = 0; j < OI; ++j) {
       const uint32_t i = tid + j * kAggThreads;
+      if (px[j] >= glen) px[j] = 0xFFFFFFFFu;  // (a bad pick list stays inside the group)
       if (i < total) {
-        sh.loc[i] = sx[j] < glen ? sx[j] : 0xFFFFFFFFu;
+        sh.loc[i] = px[j];
         sh.val[i] = sv[j];
       }
     }
@@ -289,21 +295,7 @@ __global__ void __launch_bounds__(kAggThreads, 4)
 
   float* tile = reinterpret_cast<float*>(sh.tile);
   if (staged && (nt > 1 || total <= kAggOwnerMax)) {
-    // this thread's staged picks i = tid + 256 j: position in the group,
-    // worker and the weight there (loaded now, used after the last tile)
-    static_assert(OI == 8 && LAGS_MAX_WORKERS <= 256, "eight 8-bit worker ids per thread");
-    uint32_t px[OI];
-    uint64_t pw = 0;  // byte j: worker of pick j
     uint32_t own = 0;  // bit j: this thread writes pick j's position
-#pragma unroll
-    for (uint32_t j = 0; j < OI; ++j) {
-      const uint32_t i = tid + j * kAggThreads;
-      px[j] = 0xFFFFFFFFu;
-      if (i < total) {
-        px[j] = sh.loc[i];
-        pw |= (uint64_t)worker_of(i) << (8 * j);
-      }
-    }
     // Two barriers per tile: the bitmaps alternate between tiles (a set is
     // cleared while the other is in use), and the write of tile q is
     // separated from the owners' writes of tile q + 1 by that tile's first

@@ -37,6 +37,7 @@ class Plan:
                  layer_range: Optional[Tuple[int, int]] = None,
                  aggregate_only: bool = False):
         self.device = torch.device(device if device is not None else "cuda")
+        self._destroy = B.raw_plan_destroy()
         if layer_range is None:
             lb, le = 0, len(layer_sizes)
             self.handle = B.lags_plan_create(layer_sizes, densities, P)
@@ -62,9 +63,12 @@ class Plan:
                                       self.workspace.numel(), _stream(None, self.device))
 
     def __del__(self):
+        # the raw C entry point, held by the instance: at interpreter exit the
+        # binding module's globals may already be gone
         h = getattr(self, "handle", None)
-        if h is not None and h.value:
-            B.lags_plan_destroy(h)
+        destroy = getattr(self, "_destroy", None)
+        if h is not None and h.value and destroy is not None:
+            destroy(h)
             self.handle = None
 
     # ---------------------------------------------------------------- buffers

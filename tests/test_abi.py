@@ -157,3 +157,19 @@ def test_plan_size_limit():
     # a range plan past the limit is rejected too, even if its own layers are small
     with pytest.raises(L.LagsError):
         L.lags_plan_create_range([top, 5], [0.01, 0.5], 1, 1, 2)
+
+
+def test_kernel_launch_counts():
+    # a dense-only plan runs just the fused pass; sparse plans add the
+    # estimate and one select launch per cluster size in use
+    h = L.lags_plan_create([100, 7], [1.0, 1.0], 2)
+    try:
+        assert L.lags_plan_kernel_launches(h) == (1, 3, 1)
+    finally:
+        L.lags_plan_destroy(h)
+    w = WORKLOADS["gpt_1_3b"]  # one-CTA, 8-CTA and 16-CTA selects
+    h = L.lags_plan_create(w.sizes, w.densities, w.P)
+    try:
+        assert L.lags_plan_kernel_launches(h) == (5, 3, 1)
+    finally:
+        L.lags_plan_destroy(h)
