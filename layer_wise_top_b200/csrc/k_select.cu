@@ -22,9 +22,10 @@
 //
 //  1. radix select on the magnitude key (bits 30..20, 19..9, 8..0): every CTA
 //     builds a shared-memory histogram of its share (warp-aggregated with
-//     __match_any_sync), the CTAs add their bins into CTA 0's histogram
-//     through distributed shared memory, and every CTA reads the merged
-//     histogram to pick the bin holding the k-th largest key.  It stops early
+//     __match_any_sync on the exhaustive path), the CTAs add their nonzero
+//     bins into CTA 0's histogram through distributed shared memory, and every
+//     CTA reads the merged histogram into registers to pick the bin holding
+//     the k-th largest key.  It stops early
 //     once a whole bin is taken.  The result is a key prefix (shift s, value
 //     T): entries with key>>s > T are picks, entries with key>>s == T are ties
 //     of which the `need` lowest indices are picks ("lower index wins").
@@ -37,6 +38,7 @@
 #include <cooperative_groups.h>
 
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "block_ops.cuh"
@@ -86,7 +88,6 @@ struct Cluster {
 
 template <int NT>
 struct SelectShared {
-  uint32_t hist[kBins];          // this CTA's histogram (then the merged copy)
   uint32_t tpre[kSelectWindow + 1];
   uint32_t tmp[NT + NT / 32 + 4];
   uint32_t xch[4];               // read by the other CTAs of the cluster
@@ -102,8 +103,10 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
                                                float* __restrict__ out_val) {
   using C = Cluster<CL>;
   __shared__ SelectShared<NT> sh;
-  // CTA 0 of a cluster: cluster-wide histograms, one per level
-  __shared__ uint32_t merged[CL > 1 ? 3 : 1][kBins];
+  // this CTA's histogram of the current radix level
+  __shared__ __align__(16) uint32_t hist[kBins];
+  // CTA 0 of a cluster: the cluster-wide histogram of each level
+  __shared__ __align__(16) uint32_t merged[CL > 1 ? 3 : 1][CL > 1 ? kBins : 4];
   // staged candidates: stage_cap values, then their stage_cap global indices
   extern __shared__ __align__(16) float stage_val[];
   uint32_t* stage_idx = reinterpret_cast<uint32_t*>(stage_val + stage_cap);
@@ -121,9 +124,11 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   const uint32_t* __restrict__ cand_idx = after_wait(dp.cand_idx);
 
   for (int i = tid; i < (int)kBins; i += NT) {
-    sh.hist[i] = 0;
+    hist[i] = 0;
+    if constexpr (CL > 1) {
 #pragma unroll
-    for (int q = 0; q < (CL > 1 ? 3 : 1); ++q) merged[q][i] = 0;
+      for (int q = 0; q < 3; ++q) merged[q][i] = 0;
+    }
   }
 
   // ---- mode: candidate lists or exhaustive ----
@@ -414,8 +419,8 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   };
 
   // One radix level: histogram of digit (key >> dshift) & dmask over the keys
-  // whose prefix key >> mshift equals mval (all keys when mshift == 32),
-  // merged across the cluster into sh.hist.
+  // whose prefix key >> mshift equals mval (all keys when mshift == 32), in
+  // this CTA's hist (cleared for each level after the first).
   // staged share, for the ordered emission: warp w owns the contiguous
   // positions [wb, we) and walks them 32 at a time
   constexpr uint32_t NW = NT / 32;
@@ -425,18 +430,23 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   const unsigned lanes_below = (1u << lane) - 1u;
 
   auto hist_level = [&](int level, int mshift, uint32_t mval, int dshift, uint32_t dmask) {
+    uint32_t* hl = hist;
+    if (level > 0) {  // (the previous level's reads of it ended in its search)
+      for (int i = tid; i < (int)kBins; i += NT) hl[i] = 0;
+      __syncthreads();
+    }
     if (staged) {
       for (uint32_t i = tid; i < my_pad; i += NT) {
         const uint32_t key = mag_key(stage_val[i]);
         if (mshift >= 32 || (key >> mshift) == mval)
-          atomicAdd(&sh.hist[(key >> dshift) & dmask], 1u);
+          atomicAdd(&hl[(key >> dshift) & dmask], 1u);
       }
     } else if (fast) {
       traverse([&](bool valid, uint32_t, float val) {
         // candidates sit in the sparse tail: few collisions
         const uint32_t key = mag_key(val);
         if (valid && (mshift >= 32 || (key >> mshift) == mval))
-          atomicAdd(&sh.hist[(key >> dshift) & dmask], 1u);
+          atomicAdd(&hl[(key >> dshift) & dmask], 1u);
       });
     } else {
       // a whole layer: keys crowd into few bins, add once per warp and bin
@@ -449,26 +459,43 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
           const bool m = base + tid * kExhV + j < eb && (mshift >= 32 || (key >> mshift) == mval);
           const uint32_t dig = m ? ((key >> dshift) & dmask) : 0xFFFFFFFFu;
           const unsigned peers = __match_any_sync(kFull, dig);
-          if (m && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
+          if (m && lane == __ffs(peers) - 1) atomicAdd(&hl[dig], (uint32_t)__popc(peers));
         }
       }
     }
-    __syncthreads();
+  };
+  // The cluster-wide histogram of a level (the CTAs add their nonzero bins
+  // into CTA 0's merged copy through distributed shared memory) and the bin
+  // holding the r-th largest key; thread t reads bins [t PER, t PER + PER)
+  // into registers for the search.
+  auto merge_find = [&](int level, auto nb, uint32_t r) {
+    constexpr int NB = decltype(nb)::value;
+    static_assert(NB % NT == 0 || NT % NB == 0, "bins per thread");
+    constexpr int PER = NB >= NT ? NB / NT : 1;
+    __syncthreads();  // this CTA's histogram is complete
+    const uint32_t* src = hist;
     if constexpr (CL > 1) {
       uint32_t* dst = C::remote(merged[level], 0);
-      for (int i = tid; i < (int)kBins; i += NT) {
-        const uint32_t h = sh.hist[i];
+      for (int i = tid; i < NB; i += NT) {
+        const uint32_t h = hist[i];
         if (h) atomicAdd(dst + i, h);
       }
       C::sync();
-      const uint32_t* src = C::remote(merged[level], 0);
-      for (int i = tid; i < (int)kBins; i += NT) sh.hist[i] = src[i];
-      __syncthreads();
+      src = C::remote(merged[level], 0);
     }
-  };
-  auto clear_hist = [&]() {
-    for (int i = tid; i < (int)kBins; i += NT) sh.hist[i] = 0;
-    __syncthreads();
+    uint32_t h[PER];
+    const int b0 = tid * PER;
+    if constexpr (PER == 4) {
+      const uint4 x = *reinterpret_cast<const uint4*>(src + b0);
+      h[0] = x.x;
+      h[1] = x.y;
+      h[2] = x.z;
+      h[3] = x.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < PER; ++i) h[i] = b0 < NB ? src[b0 + i] : 0u;
+    }
+    return block_find_bin_regs<NT, PER>(h, r, sh.tmp);
   };
 
   // ---- radix select ----
@@ -477,21 +504,19 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   uint32_t fpfx;
   {
     hist_level(0, 32, 0, kDigitShift0, 0x7FFu);
-    BinPick b = block_find_bin<NT, kBins>(sh.hist, rem, sh.tmp);
+    BinPick b = merge_find(0, std::integral_constant<int, kBins>(), rem);
     rem -= b.above;
     fpfx = b.bin;
     fshift = kDigitShift0;
     if (b.count != rem) {
-      clear_hist();
       hist_level(1, kDigitShift0, fpfx, kDigitShift1, 0x7FFu);
-      b = block_find_bin<NT, kBins>(sh.hist, rem, sh.tmp);
+      b = merge_find(1, std::integral_constant<int, kBins>(), rem);
       rem -= b.above;
       fpfx = (fpfx << 11) | b.bin;
       fshift = kDigitShift1;
       if (b.count != rem) {
-        clear_hist();
         hist_level(2, kDigitShift1, fpfx, kDigitShift2, 0x1FFu);
-        b = block_find_bin<NT, 512>(sh.hist, rem, sh.tmp);
+        b = merge_find(2, std::integral_constant<int, 512>(), rem);
         rem -= b.above;
         fpfx = (fpfx << 9) | b.bin;
         fshift = kDigitShift2;
