@@ -199,10 +199,6 @@ __global__ void __launch_bounds__(kAggThreads, 4)
   pdl_trigger();
   const uint2 grp = dp.agg_groups[blockIdx.x];
   const uint32_t t = grp.x, nt = grp.y;
-  const TileDesc td0 = dp.tiles[t];
-  const TileDesc tdl = dp.tiles[t + nt - 1];
-  const LayerDesc ld = dp.layers[td0.layer];
-  const uint32_t gs = td0.start, glen = tdl.start + tdl.len - td0.start;
   const uint32_t P = dp.P;
   const float fP = (float)P;
   const uint64_t K = dp.K;
@@ -213,6 +209,19 @@ __global__ void __launch_bounds__(kAggThreads, 4)
   const uint32_t* __restrict__ idx = after_wait(idx0);
   const float* __restrict__ val = after_wait(val0);
   const uint32_t* __restrict__ pick_first = after_wait(dp.pick_first);
+  // each worker's first picks of the group and of the next tile (addresses
+  // from the group alone) first, the tile and layer descriptors behind them:
+  // a load issued before the dependency wait holds the loads behind the wait
+  uint32_t first_a = 0, first_b = 0;
+  if (tid < (int)P) {
+    const uint32_t* f = pick_first + (size_t)tid * dp.T;
+    first_a = __ldg(f + t);
+    if (t + nt < dp.T) first_b = __ldg(f + t + nt);
+  }
+  const TileDesc td0 = after_wait(dp.tiles)[t];
+  const TileDesc tdl = after_wait(dp.tiles)[t + nt - 1];
+  const LayerDesc ld = after_wait(dp.layers)[td0.layer];
+  const uint32_t gs = td0.start, glen = tdl.start + tdl.len - td0.start;
 
   if (weights && tid == 0) dp.wcnt[blockIdx.x] = 0;  // (the owner path below sets it)
   if (ld.k == ld.d) {
@@ -245,8 +254,17 @@ __global__ void __launch_bounds__(kAggThreads, 4)
     }
     return c;
   };
+  uint32_t c0 = 0;  // this worker's picks of the group (as load_bounds(t, nt))
+  if (tid < (int)P) {
+    uint32_t a = first_a, b = (t + nt < ld.tile_end) ? first_b : kend;
+    a = min(max(a, ld.koff), kend);
+    b = min(max(b, a), kend);
+    sh.rng[2 * tid] = a;
+    sh.rng[2 * tid + 1] = b;
+    c0 = b - a;
+  }
   uint32_t total;
-  const uint32_t before = block_excl_scan<kAggThreads>(load_bounds(t, nt), sh.warp, &total);
+  const uint32_t before = block_excl_scan<kAggThreads>(c0, sh.warp, &total);
   if (tid < (int)P) sh.base[tid] = before;
   if (tid == 0) sh.base[P] = total;
   __syncthreads();

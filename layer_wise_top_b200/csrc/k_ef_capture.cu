@@ -54,7 +54,6 @@ __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, Worker
   pdl_trigger();
   const uint32_t t = blockIdx.x, p = blockIdx.y;
   const TileDesc td = dp.tiles[t];
-  const LayerDesc ld = dp.layers[td.layer];
   const float* g0 = wp.g[p];
   float* r0 = wp.r[p];
   const uint32_t start = td.start, end = td.start + td.len;
@@ -65,9 +64,6 @@ __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, Worker
   pdl_wait();
   const float* __restrict__ g = after_wait(g0);
   float* __restrict__ r = after_wait(r0);
-  // the layer's candidate threshold (written by k_estimate): loaded with the
-  // tile, not after it (unused in dense layers, which have none)
-  const uint32_t lo = after_wait(dp.lo_key)[(size_t)p * dp.L + td.layer];
 
   float4 a[V];
   float4 gv[V];
@@ -89,6 +85,11 @@ __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, Worker
       }
     }
   }
+  // the layer's descriptor and candidate threshold (the threshold written by
+  // k_estimate; unused in dense layers, which have none), behind the loads:
+  // a load issued before the dependency wait holds the loads behind the wait
+  const LayerDesc ld = after_wait(dp.layers)[td.layer];
+  const uint32_t lo = after_wait(dp.lo_key)[(size_t)p * dp.L + td.layer];
 #pragma unroll
   for (int v = 0; v < V; ++v) {
     a[v].x = __fadd_rn(a[v].x, __fmul_rn(lr, gv[v].x));
