@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kAggThreads, 4)
   const uint32_t* __restrict__ pick_first = after_wait(dp.pick_first);
   // each worker's first picks of the group and of the next tile (addresses
   // from the group alone) first, the tile and layer descriptors behind them:
-  // a load issued before the dependency wait holds the loads behind the wait
+  // loads issued before the dependency wait measured to delay the loads after it
   uint32_t first_a = 0, first_b = 0;
   if (tid < (int)P) {
     const uint32_t* f = pick_first + (size_t)tid * dp.T;

@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(kEfThreads, 3) k_ef_capture(DevPlan dp, Worker
   }
   // the layer's descriptor and candidate threshold (the threshold written by
   // k_estimate; unused in dense layers, which have none), behind the loads:
-  // a load issued before the dependency wait holds the loads behind the wait
+  // loads issued before the dependency wait measured to delay the loads after it
   const LayerDesc ld = after_wait(dp.layers)[td.layer];
   const uint32_t lo = after_wait(dp.lo_key)[(size_t)p * dp.L + td.layer];
 #pragma unroll
