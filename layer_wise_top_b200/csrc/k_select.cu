@@ -8,9 +8,12 @@
 // (held in the residual buffer after the fused pass).  Either way the result
 // is the exact top-k of the layer.
 //
-// CL is 1, 8, or 16. 16 is used for layers whose candidates need more shared
-// memory than 8 CTAs hold, and it is a non-portable cluster size used only
-// where the occupancy query says it fits.  Shares are equal tile ranges; a
+// CL is 1, 4, 8, or 16. 4-CTA clusters stage candidate values only (4 bytes
+// instead of 8; the picks' indices are read back from the candidate slots
+// after the emission), which keeps two CTAs per SM for layers whose
+// candidates would otherwise need 8-CTA clusters.  16 is used for layers whose
+// candidates need more shared memory than 8 CTAs hold, and it is a
+// non-portable cluster size used only where the occupancy query says it fits.  Shares are equal tile ranges; a
 // crowded clustered segment (overflow that equal shares cannot stage) is
 // split again into shares of equal candidate counts.
 //
@@ -96,7 +99,7 @@ struct SelectShared {
 
 }  // namespace
 
-template <int CL, int NT>
+template <int CL, int NT, bool VO>
 __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, WorkerPtrs wp, const uint32_t* list,
                                                uint32_t stage_cap,
                                                uint32_t* __restrict__ out_idx,
@@ -107,7 +110,8 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   __shared__ __align__(16) uint32_t hist[kBins];
   // CTA 0 of a cluster: the cluster-wide histogram of each level
   __shared__ __align__(16) uint32_t merged[CL > 1 ? 3 : 1][CL > 1 ? kBins : 4];
-  // staged candidates: stage_cap values, then their stage_cap global indices
+  // staged candidates: stage_cap values, then (unless VO: values only) their
+  // stage_cap global indices
   extern __shared__ __align__(16) float stage_val[];
   uint32_t* stage_idx = reinterpret_cast<uint32_t*>(stage_val + stage_cap);
   __shared__ __align__(8) uint64_t stage_bar;  // completion of the bulk copies
@@ -313,7 +317,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
       sh.tpre[nw] = my_pad;
       mbar_init(&stage_bar, 1);
       mbar_init_fence();
-      if (staged) mbar_arrive_expect_tx(&stage_bar, bulk * 8u);  // before any copy
+      if (staged) mbar_arrive_expect_tx(&stage_bar, bulk * (VO ? 4u : 8u));  // before any copy
     }
     __syncthreads();
     if (staged) {
@@ -322,7 +326,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
         if (n == 0 || __ldg(cnt + ta + q) > cap) continue;
         const uint64_t slot = cbase + (uint64_t)(ta + q - ld.tile_begin) * cap;
         bulk_load(stage_val + sh.tpre[q], cand_val + slot, n * 4u, &stage_bar);
-        bulk_load(stage_idx + sh.tpre[q], cand_idx + slot, n * 4u, &stage_bar);
+        if constexpr (!VO) bulk_load(stage_idx + sh.tpre[q], cand_idx + slot, n * 4u, &stage_bar);
       }
       if (ovf) {
         // overflowed tiles: the CTA recompacts the entries with key >= lo_key
@@ -345,7 +349,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
             if (mag_key(x) >= lo_key) {
               if (at < room) {
                 stage_val[sh.tpre[q] + at] = x;
-                stage_idx[sh.tpre[q] + at] = e0 + j;
+                if constexpr (!VO) stage_idx[sh.tpre[q] + at] = e0 + j;
               }
               ++at;
             }
@@ -354,7 +358,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
           // of the run is padding, never uninitialised shared memory
           for (uint32_t j = min(found, room) + tid; j < room; j += NT) {
             stage_val[sh.tpre[q] + j] = 0.0f;
-            stage_idx[sh.tpre[q] + j] = 0xFFFFFFFFu;
+            if constexpr (!VO) stage_idx[sh.tpre[q] + j] = 0xFFFFFFFFu;
           }
         }
       }
@@ -370,7 +374,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
           const uint32_t real = __ldg(cnt + ta + q);
           for (uint32_t j = sh.tpre[q] + real; j < sh.tpre[q + 1]; ++j) {
             stage_val[j] = 0.0f;
-            stage_idx[j] = 0xFFFFFFFFu;
+            if constexpr (!VO) stage_idx[j] = 0xFFFFFFFFu;
           }
         }
         __syncthreads();
@@ -600,8 +604,9 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   if (staged) {
     // warp rounds of 32 consecutive positions: ballots give each lane its
     // strict and tie ranks, so the pick-list stores are coalesced and no
-    // block barrier is needed; the emitted index replaces the staged value
-    // (0xFFFFFFFF marks "not emitted") for the residual zeroing below
+    // block barrier is needed; the emitted index (VO: the pick's position)
+    // replaces the staged value (0xFFFFFFFF marks "not emitted") for the
+    // residual zeroing (VO: the index lookup) below
     uint32_t at = a_run + (warp_ex >> 16), bt = b_run + (warp_ex & 0xFFFFu);
     for (uint32_t b0 = wb; b0 < we; b0 += 32) {
       const uint32_t i = b0 + lane;
@@ -613,20 +618,84 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
       const uint32_t sb = at + __popc(mst & lanes_below), tb_ = bt + __popc(mti & lanes_below);
       uint32_t mark = 0xFFFFFFFFu;
       if (st || (ti && tb_ < need)) {
-        const uint32_t idx = stage_idx[i];
-        emit(st ? sb + min(need, tb_) : sb + tb_, idx, val, false);
-        mark = idx;
+        const uint32_t pos = st ? sb + min(need, tb_) : sb + tb_;
+        if constexpr (VO) {
+          if (pos < ld.k) {
+            out_val[ob + pos] = val;
+            mark = pos;
+          } else {
+            atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
+          }
+        } else {
+          const uint32_t idx = stage_idx[i];
+          emit(pos, idx, val, false);
+          mark = idx;
+        }
       }
       if (valid) stage_val[i] = __uint_as_float(mark);
       at += __popc(mst);
       bt += __popc(mti);
     }
-    __syncwarp();
-    for (uint32_t i = wb + lane; i < we; i += 32) {
-      const uint32_t x = __float_as_uint(stage_val[i]);
-      if (x == 0xFFFFFFFFu) continue;
-      if (x - ld.off < ld.d) r[x] = 0.0f;  // an emitted index lies in the layer
-      else atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
+    if constexpr (VO) {
+      // the picks' indices, tile by tile (the walks cross the warps' ranges)
+      __syncthreads();
+      const uint32_t nw = tb - ta;
+      // tiles the bulk copies brought: the index of staged entry j of tile q
+      // is in the tile's slot j
+      for (uint32_t q = tid; q < nw; q += NT) {
+        const uint32_t n = __ldg(cnt + ta + q);
+        if (n > cap) continue;
+        const uint64_t slot = cbase + (uint64_t)(ta + q - ld.tile_begin) * cap;
+        const uint32_t b = sh.tpre[q];
+        for (uint32_t j = 0; j < n; ++j) {
+          const uint32_t m = __float_as_uint(stage_val[b + j]);
+          if (m == 0xFFFFFFFFu) continue;
+          const uint32_t x = __ldg(cand_idx + slot + j);
+          out_idx[ob + m] = x;
+          if (x - ld.off < ld.d) r[x] = 0.0f;  // an emitted index lies in the layer
+          else atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
+        }
+      }
+      if (ovf) {
+        // recompacted tiles: the tile's acc walked again in the recompaction's
+        // order (each thread a contiguous run); its j-th entry with key >=
+        // lo_key sits at stage tpre[q] + j.  Only these tiles' residuals are
+        // written here, each after it is read.
+        constexpr uint32_t PT = kTile / NT;
+        for (uint32_t q = 0; q < nw; ++q) {
+          const uint32_t n = __ldg(cnt + ta + q);  // block-uniform
+          if (n <= cap) continue;
+          const TileDesc tq = dp.tiles[ta + q];
+          const uint32_t e0 = tq.start + tid * PT;
+          const uint32_t mine = tid * PT < tq.len ? min(PT, tq.len - tid * PT) : 0u;
+          uint32_t c = 0;
+          for (uint32_t j = 0; j < mine; ++j) c += mag_key(r[e0 + j]) >= lo_key;
+          uint32_t found;
+          uint32_t rank_in = block_excl_scan<NT>(c, sh.tmp, &found);
+          const uint32_t room = sh.tpre[q + 1] - sh.tpre[q];
+          for (uint32_t j = 0; j < mine; ++j) {
+            const float x = r[e0 + j];
+            if (mag_key(x) >= lo_key) {
+              if (rank_in < room) {
+                const uint32_t m = __float_as_uint(stage_val[sh.tpre[q] + rank_in]);
+                if (m != 0xFFFFFFFFu) {
+                  out_idx[ob + m] = e0 + j;
+                  r[e0 + j] = 0.0f;
+                }
+              }
+              ++rank_in;
+            }
+          }
+        }
+      }
+    } else {
+      __syncwarp();
+      for (uint32_t i = wb + lane; i < we; i += 32) {
+        const uint32_t x = __float_as_uint(stage_val[i]);
+        if (x == 0xFFFFFFFFu) continue;
+        if (x - ld.off < ld.d) r[x] = 0.0f;  // an emitted index lies in the layer
+        else atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
+      }
     }
   } else if (fast) {
     traverse([&](bool valid, uint32_t idx, float val) {
@@ -684,21 +753,28 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   C::wait();  // no CTA leaves while another may still read its shared memory
 }
 
-// Dynamic shared memory of a select launch staging `cap` candidates.
-inline size_t stage_smem_bytes(uint32_t cap) { return (size_t)cap * 8; }
+// Dynamic shared memory of a select launch staging `cap` candidates (values
+// and indices, or values only).
+inline size_t stage_smem_bytes(uint32_t cap, bool values_only = false) {
+  return (size_t)cap * (values_only ? 4 : 8);
+}
 
 cudaError_t configure_select() {
   const int most = (int)stage_smem_bytes(kSelectStageMax);
-  cudaError_t e = cudaFuncSetAttribute(k_select<1, kSelectThreadsSmall>,
+  cudaError_t e = cudaFuncSetAttribute(k_select<1, kSelectThreadsSmall, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, most);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_select<kSelectCluster, kSelectThreads>,
+    e = cudaFuncSetAttribute(k_select<kSelectCluster, kSelectThreads, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, most);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_select<kSelectClusterHuge, kSelectThreads>,
+    e = cudaFuncSetAttribute(k_select<kSelectClusterMid, kSelectThreads, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)stage_smem_bytes(kSelectStageMaxValues, true));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_select<kSelectClusterHuge, kSelectThreads, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, most);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_select<kSelectClusterHuge, kSelectThreads>,
+    e = cudaFuncSetAttribute(k_select<kSelectClusterHuge, kSelectThreads, false>,
                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   return e;
 }
@@ -732,7 +808,7 @@ bool huge_clusters_fit(size_t smem) {
   cfg.numAttrs = 1;
   int clusters = 0;
   const cudaError_t e = cudaOccupancyMaxActiveClusters(
-      &clusters, k_select<kSelectClusterHuge, kSelectThreads>, &cfg);
+      &clusters, k_select<kSelectClusterHuge, kSelectThreads, false>, &cfg);
   if (e != cudaSuccess) cudaGetLastError();  // clear; use 8-CTA clusters instead
   const bool fit = e == cudaSuccess && clusters > 0;
   cache[dev].push_back(Fit{smem, fit});
@@ -743,13 +819,20 @@ bool huge_clusters_fit(size_t smem) {
 cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out_idx,
                           float* out_val, cudaStream_t s) {
   if (dp.n_small) {
-    cudaError_t e = launch_pdl(k_select<1, kSelectThreadsSmall>, dim3(dp.n_small, dp.P),
+    cudaError_t e = launch_pdl(k_select<1, kSelectThreadsSmall, false>, dim3(dp.n_small, dp.P),
                                dim3(kSelectThreadsSmall), stage_smem_bytes(dp.stage_small), s, 1,
                                dp, wp, dp.sel_small, dp.stage_small, out_idx, out_val);
     if (e != cudaSuccess) return e;
   }
+  if (dp.n_mid) {
+    cudaError_t e = launch_pdl(k_select<kSelectClusterMid, kSelectThreads, true>,
+                               dim3(dp.n_mid * kSelectClusterMid, dp.P), dim3(kSelectThreads),
+                               stage_smem_bytes(dp.stage_mid, true), s, kSelectClusterMid, dp, wp,
+                               dp.sel_mid, dp.stage_mid, out_idx, out_val);
+    if (e != cudaSuccess) return e;
+  }
   if (dp.n_large) {
-    cudaError_t e = launch_pdl(k_select<kSelectCluster, kSelectThreads>,
+    cudaError_t e = launch_pdl(k_select<kSelectCluster, kSelectThreads, false>,
                                dim3(dp.n_large * kSelectCluster, dp.P), dim3(kSelectThreads),
                                stage_smem_bytes(dp.stage_large), s, kSelectCluster, dp, wp,
                                dp.sel_large, dp.stage_large, out_idx, out_val);
@@ -758,12 +841,12 @@ cudaError_t launch_select(const DevPlan& dp, const WorkerPtrs& wp, uint32_t* out
   if (dp.n_huge) {
     const size_t smem = stage_smem_bytes(dp.stage_huge);
     if (huge_clusters_fit(smem))
-      return launch_pdl(k_select<kSelectClusterHuge, kSelectThreads>,
+      return launch_pdl(k_select<kSelectClusterHuge, kSelectThreads, false>,
                         dim3(dp.n_huge * kSelectClusterHuge, dp.P), dim3(kSelectThreads), smem, s,
                         kSelectClusterHuge, dp, wp, dp.sel_huge, dp.stage_huge, out_idx, out_val);
     // 8-CTA clusters with the same staging: shares that do not fit are read
     // from global memory on every pass (slower, same result)
-    return launch_pdl(k_select<kSelectCluster, kSelectThreads>,
+    return launch_pdl(k_select<kSelectCluster, kSelectThreads, false>,
                       dim3(dp.n_huge * kSelectCluster, dp.P), dim3(kSelectThreads), smem, s,
                       kSelectCluster, dp, wp, dp.sel_huge, dp.stage_huge, out_idx, out_val);
   }

@@ -163,10 +163,17 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
       plan->sparse.push_back((uint32_t)l);
       for (uint64_t j0 = 0; j0 < k; j0 += 256) plan->pick_chunks.push_back(make_uint2(l, j0));
       // one CTA when its shared memory can stage the expected candidates with
-      // a third to spare, else an 8-CTA cluster, else a 16-CTA cluster
+      // a third to spare, else a 4-CTA cluster staging values only, else an
+      // 8-CTA cluster, else a 16-CTA cluster
       const double expect = expected_candidates(ld);
       auto fits = [&](int ctas) { return 1.33 * expect / ctas + 512.0 <= (double)kSelectStageMax; };
-      (fits(1) ? plan->sel_small : fits(kSelectCluster) ? plan->sel_large : plan->sel_huge)
+      const bool fits_values =
+          1.33 * expect / kSelectClusterMid + 512.0 <= (double)kSelectStageMaxValues &&
+          (ld.tile_end - ld.tile_begin + kSelectClusterMid - 1) / kSelectClusterMid <= kSelectWindow;
+      (fits(1)         ? plan->sel_small
+       : fits_values   ? plan->sel_mid
+       : fits(kSelectCluster) ? plan->sel_large
+                              : plan->sel_huge)
           .push_back((uint32_t)l);
     }
     if (slots >= (1ull << 32) || koff + k >= (1ull << 32)) {
@@ -182,7 +189,8 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
   }
   // staging capacity of each select launch: 1.5x the largest expected
   // candidate count of one CTA (the sample rank scaled to the layer) plus 512
-  auto stage_for = [plan, num_workers](const std::vector<uint32_t>& list, uint32_t ctas) {
+  auto stage_for = [plan, num_workers](const std::vector<uint32_t>& list, uint32_t ctas,
+                                       uint32_t most_entries) {
     double most = 0.0;
     for (uint32_t l : list) {
       const LayerDesc& ld = plan->layers[l];
@@ -194,12 +202,13 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
     // a launch whose CTAs all run at once with one per SM (148 SMs) gives each
     // the largest stage at no cost: crowded segments (a global top-k over
     // tensors of different scales) then stay on the candidate lists
-    if ((uint64_t)list.size() * ctas * (uint64_t)num_workers <= 148) cap = kSelectStageMax;
-    return (uint32_t)std::min<uint64_t>(std::max<uint64_t>(cap, kSelectStageMin), kSelectStageMax);
+    if ((uint64_t)list.size() * ctas * (uint64_t)num_workers <= 148) cap = most_entries;
+    return (uint32_t)std::min<uint64_t>(std::max<uint64_t>(cap, kSelectStageMin), most_entries);
   };
-  plan->stage_small = stage_for(plan->sel_small, 1);
-  plan->stage_large = stage_for(plan->sel_large, kSelectCluster);
-  plan->stage_huge = stage_for(plan->sel_huge, kSelectClusterHuge);
+  plan->stage_small = stage_for(plan->sel_small, 1, kSelectStageMax);
+  plan->stage_mid = stage_for(plan->sel_mid, kSelectClusterMid, kSelectStageMaxValues);
+  plan->stage_large = stage_for(plan->sel_large, kSelectCluster, kSelectStageMax);
+  plan->stage_huge = stage_for(plan->sel_huge, kSelectClusterHuge, kSelectStageMax);
   // aggregation groups: consecutive tiles of one layer, about a thousand
   // expected picks (P k / d per element) per group and at most 16 tiles, but
   // never so few groups that the GPU has fewer than 8 per SM (grouping only
@@ -224,6 +233,7 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
     return plan->layers[a].k != plan->layers[b].k ? plan->layers[a].k > plan->layers[b].k : a < b;
   };
   std::sort(plan->sel_large.begin(), plan->sel_large.end(), by_k_desc);
+  std::sort(plan->sel_mid.begin(), plan->sel_mid.end(), by_k_desc);
   std::sort(plan->sel_huge.begin(), plan->sel_huge.end(), by_k_desc);
   std::sort(plan->sel_small.begin(), plan->sel_small.end(), by_k_desc);
   std::sort(plan->sparse.begin(), plan->sparse.end(), by_k_desc);
@@ -244,6 +254,7 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
   plan->agg_ws_bytes = (cur + kAlign - 1) / kAlign * kAlign;
   // what only the selection reads
   plan->o_large = section(cur, (plan->sel_large.size() + 1) * 4);
+  plan->o_mid = section(cur, (plan->sel_mid.size() + 1) * 4);
   plan->o_small = section(cur, (plan->sel_small.size() + 1) * 4);
   plan->o_huge = section(cur, (plan->sel_huge.size() + 1) * 4);
   plan->o_sparse = section(cur, (plan->sparse.size() + 1) * 4);
@@ -311,6 +322,7 @@ lags_status lags_plan_set_workspace(lags_plan* plan, void* workspace, size_t byt
   if (e == cudaSuccess) e = up(plan->o_tiles, plan->tiles.data(), plan->tiles.size() * sizeof(TileDesc));
   if (full) {
     if (e == cudaSuccess) e = up(plan->o_large, plan->sel_large.data(), plan->sel_large.size() * 4);
+    if (e == cudaSuccess) e = up(plan->o_mid, plan->sel_mid.data(), plan->sel_mid.size() * 4);
     if (e == cudaSuccess) e = up(plan->o_small, plan->sel_small.data(), plan->sel_small.size() * 4);
     if (e == cudaSuccess) e = up(plan->o_huge, plan->sel_huge.data(), plan->sel_huge.size() * 4);
     if (e == cudaSuccess) e = up(plan->o_sparse, plan->sparse.data(), plan->sparse.size() * 4);
@@ -488,7 +500,8 @@ lags_status lags_plan_kernel_launches(const lags_plan* plan, int32_t* sparsify,
   const bool any_sparse = !plan->sparse.empty();
   if (sparsify)
     *sparsify = (any_sparse ? 1 : 0) + 1 + (plan->sel_small.empty() ? 0 : 1) +
-                (plan->sel_large.empty() ? 0 : 1) + (plan->sel_huge.empty() ? 0 : 1);
+                (plan->sel_large.empty() ? 0 : 1) + (plan->sel_huge.empty() ? 0 : 1) +
+                (plan->sel_mid.empty() ? 0 : 1);
   if (aggregate) *aggregate = 3;  // (lags_aggregate_apply; lags_aggregate enqueues 2)
   if (apply) *apply = 1;
   return LAGS_OK;

@@ -31,6 +31,10 @@ constexpr uint32_t kEstThreads = 512;
 // Cluster size used to select layers whose expected candidates exceed what one
 // CTA stages in shared memory; the other layers use one CTA.
 constexpr int kSelectCluster = 8;
+// Layers whose expected candidates 4 CTAs stage as values only (4 bytes each;
+// the indices are read back from the candidate slots for the picks) use a
+// 4-CTA cluster instead: twice the clusters resident of the 8-CTA launch.
+constexpr int kSelectClusterMid = 4;
 // Layers whose expected candidates exceed what 8 CTAs stage use a 16-CTA
 // cluster (a non-portable size; checked on the device before use).
 constexpr int kSelectClusterHuge = 16;
@@ -42,6 +46,9 @@ constexpr uint32_t kSelectWindow = 2048;  // tiles whose prefix sits in smem at 
 // reads them from global memory on every pass instead.
 constexpr uint32_t kSelectStageMin = 1024;
 constexpr uint32_t kSelectStageMax = 20480;  // multiple of 4 (16-byte staged runs)
+// Values-only stage of the 4-CTA launch: two CTAs per SM with the kernel's
+// static shared memory (multiple of 256).
+constexpr uint32_t kSelectStageMaxValues = 17408;
 constexpr uint32_t kSelectSpinLimit = LAGS_STAGE_WAIT_POLLS;  // polls of the staging mbarrier
 
 
@@ -97,6 +104,7 @@ struct DevPlan {
   const LayerDesc* layers;
   const TileDesc* tiles;
   const uint32_t* sel_large;  // sparse layers selected by an 8-CTA cluster
+  const uint32_t* sel_mid;    // sparse layers selected by a 4-CTA cluster (values staged)
   const uint32_t* sel_huge;   // sparse layers selected by a 16-CTA cluster
   const uint32_t* sel_small;  // sparse layers selected by one CTA
   const uint32_t* sparse;     // all sparse layers (estimate pass)
@@ -111,11 +119,11 @@ struct DevPlan {
   uint32_t* wcnt;             // [groups] records of each group (0: none)
   uint32_t* status;           // kStatusWords
   uint32_t L, T, P;
-  uint32_t n_large, n_small, n_huge, n_sparse, n_chunks, n_groups;
+  uint32_t n_large, n_small, n_huge, n_mid, n_sparse, n_chunks, n_groups;
   uint32_t N;
   uint64_t K;
   uint64_t C;  // candidate slots per worker
-  uint32_t stage_small, stage_large, stage_huge;  // select staging capacity per launch
+  uint32_t stage_small, stage_large, stage_huge, stage_mid;  // select staging per launch
   uint32_t stage_spin;    // polls of the select's first staging wait before it gives up
 };
 

@@ -14,14 +14,15 @@ struct lags_plan {
   uint64_t N0 = 0, N = 0, K = 0, C = 0;  // elements [N0, N) of the model; K picks per worker
   std::vector<lags::LayerDesc> layers;
   std::vector<lags::TileDesc> tiles;
-  std::vector<uint32_t> sel_large, sel_small, sel_huge, sparse;
+  std::vector<uint32_t> sel_large, sel_small, sel_huge, sel_mid, sparse;
   std::vector<uint2> pick_chunks;  // (sparse layer, first slot) per 256 pick slots
   std::vector<uint2> agg_groups;   // (first tile, tiles) per aggregation CTA
   std::vector<int64_t> off, k, koff;
   // workspace sections (byte offsets)
   // (the sections aggregation uses come first: a workspace of agg_ws_bytes
   // serves a plan that only aggregates)
-  size_t o_layers = 0, o_tiles = 0, o_large = 0, o_small = 0, o_huge = 0, o_sparse = 0, o_lo = 0,
+  size_t o_layers = 0, o_tiles = 0, o_large = 0, o_small = 0, o_huge = 0, o_mid = 0, o_sparse = 0,
+         o_lo = 0,
          o_cnt = 0,
          o_cval = 0, o_cidx = 0, o_first = 0, o_chunks = 0, o_groups = 0, o_wrec = 0, o_wcnt = 0,
          o_status = 0,
@@ -31,7 +32,7 @@ struct lags_plan {
   int device = -1;
   uint32_t stage_spin = lags::kSelectSpinLimit;  // polls of the select's first staging wait
   cudaEvent_t ev_before = nullptr, ev_after = nullptr;
-  uint32_t stage_small = 0, stage_large = 0, stage_huge = 0;  // select staging per launch
+  uint32_t stage_small = 0, stage_large = 0, stage_huge = 0, stage_mid = 0;  // select staging per launch
   lags::DevPlan dp{};  // device view once a workspace is bound
 };
 
@@ -44,6 +45,7 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.layers = (const LayerDesc*)(base + plan->o_layers);
   dp.tiles = (const TileDesc*)(base + plan->o_tiles);
   dp.sel_large = (const uint32_t*)(base + plan->o_large);
+  dp.sel_mid = (const uint32_t*)(base + plan->o_mid);
   dp.sel_small = (const uint32_t*)(base + plan->o_small);
   dp.sel_huge = (const uint32_t*)(base + plan->o_huge);
   dp.sparse = (const uint32_t*)(base + plan->o_sparse);
@@ -61,6 +63,7 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.T = (uint32_t)plan->tiles.size();
   dp.P = (uint32_t)plan->P;
   dp.n_large = (uint32_t)plan->sel_large.size();
+  dp.n_mid = (uint32_t)plan->sel_mid.size();
   dp.n_small = (uint32_t)plan->sel_small.size();
   dp.n_huge = (uint32_t)plan->sel_huge.size();
   dp.n_sparse = (uint32_t)plan->sparse.size();
@@ -71,6 +74,7 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.C = plan->C;
   dp.stage_small = plan->stage_small;
   dp.stage_large = plan->stage_large;
+  dp.stage_mid = plan->stage_mid;
   dp.stage_huge = plan->stage_huge;
   dp.stage_spin = plan->stage_spin;
 }

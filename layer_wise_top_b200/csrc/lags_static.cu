@@ -117,6 +117,7 @@ extern "C" lags_status lags_sparsify_static(lags_plan* plan, const float* const*
   cudaError_t e = up(plan->o_layers, plan->layers.data(), plan->layers.size() * sizeof(LayerDesc));
   if (e == cudaSuccess) e = up(plan->o_tiles, plan->tiles.data(), plan->tiles.size() * sizeof(TileDesc));
   if (e == cudaSuccess) e = up(plan->o_large, plan->sel_large.data(), plan->sel_large.size() * 4);
+  if (e == cudaSuccess) e = up(plan->o_mid, plan->sel_mid.data(), plan->sel_mid.size() * 4);
   if (e == cudaSuccess) e = up(plan->o_small, plan->sel_small.data(), plan->sel_small.size() * 4);
   if (e == cudaSuccess) e = up(plan->o_huge, plan->sel_huge.data(), plan->sel_huge.size() * 4);
   if (e == cudaSuccess) e = up(plan->o_sparse, plan->sparse.data(), plan->sparse.size() * 4);

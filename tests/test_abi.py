@@ -167,7 +167,7 @@ def test_kernel_launch_counts():
         assert L.lags_plan_kernel_launches(h) == (1, 3, 1)
     finally:
         L.lags_plan_destroy(h)
-    w = WORKLOADS["gpt_1_3b"]  # one-CTA, 8-CTA and 16-CTA selects
+    w = WORKLOADS["gpt_1_3b"]  # one-CTA, 4-CTA and 16-CTA selects
     h = L.lags_plan_create(w.sizes, w.densities, w.P)
     try:
         assert L.lags_plan_kernel_launches(h) == (5, 3, 1)

@@ -47,10 +47,21 @@ def test_ragged_layers_mixed_density(dist):
 
 
 def test_large_layers_cluster_select():
-    # k >= 4096 selects with an 8-CTA cluster, smaller k with one CTA
+    # up to ~15k expected candidates: one-CTA selects
     sizes = [1_100_003, 5, 2_000_001, 1 << 20]
     dens = [0.001, 1.0, 0.003, 0.01]
     w = WORKLOADS["lstm_ptb"].scaled("big", P=2, steps=3,
+                                     tensors=[Tensor(f"t{i}", (d,)) for i, d in enumerate(sizes)])
+    run_full_compare(sizes, dens, 2, w.lr, 3, synth_grad_fn(w),
+                     expect_fallbacks=lambda fb: fb == 0)
+
+
+def test_four_and_eight_cta_cluster_select():
+    # ~49k expected candidates: a 4-CTA cluster staging values only (the picks'
+    # indices read back from the candidate slots); ~57k: an 8-CTA cluster
+    sizes = [2_000_001, 3, 4_000_037, 129]
+    dens = [0.02, 1.0, 0.01, 0.5]
+    w = WORKLOADS["lstm_ptb"].scaled("mid", P=2, steps=3,
                                      tensors=[Tensor(f"t{i}", (d,)) for i, d in enumerate(sizes)])
     run_full_compare(sizes, dens, 2, w.lr, 3, synth_grad_fn(w),
                      expect_fallbacks=lambda fb: fb == 0)
@@ -152,9 +163,10 @@ SAMPLED = {
 BIG = {
     "vgg16": ([16], 10),          # conv8 3x3x512x512, k = 2360 (one-CTA select)
     "resnet50": ([132], 10),      # layer4.0.conv2, k = 2360
-    "lstm_ptb": ([1], 3),         # lstm0.weight 6000x3000, k = 18000 (8-CTA cluster)
+    "lstm_ptb": ([1], 3),         # lstm0.weight 6000x3000, k = 18000 (4-CTA cluster)
     "gpt_1_3b": ([0, 7], 2),      # wte 50304x2048, k = 103,023 (16-CTA cluster, short
                                   # sample runs); h0.mlp.fc1 8192x2048, k = 16,778
+                                  # (4-CTA cluster)
 }
 
 
