@@ -187,6 +187,14 @@ lags_status lags_plan_create_range(const int64_t* layer_sizes, const double* den
     off += (uint64_t)d;
     koff += k;
   }
+  // 4-CTA clusters only pay when their launch fills the GPU (one CTA per SM
+  // at least); fewer clusters keep more CTAs per layer with 8-CTA clusters
+  // (VGG-16's whole-model segments: 0.742 vs 0.631 ms per step)
+  if (!plan->sel_mid.empty() &&
+      plan->sel_mid.size() * (uint64_t)num_workers * kSelectClusterMid < 148) {
+    plan->sel_large.insert(plan->sel_large.end(), plan->sel_mid.begin(), plan->sel_mid.end());
+    plan->sel_mid.clear();
+  }
   // staging capacity of each select launch: 1.5x the largest expected
   // candidate count of one CTA (the sample rank scaled to the layer) plus 512
   auto stage_for = [plan, num_workers](const std::vector<uint32_t>& list, uint32_t ctas,

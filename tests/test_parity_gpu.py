@@ -56,12 +56,23 @@ def test_large_layers_cluster_select():
                      expect_fallbacks=lambda fb: fb == 0)
 
 
-def test_four_and_eight_cta_cluster_select():
-    # ~49k expected candidates: a 4-CTA cluster staging values only (the picks'
-    # indices read back from the candidate slots); ~57k: an 8-CTA cluster
-    sizes = [2_000_001, 3, 4_000_037, 129]
-    dens = [0.02, 1.0, 0.01, 0.5]
-    w = WORKLOADS["lstm_ptb"].scaled("mid", P=2, steps=3,
+def test_four_cta_values_only_cluster_select():
+    # ~23k expected candidates per layer: 4-CTA clusters staging values only
+    # (the picks' indices read back from the candidate slots); 19 layers x 2
+    # workers make the launch fill the GPU (at least one CTA per SM)
+    sizes = [400_003 + 977 * i for i in range(19)] + [3]
+    dens = [0.05] * 19 + [1.0]
+    w = WORKLOADS["lstm_ptb"].scaled("mid", P=2, steps=2,
+                                     tensors=[Tensor(f"t{i}", (d,)) for i, d in enumerate(sizes)])
+    run_full_compare(sizes, dens, 2, w.lr, 2, synth_grad_fn(w),
+                     expect_fallbacks=lambda fb: fb == 0)
+
+
+def test_eight_cta_cluster_select():
+    # ~57k expected candidates: an 8-CTA cluster
+    sizes = [4_000_037, 3, 129]
+    dens = [0.01, 1.0, 0.5]
+    w = WORKLOADS["lstm_ptb"].scaled("large", P=2, steps=3,
                                      tensors=[Tensor(f"t{i}", (d,)) for i, d in enumerate(sizes)])
     run_full_compare(sizes, dens, 2, w.lr, 3, synth_grad_fn(w),
                      expect_fallbacks=lambda fb: fb == 0)
