@@ -642,18 +642,28 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
       const uint32_t nw = tb - ta;
       // tiles the bulk copies brought: the index of staged entry j of tile q
       // is in the tile's slot j
+      // (eight entries at a time: their index loads in flight together)
+      constexpr uint32_t B = 8;
       for (uint32_t q = tid; q < nw; q += NT) {
         const uint32_t n = __ldg(cnt + ta + q);
         if (n > cap) continue;
         const uint64_t slot = cbase + (uint64_t)(ta + q - ld.tile_begin) * cap;
         const uint32_t b = sh.tpre[q];
-        for (uint32_t j = 0; j < n; ++j) {
-          const uint32_t m = __float_as_uint(stage_val[b + j]);
-          if (m == 0xFFFFFFFFu) continue;
-          const uint32_t x = __ldg(cand_idx + slot + j);
-          out_idx[ob + m] = x;
-          if (x - ld.off < ld.d) r[x] = 0.0f;  // an emitted index lies in the layer
-          else atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
+        for (uint32_t j0 = 0; j0 < n; j0 += B) {
+          uint32_t m[B], x[B];
+#pragma unroll
+          for (uint32_t u = 0; u < B; ++u)
+            m[u] = j0 + u < n ? __float_as_uint(stage_val[b + j0 + u]) : 0xFFFFFFFFu;
+#pragma unroll
+          for (uint32_t u = 0; u < B; ++u)
+            x[u] = m[u] != 0xFFFFFFFFu ? __ldg(cand_idx + slot + j0 + u) : 0u;
+#pragma unroll
+          for (uint32_t u = 0; u < B; ++u) {
+            if (m[u] == 0xFFFFFFFFu) continue;
+            out_idx[ob + m[u]] = x[u];
+            if (x[u] - ld.off < ld.d) r[x[u]] = 0.0f;  // an emitted index lies in the layer
+            else atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
+          }
         }
       }
       if (ovf) {
