@@ -601,6 +601,17 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
       atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
     }
   };
+  // values-only staging: one bit per staged entry marks the picks for the
+  // index pass (in this CTA's histogram, free once the search is done: no
+  // peer reads it)
+  uint32_t* const picked = hist;
+  if constexpr (VO) {
+    if (staged) {
+      for (uint32_t w = tid; w < (my_pad + 31) / 32; w += NT) picked[w] = 0u;
+      __syncthreads();
+    }
+  }
+  bool restage_timeout = false;
   if (staged) {
     // warp rounds of 32 consecutive positions: ballots give each lane its
     // strict and tie ranks, so the pick-list stores are coalesced and no
@@ -623,6 +634,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
           if (pos < ld.k) {
             out_val[ob + pos] = val;
             mark = pos;
+            atomicOr(&picked[i >> 5], 1u << (i & 31));
           } else {
             atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
           }
@@ -638,8 +650,55 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
     }
     if constexpr (VO) {
       // the picks' indices, tile by tile (the walks cross the warps' ranges)
+      fence_proxy_async_shared();  // the marks above, before the copies below
       __syncthreads();
       const uint32_t nw = tb - ta;
+      if (!ovf) {
+        // every run came from the slots: copy the runs' indices over the
+        // stage (the picks' positions follow from the bits), then write each
+        // warp's picks in index order, coalesced, and zero their residuals
+        if (tid == 0) mbar_arrive_expect_tx(&stage_bar, my_pad * 4u);
+        __syncthreads();
+        for (uint32_t q = tid; q < nw; q += NT) {
+          const uint32_t n = sh.tpre[q + 1] - sh.tpre[q];
+          if (n == 0) continue;
+          const uint64_t slot = cbase + (uint64_t)(ta + q - ld.tile_begin) * cap;
+          bulk_load(stage_val + sh.tpre[q], cand_idx + slot, n * 4u, &stage_bar);
+        }
+        const bool ok = mbar_wait_bounded(&stage_bar, 1, kSelectSpinLimit);
+        restage_timeout = __syncthreads_or(!ok);
+        if (restage_timeout && tid == 0) atomicOr(dp.status + kStatusFlags, LAGS_FLAG_TIMEOUT);
+        // picks before this warp's range: strict ones plus the first `need` ties
+        uint32_t pos = a_run + (warp_ex >> 16) + min(need, b_run + (warp_ex & 0xFFFFu));
+        for (uint32_t b0 = wb; b0 < we; b0 += 32) {
+          const uint32_t i = b0 + lane;
+          const bool pk = i < we && ((picked[i >> 5] >> (i & 31)) & 1u);
+          const unsigned mp = __ballot_sync(kFull, pk);
+          if (pk) {
+            const uint32_t at_ = pos + __popc(mp & lanes_below);
+            uint32_t x;
+            if (!restage_timeout) {
+              x = __float_as_uint(stage_val[i]);
+            } else {
+              // the copies did not complete: the slot from the tile prefix
+              uint32_t lo_q = 0, hi_q = nw - 1;
+              while (lo_q < hi_q) {
+                const uint32_t mid = (lo_q + hi_q + 1) >> 1;
+                if (sh.tpre[mid] <= i) lo_q = mid; else hi_q = mid - 1;
+              }
+              x = __ldg(cand_idx + cbase + (uint64_t)(ta + lo_q - ld.tile_begin) * cap +
+                        (i - sh.tpre[lo_q]));
+            }
+            if (at_ < ld.k && x - ld.off < ld.d) {
+              out_idx[ob + at_] = x;
+              r[x] = 0.0f;
+            } else {
+              atomicOr(dp.status + kStatusFlags, LAGS_FLAG_INTERNAL);
+            }
+          }
+          pos += __popc(mp);
+        }
+      } else {
       // tiles the bulk copies brought: the index of staged entry j of tile q
       // is in the tile's slot j
       // (eight entries at a time: their index loads in flight together)
@@ -698,6 +757,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
           }
         }
       }
+      }  // (overflowed share)
     } else {
       __syncwarp();
       for (uint32_t i = wb + lane; i < we; i += 32) {
@@ -760,6 +820,8 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   }
   if (stage_timeout && tid == 0)  // give copies still in flight a bounded chance to land
     mbar_wait_bounded(&stage_bar, 0, kSelectSpinLimit);
+  if (restage_timeout && tid == 0)
+    mbar_wait_bounded(&stage_bar, 1, kSelectSpinLimit);
   C::wait();  // no CTA leaves while another may still read its shared memory
 }
 
