@@ -41,9 +41,9 @@ DEFAULT_CONFIG = "gpt_1_3b"
 # workload's, scaled by worker-elements: the passes stream over the elements,
 # so their traffic grows in proportion.
 EF_TRAFFIC = {  # k_ef_capture
-    "vgg16": (1_885_872_128 + 895_902_208, 235_517_088),
+    "vgg16": (1_885_810_432 + 895_068_928, 235_517_088),
     # one transformer block (tensors 1..8) of the 1.3B model, 8 workers
-    "gpt_1_3b[1:9]": (3_224_683_776 + 1_567_508_736, 402_718_720),
+    "gpt_1_3b[1:9]": (3_225_167_616 + 1_567_329_024, 402_718_720),
 }
 DENSE_TRAFFIC = {  # k_dense_sum
     "vgg16": (942_088_192 + 12_455_680, 235_517_088),
