@@ -301,6 +301,18 @@ LAGS_API lags_status lags_plan_set_events(lags_plan* plan, void* before, void* a
 LAGS_API lags_status lags_plan_set_stage_wait_limit(lags_plan* plan, uint32_t polls);
 
 /*
+ * lags_plan_set_index_wait_limit - failure-injection knob for the second
+ * bounded wait of the selections that stage candidate values only: after the
+ * emission they bulk-copy the candidate indices over their stage and poll
+ * that copy's completion at most `polls` times (default
+ * LAGS_STAGE_WAIT_POLLS).  On timeout they set LAGS_FLAG_TIMEOUT and read
+ * each pick's index from global memory instead (the same index, so every
+ * output stays exact), then still wait (up to the default limit) for the
+ * copies before they exit.  Takes effect from the next lags_sparsify.
+ */
+LAGS_API lags_status lags_plan_set_index_wait_limit(lags_plan* plan, uint32_t polls);
+
+/*
  * lags_adaptive_densities - per-layer densities from each layer's
  * communication-to-computation ratio ("Layer-wise Adaptive Gradient
  * Sparsification ..." review, "proposed method": each layer's sparsification

@@ -14,7 +14,8 @@ from ._binding import (  # noqa: F401
     lags_dense_finish, lags_dense_sum, lags_error_string, lags_merge_layers,
     lags_plan_aggregate_workspace_bytes, lags_plan_create, lags_plan_create_range,
     lags_plan_destroy, lags_plan_info, lags_plan_kernel_launches, lags_plan_layer,
-    lags_plan_set_events, lags_plan_set_stage_wait_limit, lags_plan_set_workspace,
+    lags_plan_set_events, lags_plan_set_index_wait_limit, lags_plan_set_stage_wait_limit,
+    lags_plan_set_workspace,
     lags_sparsify, lags_sparsify_static, lags_static_status_poll, lags_status_poll, library,
 )
 

@@ -33,7 +33,8 @@ EXPORTED = ("lags_plan_create", "lags_plan_destroy", "lags_plan_info", "lags_pla
             "lags_aggregate_apply", "lags_plan_kernel_launches", "lags_adaptive_densities",
             "lags_plan_create_range", "lags_merge_layers", "lags_dense_sum",
             "lags_dense_finish", "lags_plan_aggregate_workspace_bytes",
-            "lags_plan_set_stage_wait_limit", "lags_static_status_poll", "lags_error_string")
+            "lags_plan_set_stage_wait_limit", "lags_plan_set_index_wait_limit",
+            "lags_static_status_poll", "lags_error_string")
 
 
 class LagsError(RuntimeError):
@@ -88,6 +89,7 @@ def _load() -> ctypes.CDLL:
                                             ctypes.POINTER(ctypes.c_uint32), vp]
     lib.lags_plan_aggregate_workspace_bytes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t)]
     lib.lags_plan_set_stage_wait_limit.argtypes = [vp, ctypes.c_uint32]
+    lib.lags_plan_set_index_wait_limit.argtypes = [vp, ctypes.c_uint32]
     lib.lags_error_string.argtypes = [st]
     lib.lags_error_string.restype = ctypes.c_char_p
     for name in EXPORTED[:-1]:
@@ -165,6 +167,11 @@ def lags_plan_aggregate_workspace_bytes(plan) -> int:
 def lags_plan_set_stage_wait_limit(plan, polls: int) -> None:
     _check(_LIB.lags_plan_set_stage_wait_limit(plan, int(polls)),
            "lags_plan_set_stage_wait_limit")
+
+
+def lags_plan_set_index_wait_limit(plan, polls: int) -> None:
+    _check(_LIB.lags_plan_set_index_wait_limit(plan, int(polls)),
+           "lags_plan_set_index_wait_limit")
 
 
 def lags_plan_layer(plan, l: int) -> Tuple[int, int, int]:

@@ -665,7 +665,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
           const uint64_t slot = cbase + (uint64_t)(ta + q - ld.tile_begin) * cap;
           bulk_load(stage_val + sh.tpre[q], cand_idx + slot, n * 4u, &stage_bar);
         }
-        const bool ok = mbar_wait_bounded(&stage_bar, 1, kSelectSpinLimit);
+        const bool ok = mbar_wait_bounded(&stage_bar, 1, dp.index_spin);
         restage_timeout = __syncthreads_or(!ok);
         if (restage_timeout && tid == 0) atomicOr(dp.status + kStatusFlags, LAGS_FLAG_TIMEOUT);
         // picks before this warp's range: strict ones plus the first `need` ties

@@ -542,6 +542,13 @@ lags_status lags_plan_set_stage_wait_limit(lags_plan* plan, uint32_t polls) {
   return LAGS_OK;
 }
 
+lags_status lags_plan_set_index_wait_limit(lags_plan* plan, uint32_t polls) {
+  if (!plan) return LAGS_ERR_INVALID_ARG;
+  plan->index_spin = polls;
+  plan->dp.index_spin = polls;
+  return LAGS_OK;
+}
+
 lags_status lags_status_poll(lags_plan* plan, uint32_t* flags, uint32_t* exact_fallbacks,
                              void* stream) {
   if (!plan) return LAGS_ERR_INVALID_ARG;

@@ -125,6 +125,7 @@ struct DevPlan {
   uint64_t C;  // candidate slots per worker
   uint32_t stage_small, stage_large, stage_huge, stage_mid;  // select staging per launch
   uint32_t stage_spin;    // polls of the select's first staging wait before it gives up
+  uint32_t index_spin;    // polls of the values-only select's index-copy wait
 };
 
 // Launchers (each returns the launch's cudaError_t).

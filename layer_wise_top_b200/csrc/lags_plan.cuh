@@ -31,6 +31,7 @@ struct lags_plan {
   bool ws_full = false;  // the bound workspace also serves lags_sparsify
   int device = -1;
   uint32_t stage_spin = lags::kSelectSpinLimit;  // polls of the select's first staging wait
+  uint32_t index_spin = lags::kSelectSpinLimit;  // polls of the values-only index-copy wait
   cudaEvent_t ev_before = nullptr, ev_after = nullptr;
   uint32_t stage_small = 0, stage_large = 0, stage_huge = 0, stage_mid = 0;  // select staging per launch
   lags::DevPlan dp{};  // device view once a workspace is bound
@@ -77,6 +78,7 @@ inline void bind_dev_plan(const lags_plan* plan, char* base, lags::DevPlan* out)
   dp.stage_mid = plan->stage_mid;
   dp.stage_huge = plan->stage_huge;
   dp.stage_spin = plan->stage_spin;
+  dp.index_spin = plan->index_spin;
 }
 
 // The status a poll returns for the flags it read: a timeout first (its picks

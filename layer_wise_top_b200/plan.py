@@ -140,6 +140,11 @@ class Plan:
         """Failure-injection knob: polls of the selection's first staging wait."""
         B.lags_plan_set_stage_wait_limit(self.handle, polls)
 
+    def set_index_wait_limit(self, polls: int) -> None:
+        """Failure-injection knob: polls of the values-only selection's wait for
+        its index copies."""
+        B.lags_plan_set_index_wait_limit(self.handle, polls)
+
 
 class DenseKernels:
     """The dense S-SGD baseline's two kernels on torch tensors (no plan)."""

@@ -21,7 +21,7 @@ def declared():
 
 def test_exports_every_declared_symbol():
     names = declared()
-    assert len(names) == 22, names
+    assert len(names) == 23, names
     lib = ctypes.CDLL(L.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
@@ -65,6 +65,17 @@ def test_aggregate_only_workspace_is_a_smaller_prefix(name):
         assert agg >= 16 * tiles + 4 * w.P * tiles
         if name != "resnet20":
             assert agg < full / 4
+    finally:
+        L.lags_plan_destroy(h)
+
+
+def test_index_wait_limit_knob_validates():
+    with pytest.raises(L.LagsError):
+        L.lags_plan_set_index_wait_limit(None, 0)
+    h = L.lags_plan_create([100, 7], [0.1, 1.0], 2)
+    try:
+        L.lags_plan_set_index_wait_limit(h, 0)
+        L.lags_plan_set_index_wait_limit(h, L.LAGS_STAGE_WAIT_POLLS)
     finally:
         L.lags_plan_destroy(h)
 

@@ -19,14 +19,17 @@ def _u32(t):
     return t.detach().cpu().numpy().view(np.uint32)
 
 
-def _run_against_oracle(sizes, dens, P, lr, steps, grad_fn, wait_limit):
-    """Steps with the given staging-wait limit; every output compared with
-    the oracle.  Returns the (status, flags, fallbacks) of each step's poll."""
+def _run_against_oracle(sizes, dens, P, lr, steps, grad_fn, wait_limit, index_limit=None):
+    """Steps with the given staging-wait limit (and index-copy wait limit);
+    every output compared with the oracle.  Returns the (status, flags,
+    fallbacks) of each step's poll."""
     import torch
     import layer_wise_top_b200 as L
     from gpu_harness import GpuRun
     run = GpuRun(sizes, dens, P, lr)
     run.plan.set_stage_wait_limit(wait_limit)
+    if index_limit is not None:
+        run.plan.set_index_wait_limit(index_limit)
     hist = lo.run_workload(sizes, dens, P, lr, steps, grad_fn)
     polls = []
     for s in range(steps):
@@ -99,6 +102,22 @@ def test_timeout_with_overflowed_tile_walks_acc_exactly():
     import layer_wise_top_b200 as L
     sizes, dens, fn = _crowded_tile_case()
     polls = _run_against_oracle(sizes, dens, 2, 1.0, 3, fn, wait_limit=0)
+    for status, flags, fb in polls:
+        assert status == L.LAGS_ERR_TIMEOUT and flags == L.LAGS_FLAG_TIMEOUT and fb == 0
+
+
+def test_index_copy_wait_timeout_reads_slots_exactly():
+    # 4-CTA values-only selects (19 layers x 2 workers fill the GPU) whose
+    # wait for the index copies gives up at once: each pick's index comes from
+    # its candidate slot instead, and the poll reports the timeout
+    import layer_wise_top_b200 as L
+    from gpu_harness import synth_grad_fn
+    sizes = [400_003 + 977 * i for i in range(19)] + [3]
+    dens = [0.05] * 19 + [1.0]
+    w = WORKLOADS["lstm_ptb"].scaled("mid", P=2, steps=2,
+                                     tensors=[Tensor(f"t{i}", (d,)) for i, d in enumerate(sizes)])
+    polls = _run_against_oracle(sizes, dens, 2, w.lr, 2, synth_grad_fn(w),
+                                wait_limit=L.LAGS_STAGE_WAIT_POLLS, index_limit=0)
     for status, flags, fb in polls:
         assert status == L.LAGS_ERR_TIMEOUT and flags == L.LAGS_FLAG_TIMEOUT and fb == 0
 
