@@ -8,14 +8,15 @@
 // (held in the residual buffer after the fused pass).  Either way the result
 // is the exact top-k of the layer.
 //
-// CL is 1, 4, 8, or 16. 4-CTA clusters stage candidate values only (4 bytes
-// instead of 8; the picks' indices are read back from the candidate slots
-// after the emission), which keeps two CTAs per SM for layers whose
-// candidates would otherwise need 8-CTA clusters.  16 is used for layers whose
-// candidates need more shared memory than 8 CTAs hold, and it is a
-// non-portable cluster size used only where the occupancy query says it fits.  Shares are equal tile ranges; a
-// crowded clustered segment (overflow that equal shares cannot stage) is
-// split again into shares of equal candidate counts.
+// CL is 1, 4, 8, or 16.  4-CTA clusters stage candidate values only (4 bytes
+// instead of 8), which keeps two CTAs per SM for layers whose candidates
+// would otherwise need 8-CTA clusters; after the emission they copy the
+// candidates' indices over the stage for the index write-back.  16 is used
+// for layers whose candidates need more shared memory than 8 CTAs hold, and
+// it is a non-portable cluster size used only where the occupancy query says
+// it fits.  Shares are equal tile ranges; a crowded clustered segment
+// (overflow that equal shares cannot stage) is split again into shares of
+// equal candidate counts.
 //
 // A CTA whose candidates fit in shared memory stages them there, with plain
 // bulk copies (cp.async.bulk, one per tile and array, completing on one
@@ -28,15 +29,15 @@
 //     __match_any_sync on the exhaustive path), the CTAs add their nonzero
 //     bins into CTA 0's histogram through distributed shared memory, and every
 //     CTA reads the merged histogram into registers to pick the bin holding
-//     the k-th largest key.  It stops early
-//     once a whole bin is taken.  The result is a key prefix (shift s, value
-//     T): entries with key>>s > T are picks, entries with key>>s == T are ties
-//     of which the `need` lowest indices are picks ("lower index wins").
+//     the k-th largest key.  It stops early once a whole bin is taken.  The
+//     result is a key prefix (shift s, value T): entries with key>>s > T are
+//     picks, entries with key>>s == T are ties of which the `need` lowest
+//     indices are picks ("lower index wins").
 //  2. each CTA counts its strict picks and ties, the counts are exchanged, and
 //     each CTA emits its picks in index order at
 //         pos = strict_before + min(need, ties_before)
-//     with block-wide scans, writing (index, acc) to the pick list and +0 over
-//     the picked residuals.
+//     (staged shares: warp ballots; otherwise block-wide scans), writing
+//     (index, acc) to the pick list and +0 over the picked residuals.
 // No CTA ever waits on another outside the hardware cluster barrier.
 #include <cooperative_groups.h>
 
