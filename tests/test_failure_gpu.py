@@ -96,6 +96,36 @@ def test_crowded_tile_recompaction_exact():
         assert fb == 0  # staged and recompacted, not the exhaustive path
 
 
+def test_values_only_select_with_recompacted_tiles_exact():
+    # 4-CTA values-only selects (19 layers x 2 workers fill the GPU) where one
+    # tile of every layer holds 6000 values three times larger than the rest:
+    # about 2.2k candidates there, more than the tile's ~1.5k slots, so the
+    # CTA recompacts the tile from its acc and recovers those picks' indices
+    # with a second walk (moderate scaling keeps the sampled threshold below
+    # the k-th largest even when a sample run lands in the crowded tile)
+    import layer_wise_top_b200 as L
+    # (a seed whose sampled thresholds keep the k largest of every segment in
+    # both steps, so every segment takes the staged path checked here)
+    rng = np.random.default_rng(37)
+    sizes = [2_000_003 + 977 * i for i in range(19)] + [3]
+    dens = [0.005] * 19 + [1.0]
+    N = sum(sizes)
+    offs = np.cumsum([0] + sizes[:-1])
+    data = {}
+    for p in range(2):
+        for s in range(2):
+            g = rng.standard_normal(N).astype(F32)
+            for o in offs[:19]:
+                a = int(o) + 91 * 8192 + 700 + 200 * p
+                g[a:a + 6000] *= F32(3.0)
+            data[(p, s)] = g
+    polls = _run_against_oracle(sizes, dens, 2, 1.0, 2, lambda p, s: data[(p, s)],
+                                wait_limit=L.LAGS_STAGE_WAIT_POLLS)
+    for status, flags, fb in polls:
+        assert status == L.LAGS_OK and flags == 0
+        assert fb == 0  # staged and recompacted, not the exhaustive path
+
+
 def test_timeout_with_overflowed_tile_walks_acc_exactly():
     # after a timeout the selecting CTA takes its candidates from acc, so an
     # overflowed tile (only part of its candidates in the slots) is complete
