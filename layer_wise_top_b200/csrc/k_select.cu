@@ -606,6 +606,7 @@ __global__ void __launch_bounds__(NT, CL == 1 ? 4 : 2) k_select(DevPlan dp, Work
   // index pass (in this CTA's histogram, free once the search is done: no
   // peer reads it)
   uint32_t* const picked = hist;
+  static_assert(kSelectStageMaxValues <= kBins * 32, "one bit per staged entry fits the histogram");
   if constexpr (VO) {
     if (staged) {
       for (uint32_t w = tid; w < (my_pad + 31) / 32; w += NT) picked[w] = 0u;
