@@ -172,10 +172,9 @@ __device__ __forceinline__ void agg_write_tile(AggShared& sh, uint32_t start, ui
 }
 
 // One CTA per group of consecutive tiles of one layer (the plan sizes groups
-// to about a thousand expected picks).  The CTA loads the group's pick bounds,
-// stages every worker's picks of the group in shared memory and issues the
-// loads of the weights at the picked positions (consumed only at the end, so
-// their latency hides behind the dense stream).  Then, tile by tile:
+// to about a thousand expected picks).  The CTA loads the group's pick bounds
+// and stages every worker's picks of the group in shared memory.  Then, tile
+// by tile:
 //   1. every pick marks its position in a bitmap; a second bitmap marks the
 //      positions that several workers picked;
 //   2. a position picked by one worker gets fl(+0 + v) in the shared tile
