@@ -13,8 +13,10 @@
 // of the update is composed in shared memory and written once, with aligned
 // 16-byte stores: the kernel streams the dense output at the HBM rate and
 // never writes a position twice.  No atomics, so the result is bit-identical
-// however the grid is scheduled.  With a weights pointer the same kernel also
-// applies the SGD update (weights -= dense) at the picked positions.
+// however the grid is scheduled.  With a weights pointer the SGD update
+// (weights -= dense) follows at the picked positions: the kernel leaves one
+// (position, quotient) record per pick for k_weight_updates, and groups of
+// one high-density tile apply it themselves.
 //
 // Pick lists are read through the read-only path (they are inputs; plain
 // loads would be ordered behind the kernels' own scattered stores).
