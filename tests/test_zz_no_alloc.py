@@ -155,3 +155,27 @@ def test_static_scratch_rejects_large_plan():
         assert e.value.status == L.LAGS_ERR_WORKSPACE
     finally:
         L.lags_plan_destroy(h)
+
+
+_EXIT_WITH_PLAN = """
+import torch
+from layer_wise_top_b200 import Plan
+plan = Plan([1000, 77], [0.01, 1.0], 2)   # still alive when the interpreter exits
+idx, val = plan.empty_picks()
+torch.cuda.synchronize()
+print("EXIT_OK")
+"""
+
+
+def test_plan_alive_at_interpreter_exit_is_destroyed_quietly():
+    """A Plan held by a module global is destroyed during interpreter exit,
+    after the binding's globals may be gone: no exception is reported."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, PYTHONPATH=root + os.pathsep + os.environ.get("PYTHONPATH", ""))
+    out = subprocess.run([sys.executable, "-c", _EXIT_WITH_PLAN], cwd=root, env=env,
+                         capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0 and "EXIT_OK" in out.stdout, out.stdout + out.stderr
+    assert "Exception ignored" not in out.stderr and "Traceback" not in out.stderr, out.stderr
