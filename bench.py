@@ -189,6 +189,14 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def pinned_host_buffers(avail_bytes: int, local_ranks: int, P: int, N: int) -> int:
+    """Pinned host gradient buffers of N fp32 for one rank's e2e leg: as many
+    as its workers (P) while they fit in its share of a quarter of the host's
+    free memory (the node's ranks split it), at least one."""
+    share = int(avail_bytes * 0.25) // max(1, local_ranks)
+    return max(1, min(P, share // (N * 4)))
+
+
 # ------------------------------------------------------------------- oracle timing
 # The CPU oracle (plain numpy: one sort per worker-layer segment, worker-ordered
 # aggregation) timed on the host cores.  Gradients are generated into shared
@@ -659,8 +667,7 @@ def run_ours(args):
         except Exception:  # pragma: no cover
             avail = 64 << 30
         local_ranks = max(1, int(os.environ.get("LOCAL_WORLD_SIZE", str(world))))
-        share = int(avail * 0.25) // local_ranks
-        n_host = max(1, min(P, share // (N * 4)))
+        n_host = pinned_host_buffers(avail, local_ranks, P, N)
         host = [torch.empty(N, dtype=torch.float32, pin_memory=True) for _ in range(n_host)]
         for p in range(n_host):
             host[p].copy_(grads[0][p])

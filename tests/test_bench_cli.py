@@ -77,3 +77,15 @@ def test_tensor_range_rejects_bad_ranges(spec):
     bench, args = _bench(["--config", "resnet20", "--tensors", spec])
     with pytest.raises(SystemExit):
         bench.workload(args)
+
+
+def test_pinned_host_buffers_split_across_local_ranks():
+    import bench
+    N = 1_311_178_752                      # 5.24 GB per buffer
+    gb = 1 << 30
+    assert bench.pinned_host_buffers(190 * gb, 1, 8, N) == min(8, (190 * gb // 4) // (N * 4))
+    # eight ranks on one node: each gets an eighth of the quarter
+    assert bench.pinned_host_buffers(190 * gb, 8, 8, N) == 1
+    # never fewer than one buffer, never more than the workers
+    assert bench.pinned_host_buffers(1 * gb, 8, 8, N) == 1
+    assert bench.pinned_host_buffers(10_000 * gb, 1, 8, N) == 8
